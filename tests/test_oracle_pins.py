@@ -1,0 +1,343 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself --
+printed values, textbook tables, closed forms, library routines, brute force."""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import scipy.optimize
+import scipy.stats
+import torch
+
+from oracle import attention, codebook, encode, opcount, packing, rotation
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    vals = {}
+    for line in open(os.path.join(GOLDEN, name)):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, *v = line.split()
+        vals[k] = v
+    return vals
+
+
+def _params(seed=1, layer=0, head=0):
+    return rotation.init_rotation(seed, layer + 1, head + 1)[layer, head]
+
+
+# ------------------------------------------------------------------ codebook
+def test_lloyd_max_matches_textbook_table():
+    g = _golden("lloyd_max_gaussian_3bit.txt")
+    c, b = codebook.codebook(3)
+    def half_unit(v):  # 0.6 units of the last printed digit (the 1960 table's own rounding slack)
+        return 0.6 * 10.0 ** -(len(v.split(".")[1]) if "." in v else 0)
+
+    for got, printed in [(c[4:], g["output_levels"]), (-c[:4][::-1], g["output_levels"]), (b[3:], g["decision_levels"])]:
+        for x, v in zip(got, printed):
+            assert abs(x - float(v)) <= half_unit(v) + 1e-12, (x, v)
+    assert abs(codebook.gaussian_mse(c, b) - float(g["mse"][0])) <= half_unit(g["mse"][0])
+
+
+def test_lloyd_max_is_a_minimum_of_mse():
+    """An independent optimiser (Nelder-Mead on the MSE functional) finds the same levels."""
+    c, b = codebook.codebook(3)
+
+    def mse(pos):
+        levels = np.sort(np.concatenate([-pos[::-1], pos]))
+        bounds = 0.5 * (levels[1:] + levels[:-1])
+        return codebook.gaussian_mse(levels, bounds)
+
+    res = scipy.optimize.minimize(mse, x0=np.array([0.3, 0.9, 1.5, 2.4]), method="Nelder-Mead",
+                                  options={"xatol": 1e-10, "fatol": 1e-14, "maxiter": 20000})
+    np.testing.assert_allclose(np.sort(res.x), c[4:], atol=1e-5)
+
+
+def test_gaussian_mse_against_monte_carlo():
+    c, b = codebook.codebook(3)
+    x = np.random.default_rng(7).standard_normal(2_000_000)
+    q = c[np.searchsorted(b, x, side="left")]
+    assert abs(np.mean((x - q) ** 2) - codebook.gaussian_mse(c, b)) < 2e-4
+
+
+def test_codebook_scaled_for_dimension():
+    c, b = codebook.codebook(3)
+    ct, bt = codebook.codebook_for_dim(128, 3)
+    np.testing.assert_allclose(ct * math.sqrt(128), c, rtol=0, atol=1e-15)
+    assert b[3] == 0.0 and np.all(np.diff(c) > 0)
+
+
+# ------------------------------------------------------------------ WHT
+def test_hadamard_matches_scipy_and_orthogonality():
+    H = rotation.hadamard_matrix(128)
+    np.testing.assert_array_equal(H, scipy.linalg.hadamard(128))
+    np.testing.assert_array_equal(H @ H.T, 128 * np.eye(128))
+
+
+def test_fast_wht_equals_matrix():
+    x = np.random.default_rng(1).standard_normal((5, 128))
+    H = scipy.linalg.hadamard(128) / math.sqrt(128)
+    np.testing.assert_allclose(rotation.wht(x), x @ H.T, atol=1e-13)
+    np.testing.assert_allclose(rotation.wht(rotation.wht(x)), x, atol=1e-13)
+
+
+# ------------------------------------------------------------------ SO(4) blocks
+def test_hamilton_product_against_textbook_table():
+    """i*j = k, j*k = i, k*i = j, i*i = -1 (Hamilton's rules)."""
+    one, i, j, k = np.eye(4)
+    np.testing.assert_array_equal(rotation.quat_mul(i, j), k)
+    np.testing.assert_array_equal(rotation.quat_mul(j, k), i)
+    np.testing.assert_array_equal(rotation.quat_mul(k, i), j)
+    np.testing.assert_array_equal(rotation.quat_mul(i, i), -one)
+    np.testing.assert_array_equal(rotation.quat_mul(j, i), -k)
+
+
+def test_sandwich_is_rodrigues_rotation():
+    """q v q^-1 with q = (cos t, sin t a) rotates the vector part by 2t about a (Rodrigues)."""
+    rng = np.random.default_rng(3)
+    for _ in range(10):
+        a = rng.standard_normal(3)
+        a /= np.linalg.norm(a)
+        t = rng.uniform(-math.pi, math.pi)
+        v = rng.standard_normal(3)
+        q = np.concatenate([[math.cos(t)], math.sin(t) * a])
+        params = np.zeros((32, 2, 4))
+        params[:] = np.eye(4)[0]
+        params[0, 0] = q
+        params[0, 1] = q
+        z = rotation.so4_apply(np.concatenate([[0.0], v, np.zeros(124)]), params)
+        th = 2 * t
+        rod = v * math.cos(th) + np.cross(a, v) * math.sin(th) + a * np.dot(a, v) * (1 - math.cos(th))
+        np.testing.assert_allclose(z[1:4], rod, atol=1e-13)
+        assert abs(z[0]) < 1e-13
+
+
+def test_blocks_are_so4_and_match_left_right_matrices():
+    p = rotation.unit_params(_params())
+    mats = rotation.block_matrices(p)
+
+    def Lmat(q):  # left multiplication by q, explicit
+        w, x, y, z = q
+        return np.array([[w, -x, -y, -z], [x, w, -z, y], [y, z, w, -x], [z, -y, x, w]])
+
+    def Rmat(q):  # right multiplication by q, explicit
+        w, x, y, z = q
+        return np.array([[w, -x, -y, -z], [x, w, z, -y], [y, -z, w, x], [z, y, -x, w]])
+
+    for kk, m in enumerate(mats):
+        qL, qR = p[kk]
+        qRc = qR * np.array([1, -1, -1, -1])
+        np.testing.assert_allclose(m, Lmat(qL) @ Rmat(qRc), atol=1e-14)
+        np.testing.assert_allclose(m.T @ m, np.eye(4), atol=1e-14)
+        assert abs(np.linalg.det(m) - 1.0) < 1e-13
+        # left and right isoclinic factors commute
+        np.testing.assert_allclose(Lmat(qL) @ Rmat(qRc), Rmat(qRc) @ Lmat(qL), atol=1e-14)
+
+
+def test_round_trip_and_explicit_matrix():
+    p = _params(1, 3, 2)
+    x = np.random.default_rng(5).standard_normal((7, 128))
+    R = rotation.rotation_matrix(p)
+    np.testing.assert_allclose(R @ R.T, np.eye(128), atol=1e-13)
+    np.testing.assert_allclose(rotation.rotate(x, p), x @ R.T, atol=1e-13)
+    assert np.abs(rotation.rotate_inverse(rotation.rotate(x, p), p) - x).max() <= 1e-12
+    # the inverse is the transpose, written out
+    np.testing.assert_allclose(rotation.rotate_inverse(x, p), x @ R, atol=1e-13)
+
+
+def test_params_unit_deterministic_and_spread():
+    P = rotation.init_rotation(1, 2, 3)
+    assert P.shape == (2, 3, 32, 2, 4) and P.dtype == np.float32
+    n = np.linalg.norm(P.astype(np.float64), axis=-1)
+    assert np.abs(n - 1).max() < 3e-7
+    np.testing.assert_array_equal(P, rotation.init_rotation(1, 2, 3))
+    assert not np.array_equal(P, rotation.init_rotation(2, 2, 3))
+    # Haar measure on S^3: each coordinate has mean 0 and second moment 1/4
+    Q = rotation.init_rotation(9, 8, 8).reshape(-1, 4).astype(np.float64)
+    assert np.abs(Q.mean(0)).max() < 0.03
+    assert np.abs((Q ** 2).mean(0) - 0.25).max() < 0.02
+
+
+def test_rotated_unit_vectors_have_variance_one_over_d():
+    """Coordinates of rotated random unit vectors: mean 0, variance 1/d; near N(0, 1/d)."""
+    p = _params()
+    x = np.random.default_rng(2).standard_normal((4000, 128))
+    x /= np.linalg.norm(x, axis=1, keepdims=True)
+    z = rotation.rotate(x, p)
+    assert abs(z.var() * 128 - 1) < 0.01
+    ks = scipy.stats.kstest(z.ravel() * math.sqrt(128), "norm")
+    assert ks.statistic < 0.01
+
+
+# ------------------------------------------------------------------ op counts
+def test_op_counts_match_the_printed_figures():
+    g = _golden("rotation_op_counts.txt")
+    cnt = opcount.rotation_op_counts(_params())
+    assert cnt["total"] == int(g["total_fma"][0])
+    assert cnt["so4"] == int(g["so4_fma"][0])
+    assert cnt["dense"] == int(g["dense_fma"][0])
+    assert cnt["params"] == int(g["params_per_head"][0])
+    assert cnt["dense_params"] == int(g["dense_params"][0])
+    assert cnt["wht"] == 7 * 128
+
+
+def test_counted_transforms_compute_the_rotation():
+    p = _params()
+    _, y = opcount.count_wht(128)
+    _, z = opcount.count_blocks(p, y)
+    x = np.arange(128, dtype=np.float64)
+    np.testing.assert_allclose(np.array(z), rotation.rotate(x, p) * math.sqrt(128), atol=1e-9)
+
+
+# ------------------------------------------------------------------ encoder
+def test_quantise_tie_rule_and_brute_force():
+    c, b = codebook.codebook(3)
+    for j, bj in enumerate(b):
+        assert encode.quantise(np.array([bj]))[0] == j  # a boundary goes to the lower cell
+    u = np.random.default_rng(4).standard_normal(100000) * 1.3
+    np.testing.assert_array_equal(encode.quantise(u), encode.nearest_centroid(u))
+
+
+def test_encode_constructed_centroid_vectors():
+    """x = n R^T c~[k*] (rounded to fp16) must encode to k* with norm ~ n ||c~[k*]||.
+
+    The encoder rescales to unit length, so u = f c[k*] with f = sqrt(d)/||c[k*]||; the
+    codes are preserved while f keeps every level inside its cell (0.82 < f < 1.29), which
+    holds when k* is drawn with the Gaussian cell probabilities."""
+    p = _params(1, 0, 0)
+    c, b = codebook.codebook(3)
+    ct, _ = codebook.codebook_for_dim(128)
+    e_ = np.concatenate([[-np.inf], b, [np.inf]])
+    mass = scipy.stats.norm.cdf(e_[1:]) - scipy.stats.norm.cdf(e_[:-1])
+    rng = np.random.default_rng(11)
+    for _ in range(20):
+        kstar = rng.choice(8, size=128, p=mass / mass.sum())
+        f = math.sqrt(128) / np.linalg.norm(c[kstar])
+        assert 0.85 < f < 1.25
+        n = rng.uniform(0.5, 300.0)
+        x = (n * rotation.rotate_inverse(ct[kstar], p)).astype(np.float16)
+        e = encode.encode(x[None], p)
+        np.testing.assert_array_equal(e["codes"][0], kstar)
+        assert abs(e["norm"][0] - n * np.linalg.norm(ct[kstar])) < 1e-2 * n
+
+
+def test_encode_zero_vector_and_saturation():
+    p = _params()
+    e = encode.encode(np.zeros((1, 128), np.float16), p)
+    assert np.all(e["codes"] == 3) and e["norm16"][0] == 0
+    big = np.full((1, 128), 60000.0, np.float16)
+    e = encode.encode(big, p)
+    assert e["saturated"] == 1 and e["norm16"][0] == np.float16(65504).view(np.uint16)
+
+
+def test_norm_fp16_rounding_is_nearest_even():
+    # 1 + 2^-11 lies halfway between 1 and 1 + 2^-10: ties to even -> 1.0
+    bits, _ = encode.norm_to_fp16_bits(np.array([1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2049.0]))
+    np.testing.assert_array_equal(bits.view(np.float16).astype(np.float64), [1.0, 1.0 + 2 * 2.0 ** -10, 2048.0])
+
+
+# ------------------------------------------------------------------ packing
+def test_chunk_golden_fixtures():
+    g = _golden("packing_chunks.txt")
+    ya = [s % 8 for s in range(32)]
+    assert packing.pack_chunk(ya).hex() == g["chunk_mod8"][0]
+    yb = [7 if s % 4 < 2 else 0 for s in range(32)]
+    assert packing.pack_chunk(yb).hex() == g["chunk_vpair_7_0"][0]
+    assert packing.unpack_chunk(bytes.fromhex(g["chunk_mod8"][0])) == ya
+
+
+def test_pack_round_trip_and_ownership():
+    rng = np.random.default_rng(12)
+    codes = rng.integers(0, 8, (9, 128)).astype(np.uint8)
+    np.testing.assert_array_equal(packing.unpack_k(packing.pack_k(codes)), codes)
+    np.testing.assert_array_equal(packing.unpack_v(packing.pack_v(codes), 9), codes)
+    # a V record's even bytes depend only on the first token, odd bytes only on the second
+    a = rng.integers(0, 8, (2, 128)).astype(np.uint8)
+    b = a.copy()
+    b[1] = rng.integers(0, 8, 128)
+    ra, rb = packing.pack_v(a)[0], packing.pack_v(b)[0]
+    own = packing.v_byte_owner()
+    np.testing.assert_array_equal(ra[own == 0], rb[own == 0])
+    # K record for codes = coordinate mod 8 is four copies of the mod-8 fixture
+    k = packing.pack_k(np.array([np.arange(128) % 8], np.uint8))[0].tobytes().hex()
+    assert k == _golden("packing_chunks.txt")["chunk_mod8"][0] * 4
+    v = packing.pack_v(np.array([np.full(128, 7), np.zeros(128)], np.uint8))[0].tobytes().hex()
+    assert v == "ff00" * 48
+
+
+# ------------------------------------------------------------------ attention
+def _cache(Hkv, T, seed=0):
+    rng = np.random.default_rng(seed)
+    P = rotation.init_rotation(1, 1, Hkv)[0]
+    kc = rng.integers(0, 8, (Hkv, T, 128)).astype(np.uint8)
+    vc = rng.integers(0, 8, (Hkv, T, 128)).astype(np.uint8)
+    kn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 60, (Hkv, T)))
+    vn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 10, (Hkv, T)))
+    return P, kc, kn, vc, vn
+
+
+def test_rotated_equals_dequantised_attention():
+    P, kc, kn, vc, vn = _cache(2, 37)
+    q = np.random.default_rng(1).standard_normal((8, 128))
+    a = attention.attention_rotated(q, kc, kn, vc, vn, P)
+    b = attention.attention_dequant(q, kc, kn, vc, vn, P)
+    assert np.abs(a - b).max() / np.abs(b).max() < 1e-10
+
+
+def test_dequantised_attention_matches_torch_sdpa():
+    P, kc, kn, vc, vn = _cache(2, 29)
+    q = np.random.default_rng(2).standard_normal((6, 128))
+    out = attention.attention_dequant(q, kc, kn, vc, vn, P)
+    for kv in range(2):
+        K = torch.from_numpy(attention.dequantise(kc[kv], kn[kv], P[kv]))
+        V = torch.from_numpy(attention.dequantise(vc[kv], vn[kv], P[kv]))
+        Q = torch.from_numpy(q[3 * kv : 3 * kv + 3])
+        ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None])[0]
+        np.testing.assert_allclose(out[3 * kv : 3 * kv + 3], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    P, kc, kn, vc, vn = _cache(1, 16)
+    q = np.random.default_rng(3).standard_normal((2, 128))
+    V0 = attention.dequantise(vc[0], vn[0], P[0])
+    one = attention.attention_rotated(q, kc[:, :1], kn[:, :1], vc[:, :1], vn[:, :1], P)
+    np.testing.assert_allclose(one, np.repeat(V0[:1], 2, 0), atol=1e-12)
+    zero_q = attention.attention_rotated(np.zeros((1, 128)), kc, kn, vc, vn, P)
+    np.testing.assert_allclose(zero_q[0], V0.mean(0), atol=1e-12)
+    same_k = attention.attention_rotated(q, np.repeat(kc[:, :1], 16, 1), np.repeat(kn[:, :1], 16, 1), vc, vn, P)
+    np.testing.assert_allclose(same_k, np.repeat(V0.mean(0)[None], 2, 0), atol=1e-12)
+    empty = attention.attention_rotated(q, kc[:, :0], kn[:, :0], vc[:, :0], vn[:, :0], P)
+    assert np.all(empty == 0)
+
+
+def test_gqa_head_mapping():
+    P, kc, kn, vc, vn = _cache(2, 10)
+    q = np.random.default_rng(4).standard_normal((4, 128))
+    out = attention.attention_rotated(q, kc, kn, vc, vn, P)
+    swapped = attention.attention_rotated(q[[2, 3, 0, 1]], kc[::-1], kn[::-1], vc[::-1], vn[::-1], P[::-1])
+    np.testing.assert_allclose(out, swapped[[2, 3, 0, 1]], atol=1e-13)
+
+
+def test_planted_mistakes_are_caught():
+    """A dropped inverse rotation or a transposed block must break the pins above."""
+    P, kc, kn, vc, vn = _cache(1, 8)
+    q = np.random.default_rng(5).standard_normal((1, 128))
+    good = attention.attention_dequant(q, kc, kn, vc, vn, P)
+    ct, _ = codebook.codebook_for_dim(128)
+    # mistake 1: accumulate V in the rotated basis and forget the inverse rotation
+    nk = encode.fp16_bits_to_float(kn[0])
+    nv = encode.fp16_bits_to_float(vn[0])
+    s = nk * (ct[kc[0].astype(int)] @ rotation.rotate(q[0], P[0])) / math.sqrt(128)
+    p = np.exp(s - s.max())
+    no_inverse = (p * nv) @ ct[vc[0].astype(int)] / p.sum()
+    assert np.abs(no_inverse - good[0]).max() > 0.1 * np.abs(good).max()
+    # mistake 2: transposed blocks (conj on the wrong side) is not the same rotation
+    Pbad = P.copy()
+    Pbad[..., 0, :], Pbad[..., 1, :] = P[..., 1, :], P[..., 0, :]
+    x = np.random.default_rng(6).standard_normal(128)
+    assert np.abs(rotation.rotate(x, Pbad[0]) - rotation.rotate(x, P[0])).max() > 1e-3
