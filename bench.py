@@ -1,0 +1,440 @@
+"""Benchmark of the packed-3-bit KV path on B200 (one JSON line on rank 0).
+
+Headline workload (qwen30b_32k): one decode step of a Qwen3-30B-A3B-shaped stack -- batch 1,
+32 query / 4 kv heads, d = 128, 48 layers back to back, context 32768.  A step appends the
+new token's K and V to every layer's packed cache (encode) and runs decode attention over
+the 32768 cached tokens of every layer; the 48 layers are replayed as one CUDA graph.
+value = algorithmic packed-KV bytes of the step / step time (GB/s); the step reads 629 MB
+of packed cache, far more than L2, so no flush is needed between steps.
+
+Also reported: the ingest workload (quantise-and-append 32768 tokens x 8 kv heads x 32
+layers of K and V, 16.8 M vectors: encode Mvec/s and GB/s) and the batched serving workload
+(16 paged sequences, contexts in [2048, 32768], 32 layers).
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the headline workload.
+"""
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+BYTES_PER_TOKEN_HEAD = 100  # 48 B K codes + 2 B K norm + 48 B V codes + 2 B V norm
+BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
+HEADLINE = "qwen30b_32k"
+METRIC = "packed-KV decode attention GB/s & % HBM peak at 32K ctx; encode Mvec/s"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of the SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:6]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workloads
+class DecodeStack:
+    """Packed caches of an L-layer stack, filled by the library's own encoder."""
+
+    def __init__(self, B, Hq, Hkv, L, ctx, page_size, device, seed=0, block_table=None, n_pages=None):
+        import torch
+
+        from rotated_bit_kv_iq_b200 import binding as Bd
+        from rotated_bit_kv_iq_b200 import inputs
+
+        self.Bd, self.torch = Bd, torch
+        self.B, self.Hq, self.Hkv, self.L = B, Hq, Hkv, L
+        self.ctx = np.asarray(ctx, dtype=np.int32)
+        self.max_ctx = int(self.ctx.max())
+        self.dev = device
+        n_pages = n_pages if n_pages is not None else B
+        self.cache = Bd.PagedCache(L, Hkv, page_size, n_pages, block_table=block_table, device=device)
+        self.params = torch.from_numpy(Bd.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)).to(device)
+        # prefill: tokens 0..ctx-2 of every sequence and layer, encoded by iq_encode_append
+        pre = self.ctx - 1
+        n_max = int(pre.max())
+        start = torch.zeros(B, dtype=torch.int32, device=device)
+        for l in range(L):
+            k = inputs.kv_tokens_device(seed, l, Hkv, 0, n_max * B, device=device).view(B, n_max, Hkv, 128)
+            v = inputs.kv_tokens_device(seed, l, Hkv, 1, n_max * B, device=device).view(B, n_max, Hkv, 128)
+            Bd.iq_encode_append(self.cache, l, k, v, start, self.params)
+        # the step's inputs: the new token (position ctx-1) and the queries, per layer
+        self.new_pos = torch.from_numpy(pre).to(device)
+        self.ctx_dev = torch.from_numpy(self.ctx).to(device)
+        self.knew = torch.stack([inputs.kv_tokens_device(seed + 1, l, Hkv, 0, B, device=device) for l in range(L)]).view(
+            L, B, 1, Hkv, 128)
+        self.vnew = torch.stack([inputs.kv_tokens_device(seed + 1, l, Hkv, 1, B, device=device) for l in range(L)]).view(
+            L, B, 1, Hkv, 128)
+        self.q = torch.stack([inputs.queries_device(seed, l, B, Hq, device=device) for l in range(L)])
+        self.out = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=device)
+        self.ws = torch.empty(Bd.iq_decode_workspace_size(B, Hq, Hkv, self.max_ctx), dtype=torch.uint8, device=device)
+        torch.cuda.synchronize()
+
+    @property
+    def bytes_per_step(self):
+        return int(self.ctx.sum()) * self.Hkv * self.L * BYTES_PER_TOKEN_HEAD + \
+            self.B * self.Hkv * 2 * self.L * BYTES_PER_VECTOR_ENCODE
+
+    def layer(self, l, stream=None):
+        Bd = self.Bd
+        Bd.iq_encode_append(self.cache, l, self.knew[l], self.vnew[l], self.new_pos, self.params, stream)
+        Bd.iq_decode_attention(self.cache, l, self.q[l], self.ctx_dev, self.max_ctx, self.params, self.out[l], self.ws,
+                               stream)
+
+    def step(self, stream=None):
+        for l in range(self.L):
+            self.layer(l, stream)
+
+    launches_per_layer = 3  # encode + split-K decode + combine
+
+
+def time_graph(stack, steps, warmup, stream):
+    """Replay the whole step as one CUDA graph; device time per step via events."""
+    torch = stack.torch
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            stack.step(stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        stack.step(stream)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps, graph
+
+
+def time_decode_kernel(stack, steps, stream):
+    """Average duration of one decode-attention call (split-K kernel + combine) per layer."""
+    torch = stack.torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(stack.L)]
+    tot, n = 0.0, 0
+    Bd = stack.Bd
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            for l in range(stack.L):
+                evs[l][0].record(stream)
+                Bd.iq_decode_attention(stack.cache, l, stack.q[l], stack.ctx_dev, stack.max_ctx, stack.params,
+                                       stack.out[l], stack.ws, stream)
+                evs[l][1].record(stream)
+            stream.synchronize()
+            for a, b in evs:
+                tot += a.elapsed_time(b)
+                n += 1
+    return tot / n
+
+
+def time_e2e(stack, steps, warmup, stream):
+    """Same step through the public API with host buffers: per layer the new K/V and the
+    queries come from pinned host memory and the attention output goes back to it."""
+    torch = stack.torch
+    hk = stack.knew.cpu().pin_memory()
+    hv = stack.vnew.cpu().pin_memory()
+    hq = stack.q.cpu().pin_memory()
+    ho = torch.empty(stack.out.shape, dtype=torch.float32).pin_memory()
+    dk, dv, dq = torch.empty_like(stack.knew), torch.empty_like(stack.vnew), torch.empty_like(stack.q)
+    Bd = stack.Bd
+
+    def step():
+        for l in range(stack.L):
+            dk[l].copy_(hk[l], non_blocking=True)
+            dv[l].copy_(hv[l], non_blocking=True)
+            dq[l].copy_(hq[l], non_blocking=True)
+            Bd.iq_encode_append(stack.cache, l, dk[l], dv[l], stack.new_pos, stack.params, stream)
+            Bd.iq_decode_attention(stack.cache, l, dq[l], stack.ctx_dev, stack.max_ctx, stack.params, stack.out[l],
+                                   stack.ws, stream)
+            ho[l].copy_(stack.out[l], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            step()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
+    d2h = ho.numel() * 4
+    return ms, h2d, d2h
+
+
+def bench_encode(steps, warmup, device, stream):
+    """Ingest workload: 32 layers x (32768 tokens x 8 kv heads) of K and V per step."""
+    import torch
+
+    from rotated_bit_kv_iq_b200 import binding as Bd
+    from rotated_bit_kv_iq_b200 import inputs
+
+    L, Hkv, T = 32, 8, 32768
+    cache = Bd.PagedCache(L, Hkv, T, 1, device=device)
+    params = torch.from_numpy(Bd.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)).to(device)
+    K = [inputs.kv_tokens_device(0, l, Hkv, 0, T, heavy_frac=0.01, device=device).view(1, T, Hkv, 128) for l in range(L)]
+    V = [inputs.kv_tokens_device(0, l, Hkv, 1, T, heavy_frac=0.01, device=device).view(1, T, Hkv, 128) for l in range(L)]
+    start = torch.zeros(1, dtype=torch.int32, device=device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            for l in range(L):
+                Bd.iq_encode_append(cache, l, K[l], V[l], start, params, stream)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            for l in range(L):
+                Bd.iq_encode_append(cache, l, K[l], V[l], start, params, stream)
+        e1.record(stream)
+        e1.synchronize()
+        step_ms = e0.elapsed_time(e1) / steps
+        tot = 0.0
+        for _ in range(steps):
+            for l in range(L):
+                evs[l][0].record(stream)
+                Bd.iq_encode_append(cache, l, K[l], V[l], start, params, stream)
+                evs[l][1].record(stream)
+            stream.synchronize()
+            tot += sum(a.elapsed_time(b) for a, b in evs)
+    launch_ms = tot / (steps * L)
+    vecs = L * T * Hkv * 2
+    return {"vectors_per_step": vecs, "ms_per_step": step_ms, "launch_ms": launch_ms,
+            "bytes_per_launch": T * Hkv * 2 * BYTES_PER_VECTOR_ENCODE}
+
+
+# ------------------------------------------------------------------ oracle baseline
+def oracle_decode_sample(seconds=12.0):
+    """fp64 oracle decode attention on slices of the headline workload (one kv head, 8 query
+    heads, 32768 tokens per slice) until about `seconds` of CPU time; returns GB/s."""
+    from oracle import attention, encode
+    from rotated_bit_kv_iq_b200 import binding as Bd
+    from rotated_bit_kv_iq_b200 import inputs
+
+    T, G = 32768, 8
+    P = Bd.iq_init_rotation(inputs.ROTATION_SEED, 1, 4)
+    slices = []
+    for h in range(2):  # encode outside the timed part
+        ek = encode.encode(inputs.kv_tokens(0, 0, h, 0, 0, T), P[0, h])
+        ev = encode.encode(inputs.kv_tokens(0, 0, h, 1, 0, T), P[0, h])
+        slices.append((h, ek, ev))
+    q = inputs.queries(0, 0, 1, 32)[0].astype(np.float64)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        h, ek, ev = slices[n % len(slices)]
+        attention.attention_rotated(q[h * G:(h + 1) * G], ek["codes"][None], ek["norm16"][None], ev["codes"][None],
+                                    ev["norm16"][None], P[0, h:h + 1])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    gbs = n * T * BYTES_PER_TOKEN_HEAD / el / 1e9
+    return gbs, n, el
+
+
+def reference_arm(args):
+    """--impl reference: the oracle on bounded samples of the headline workload."""
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        gbs, n, el = oracle_decode_sample(seconds=2.0)
+        if i >= args.warmup:
+            per_step.append((gbs, el))
+    gbs = float(np.mean([g for g, _ in per_step]))
+    sample = "fp64 oracle decode attention, 1 kv head x 8 q heads x 32768 tokens per slice, repeated ~2 s per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([e for _, e in per_step]) * 1e3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": HEADLINE + " (oracle sample)"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="headline workload only")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from rotated_bit_kv_iq_b200 import build
+
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from rotated_bit_kv_iq_b200 import binding as Bd
+    from rotated_bit_kv_iq_b200 import inputs
+
+    Bd.lib()
+    stream = torch.cuda.Stream(device=dev)
+    cfg = inputs.CONFIGS[HEADLINE]
+    stack = DecodeStack(cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["n_layers"], [cfg["ctx"]],
+                        cfg["page_size"], dev, seed=rank)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    barrier()
+    with ClockSampler(local) as clk:
+        ms, graph = time_graph(stack, args.steps, args.warmup, stream)
+    barrier()
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * stack.bytes_per_step / (ms * 1e-3) / 1e9
+
+    kern_ms = time_decode_kernel(stack, max(2, args.steps // 2), stream)
+    layer_bytes = int(stack.ctx.sum()) * stack.Hkv * BYTES_PER_TOKEN_HEAD
+    peak, peak_kind = _peaks()
+    achieved = layer_bytes / (kern_ms * 1e-3) / 1e9
+    e2e_ms, h2d, d2h = time_e2e(stack, args.steps, args.warmup, stream)
+    del graph
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 tensor-core inputs, f32 accumulate, 3-bit codes", "data": "synthetic",
+        "config": {"workload": "qwen30b_32k: decode step (append + attend) B=1, 32 q / 4 kv heads, d=128, "
+                               "48 layers, ctx 32768, packed 3-bit cache", "l2": "inputs larger than L2 (629 MB/step)",
+                   "graph": "48-layer step replayed as one CUDA graph", "bytes_per_step": stack.bytes_per_step},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "decode attention (split-K + combine) per layer",
+                     "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
+        "e2e": {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": stack.L * DecodeStack.launches_per_layer * args.steps,
+        "clocks": clk.summary(),
+    }
+    del stack
+    torch.cuda.empty_cache()
+
+    if not args.no_extras:
+        enc = bench_encode(args.steps, args.warmup, dev, stream)
+        mvec = world * enc["vectors_per_step"] / (enc["ms_per_step"] * 1e-3) / 1e6
+        enc_ach = enc["bytes_per_launch"] / (enc["launch_ms"] * 1e-3) / 1e9
+        result["encode"] = {
+            "workload": "ingest_32k: 32768 tokens x 8 kv heads x 32 layers of K and V (16.8 M vectors), 1% Student-t",
+            "value": mvec, "unit": "Mvec/s", "GBps": mvec * 1e6 * BYTES_PER_VECTOR_ENCODE / 1e9,
+            "ms_per_step": enc["ms_per_step"],
+            "roofline": {"bound": "hbm", "achieved": enc_ach, "peak": peak, "unit": "GB/s", "frac": enc_ach / peak,
+                         "traffic": None, "kernel": "encode (one layer, K and V)", "peak_kind": peak_kind},
+        }
+        result["gpu_launches"] += 32 * args.steps
+        torch.cuda.empty_cache()
+
+    if rank == 0 and world == 1:
+        gbs, n, el = oracle_decode_sample(args.cpu_seconds)
+        result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                  "sample": f"{n} x (1 kv head, 8 q heads, 32768 tokens) decode slices in {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

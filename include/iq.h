@@ -1,0 +1,166 @@
+/*
+ * iq.h -- C ABI of the IsoQuant packed-3-bit KV cache library (libiq.so, sm_100a).
+ *
+ * What the library computes (sources are web pages, cited by title and section):
+ *   - "RotaryQuant" write-up, rebasdaily.com 2026-08-14, section
+ *     "妙处不只是压缩，而是不再展开": KV vectors are mixed by a Walsh-Hadamard
+ *     transform and block-diagonal SO(4) rotations, scalar-quantised to 3 bits, and
+ *     attention runs directly on the packed tensors (scores, softmax, value
+ *     accumulation, one inverse rotation) without rebuilding full-precision K/V.
+ *   - RotaryQuant abstract, arXiv 2608.08081 (arxivdaily entry): WHT followed by
+ *     block-diagonal SO(4), 256 parameters per head, 3-bit scalar quantisation.
+ *   - "压缩与速度的博弈——TurboQuant 和 RotorQuant 的真相" (zhichai.net), sections
+ *     "Beta 分布的魔力" (rotated unit-vector coordinates ~ N(0, 1/d)) and
+ *     "Lloyd-Max 最优量化" (the optimal scalar quantiser, applied by lookup).
+ *   - "RotorQuant：LLM KV 缓存压缩的“几何革命”" (sd114.wiki), section
+ *     "3. V 缓存的逆旋转修复": values must be rotated back with the inverse rotation.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev / all tensors are DEVICE memory owned by the caller; the
+ *     library never allocates, frees or retains them.  Host pointers are marked.
+ *   - Calls are asynchronous on the given CUDA stream (NULL = legacy default stream);
+ *     argument errors are detected on the host and returned before any launch.
+ *   - Launch failures return IQ_ERR_CUDA (the CUDA error is left for the caller to
+ *     read with cudaGetLastError / cudaPeekAtLastError).
+ *   - Data-dependent errors found on the device (a position outside a sequence's
+ *     pages, a block-table entry outside the pool, a context length outside
+ *     [0, max_ctx]) never cause an out-of-range access: the offending token or
+ *     sequence is skipped and an IQ_DEVERR_* bit is OR-ed into cache->status_dev
+ *     when that pointer is non-NULL.
+ *   - No C++ exception crosses this interface.
+ *   - head_dim is 128; every device pointer must be 16-byte aligned (workspace 256).
+ *
+ * Cache layout (one pool per layer stacked along the first axis):
+ *   k_codes  [L][n_pages][Hkv][page_size]   x 48-byte K records
+ *   v_codes  [L][n_pages][Hkv][page_size/2] x 96-byte V records (token pairs)
+ *   k_norms, v_norms [L][n_pages][Hkv][page_size] binary16 norms
+ *   Token t of sequence b lives on page
+ *       block_table_dev[b * max_pages_per_seq + t / page_size]   (paged), or
+ *       b                                                         (block_table_dev == NULL)
+ *   at slot t % page_size.  page_size is a positive multiple of 16.
+ *
+ * Record formats (this library's own; the pages fix none):
+ *   code k in 0..7 = index of the ascending Lloyd-Max centroid of N(0,1):
+ *       k = #{ j : u > b_j },  u = sqrt(128) * (R x / ||x||),  R = S * H/sqrt(128)
+ *   32-code chunk = 12 bytes = little-endian uint32 W0,W1,W2; for j in 0..7:
+ *       bits [4j,4j+3) of Ww = code of slot 8w+j; bit 4j+3 of Ww = bit w of slot 24+j
+ *   K record (per token): chunk c = 0..3, slot s -> coordinate 32c+s.
+ *   V record (per token pair 2p,2p+1): chunk g = 0..7, slot s -> token 2p+(s%4>=2),
+ *       coordinate 16g + 2*(s/4) + (s%2); even bytes belong to token 2p, odd to 2p+1.
+ *   Norm: ||x||_2 of the fp16 input, rounded to binary16 (nearest even), saturating
+ *       at 65504.
+ *
+ * Rotation parameters: float32 [L][Hkv][32][2][4] = per 4-coordinate block k the unit
+ *   quaternions (qL, qR), each (w,x,y,z); block k maps y[4k..4k+3] (read as a
+ *   quaternion) to qL * y * conj(qR).  R x = S(H x / sqrt(128)), H Sylvester-ordered.
+ */
+#ifndef IQ_H
+#define IQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* iq_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  IQ_OK = 0,
+  IQ_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, inconsistent shapes */
+  IQ_ERR_UNSUPPORTED = 2, /* head_dim != 128, GQA group size not 1, 2, 4 or 8, bad dtype */
+  IQ_ERR_CAPACITY = 3,    /* a host-known size exceeds the cache's capacity */
+  IQ_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than iq_decode_workspace_size */
+  IQ_ERR_ALIGNMENT = 5,   /* a device pointer is not 16-byte aligned (workspace: 256) */
+  IQ_ERR_CUDA = 6         /* a kernel launch or CUDA runtime call failed */
+} iq_status;
+
+typedef enum { IQ_F16 = 0, IQ_F32 = 1 } iq_dtype;
+
+/* Bits OR-ed into *status_dev by kernels that meet bad data (see conventions). */
+#define IQ_DEVERR_POSITION 1u /* token position outside its sequence's pages */
+#define IQ_DEVERR_PAGE 2u     /* block-table entry outside [0, n_pages) */
+#define IQ_DEVERR_CTX 4u      /* context length outside [0, max_ctx] */
+
+typedef struct {
+  void* k_codes;                   /* device, see layout above */
+  void* v_codes;                   /* device */
+  void* k_norms;                   /* device, uint16 binary16 bits */
+  void* v_norms;                   /* device */
+  int32_t n_layers;                /* L >= 1 */
+  int32_t n_kv_heads;              /* Hkv >= 1 */
+  int32_t head_dim;                /* must be 128 */
+  int32_t page_size;               /* tokens per page, multiple of 16 */
+  int32_t n_pages;                 /* pages in the pool */
+  const int32_t* block_table_dev;  /* [batch][max_pages_per_seq] or NULL */
+  int32_t max_pages_per_seq;       /* ignored when block_table_dev is NULL */
+  uint32_t* status_dev;            /* device word for IQ_DEVERR_* bits, or NULL */
+} iq_cache;
+
+/* Library version string (static storage). */
+const char* iq_version(void);
+
+/* Human-readable text of a status code (static storage; never NULL). */
+const char* iq_status_string(iq_status s);
+
+/* Bytes of one code pool (k_codes or v_codes) and of one norm pool (k_norms or v_norms)
+ * for the given geometry.  Host-only; returns IQ_ERR_INVALID_ARG on bad sizes. */
+iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
+                         size_t* code_bytes_host, size_t* norm_bytes_host);
+
+/* Rotation parameters from a seed (host-only; writes n_layers*n_kv_heads*256 floats to
+ * params_host).  Each quaternion is drawn uniformly from the unit 3-sphere by Marsaglia's
+ * method from a splitmix64 counter stream keyed by (seed, layer, head, block, side); the
+ * pages publish no parameter values, they fix only their number (256 per head).
+ * Errors: IQ_ERR_INVALID_ARG for NULL params_host or non-positive sizes. */
+iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, float* params_host);
+
+/* Quantise-and-append: encode n_new new tokens of every sequence into layer `layer`.
+ *   k_dev, v_dev : fp16 [batch][n_new][Hkv][128]; either may be NULL (that side skipped).
+ *   start_pos_dev: int32 [batch], position of each sequence's first new token.
+ *   params_dev   : float32 [L][Hkv][32][2][4].
+ * Per vector: norm (fp32 accumulate) -> WHT -> SO(4) blocks -> threshold search against
+ * the 7 Lloyd-Max boundaries -> packed record + binary16 norm written at its slot.
+ * Writes only the record bytes of the tokens it encodes (the other token of a V pair is
+ * preserved).  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; IQ_DEVERR_POSITION /
+ * IQ_DEVERR_PAGE on the device. */
+iq_status iq_encode_append(const iq_cache* cache, int32_t layer, const void* k_dev, const void* v_dev,
+                           int32_t batch, int32_t n_new, const int32_t* start_pos_dev,
+                           const float* params_dev, iq_stream_t stream);
+
+/* Workspace bytes iq_decode_attention needs for these sizes (split-K partials). */
+size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx);
+
+/* Decode attention over the packed cache of layer `layer`.
+ *   q_dev        : [batch][n_q_heads][128], fp16 (IQ_F16) or fp32 (IQ_F32).
+ *   ctx_len_dev  : int32 [batch], tokens 0..ctx_len-1 of each sequence are attended;
+ *                  0 gives a zero output row; values outside [0, max_ctx] are clamped
+ *                  into range and flagged with IQ_DEVERR_CTX.
+ *   max_ctx      : host upper bound on ctx_len (sizes the split-K grid); must not exceed
+ *                  the per-sequence capacity (page_size, or page_size*max_pages_per_seq).
+ *   params_dev   : float32 [L][Hkv][32][2][4], the parameters used when encoding.
+ *   out_dev      : float32 [batch][n_q_heads][128].
+ *   workspace_dev: at least iq_decode_workspace_size(...) bytes, 256-byte aligned; its
+ *                  contents need no initialisation and are scratch after the call.
+ * q head h reads kv head h / (n_q_heads / n_kv_heads); that group size must be 1, 2, 4 or 8.
+ * out[b][h] = sum_t softmax_t(<q, K_t>/sqrt(128)) V_t with K_t, V_t the dequantised
+ * vectors n * R^T c[codes] / sqrt(128), computed without forming them: q is rotated once,
+ * scores and the value sum are formed in the rotated basis from codes and norms,
+ * split-K partials are merged, and one inverse rotation is applied per output row. */
+iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
+                              int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
+                              const float* params_dev, float* out_dev, void* workspace_dev,
+                              size_t workspace_bytes, iq_stream_t stream);
+
+/* Read back tokens [t0, t0+n) of sequence `seq` in layer `layer` as canonical codes:
+ *   codes_dev: uint8 [Hkv][n][128] (coordinate order), norms_dev: uint16 [Hkv][n] or NULL.
+ *   kv: 0 = K pool, 1 = V pool.  Host-checked against the sequence capacity. */
+iq_status iq_export_codes(const iq_cache* cache, int32_t layer, int32_t kv, int32_t seq, int32_t t0,
+                          int32_t n, uint8_t* codes_dev, uint16_t* norms_dev, iq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IQ_H */

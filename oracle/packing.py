@@ -127,3 +127,69 @@ def unpack_v(records, T=None):
 def v_byte_owner():
     """For each of the 96 bytes of a V record, which token of the pair (0 or 1) owns it."""
     return np.arange(V_PAIR_BYTES) % 2
+
+
+# --------------------------------------------------------------------- vectorised forms
+# The same layout written with numpy array operations for large inputs; tests check them
+# against the per-slot loops above.
+def _chunk_words(y):
+    """y: (..., 32) codes -> (..., 3) uint32 words."""
+    y = np.asarray(y, dtype=np.uint32) & 7
+    j = np.arange(8, dtype=np.uint32)
+    words = []
+    for w in range(3):
+        word = np.bitwise_or.reduce(y[..., 8 * w : 8 * w + 8] << (4 * j), axis=-1)
+        word |= np.bitwise_or.reduce(((y[..., 24:32] >> w) & 1) << (4 * j + 3), axis=-1)
+        words.append(word)
+    return np.stack(words, axis=-1).astype(np.uint32)
+
+
+def _words_chunk(words):
+    """(..., 3) uint32 words -> (..., 32) codes."""
+    words = np.asarray(words, dtype=np.uint32)
+    j = np.arange(8, dtype=np.uint32)
+    y = np.zeros(words.shape[:-1] + (32,), dtype=np.uint32)
+    for w in range(3):
+        y[..., 8 * w : 8 * w + 8] = (words[..., w : w + 1] >> (4 * j)) & 7
+        y[..., 24:32] |= ((words[..., w : w + 1] >> (4 * j + 3)) & 1) << w
+    return y.astype(np.uint8)
+
+
+_V_TOK = np.array([1 if (s % 4) >= 2 else 0 for s in range(32)])
+_V_COORD = np.array([[16 * g + 2 * (s // 4) + (s % 2) for s in range(32)] for g in range(8)])
+
+
+def pack_k_fast(codes):
+    codes = np.asarray(codes)
+    T = codes.shape[0]
+    y = codes.reshape(T, 4, 32)  # chunk c holds coordinates 32c .. 32c+31 in slot order
+    return _chunk_words(y).reshape(T, 12).view("<u4").view(np.uint8).reshape(T, K_BYTES)
+
+
+def unpack_k_fast(records):
+    records = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
+    T = records.shape[0]
+    words = records.view("<u4").reshape(T, 4, 3)
+    return _words_chunk(words).reshape(T, 128)
+
+
+def pack_v_fast(codes):
+    codes = np.asarray(codes)
+    T = codes.shape[0]
+    P = (T + 1) // 2
+    pad = np.zeros((2 * P, 128), dtype=codes.dtype)
+    pad[:T] = codes
+    pairs = pad.reshape(P, 2, 128)
+    y = pairs[:, _V_TOK[None, :], _V_COORD]  # (P, 8, 32)
+    return _chunk_words(y).reshape(P, 24).view("<u4").view(np.uint8).reshape(P, V_PAIR_BYTES)
+
+
+def unpack_v_fast(records, T=None):
+    records = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
+    P = records.shape[0]
+    if T is None:
+        T = 2 * P
+    y = _words_chunk(records.view("<u4").reshape(P, 8, 3))  # (P, 8, 32)
+    pairs = np.zeros((P, 2, 128), dtype=np.uint8)
+    pairs[:, _V_TOK[None, :], _V_COORD] = y
+    return pairs.reshape(2 * P, 128)[:T]

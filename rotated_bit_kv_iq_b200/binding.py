@@ -1,0 +1,196 @@
+"""ctypes binding of libiq (include/iq.h): argument marshalling only.
+
+Every entry point keeps its C name.  Device buffers are torch CUDA tensors (PyTorch is used
+for device memory and streams only); every step of the computation runs in libiq's kernels.
+Loading fails loudly when libiq.so is missing: there is no CPU fallback.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libiq.so")
+
+IQ_OK = 0
+IQ_ERR_INVALID_ARG = 1
+IQ_ERR_UNSUPPORTED = 2
+IQ_ERR_CAPACITY = 3
+IQ_ERR_WORKSPACE = 4
+IQ_ERR_ALIGNMENT = 5
+IQ_ERR_CUDA = 6
+IQ_F16 = 0
+IQ_F32 = 1
+IQ_DEVERR_POSITION = 1
+IQ_DEVERR_PAGE = 2
+IQ_DEVERR_CTX = 4
+
+HEAD_DIM = 128
+K_RECORD_BYTES = 48
+V_PAIR_BYTES = 96
+
+
+class IqError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn}: {iq_status_string(status)} (status {status})")
+        self.status = status
+
+
+class iq_cache(ctypes.Structure):
+    _fields_ = [
+        ("k_codes", ctypes.c_void_p),
+        ("v_codes", ctypes.c_void_p),
+        ("k_norms", ctypes.c_void_p),
+        ("v_norms", ctypes.c_void_p),
+        ("n_layers", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("n_pages", ctypes.c_int32),
+        ("block_table_dev", ctypes.c_void_p),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("status_dev", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libiq.so once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libiq.so not built at {LIB_PATH}; run `python -m rotated_bit_kv_iq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        P = ctypes.POINTER(iq_cache)
+        L.iq_version.restype = ctypes.c_char_p
+        L.iq_version.argtypes = []
+        L.iq_status_string.restype = ctypes.c_char_p
+        L.iq_status_string.argtypes = [ctypes.c_int]
+        L.iq_cache_bytes.restype = ctypes.c_int
+        L.iq_cache_bytes.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.iq_init_rotation.restype = ctypes.c_int
+        L.iq_init_rotation.argtypes = [ctypes.c_uint64, i32, i32, vp]
+        L.iq_encode_append.restype = ctypes.c_int
+        L.iq_encode_append.argtypes = [P, i32, vp, vp, i32, i32, vp, vp, vp]
+        L.iq_decode_workspace_size.restype = sz
+        L.iq_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.iq_decode_attention.restype = ctypes.c_int
+        L.iq_decode_attention.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp, sz, vp]
+        L.iq_export_codes.restype = ctypes.c_int
+        L.iq_export_codes.argtypes = [P, i32, i32, i32, i32, i32, vp, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, st):
+    if st != IQ_OK:
+        raise IqError(fn, st)
+
+
+# ----------------------------------------------------------------------- entry points
+def iq_version():
+    return lib().iq_version().decode()
+
+
+def iq_status_string(status):
+    return lib().iq_status_string(int(status)).decode()
+
+
+def iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages):
+    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check("iq_cache_bytes", lib().iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def iq_init_rotation(seed, n_layers, n_kv_heads):
+    """Seeded rotation parameters as a host float32 array [L][Hkv][32][2][4]."""
+    out = np.zeros((n_layers, n_kv_heads, 32, 2, 4), dtype=np.float32)
+    _check("iq_init_rotation", lib().iq_init_rotation(ctypes.c_uint64(seed), n_layers, n_kv_heads,
+                                                      out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def iq_encode_append(cache, layer, k, v, start_pos, params, stream=None):
+    """k, v: fp16 [batch][n_new][Hkv][128] CUDA tensors (either may be None)."""
+    ref = k if k is not None else v
+    batch, n_new = int(ref.shape[0]), int(ref.shape[1])
+    _check("iq_encode_append", lib().iq_encode_append(ctypes.byref(cache.c), layer, _ptr(k), _ptr(v), batch, n_new,
+                                                      _ptr(start_pos), _ptr(params), _stream(stream)))
+
+
+def iq_decode_workspace_size(batch, n_q_heads, n_kv_heads, max_ctx):
+    return int(lib().iq_decode_workspace_size(batch, n_q_heads, n_kv_heads, max_ctx))
+
+
+def iq_decode_attention(cache, layer, q, ctx_len, max_ctx, params, out, workspace, stream=None):
+    """q: [batch][Hq][128] fp16|fp32; out: fp32 [batch][Hq][128]; workspace: uint8 CUDA tensor."""
+    import torch
+
+    dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
+    _check("iq_decode_attention", lib().iq_decode_attention(
+        ctypes.byref(cache.c), layer, _ptr(q), dtype, int(q.shape[0]), int(q.shape[1]), _ptr(ctx_len), int(max_ctx),
+        _ptr(params), _ptr(out), _ptr(workspace), int(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def iq_export_codes(cache, layer, kv, seq, t0, n, codes, norms=None, stream=None):
+    """codes: uint8 [Hkv][n][128] CUDA tensor; norms: int16/uint16 [Hkv][n] or None."""
+    _check("iq_export_codes", lib().iq_export_codes(ctypes.byref(cache.c), layer, kv, seq, t0, n, _ptr(codes),
+                                                    _ptr(norms), _stream(stream)))
+
+
+# ----------------------------------------------------------------------- cache holder
+class PagedCache:
+    """Device pools for a packed K/V cache (torch tensors) and the iq_cache struct over them.
+
+    page_size tokens per page; with block_table None, sequence b owns page b (a contiguous
+    cache of capacity page_size tokens per sequence)."""
+
+    def __init__(self, n_layers, n_kv_heads, page_size, n_pages, block_table=None, device="cuda"):
+        import torch
+
+        code_bytes, norm_bytes = iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages)
+        self.k_codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
+        self.v_codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
+        self.k_norms = torch.empty(norm_bytes // 2, dtype=torch.int16, device=device)
+        self.v_norms = torch.empty(norm_bytes // 2, dtype=torch.int16, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.block_table = block_table
+        self.n_layers, self.n_kv_heads, self.page_size, self.n_pages = n_layers, n_kv_heads, page_size, n_pages
+        self.max_pages_per_seq = int(block_table.shape[1]) if block_table is not None else 1
+        self.c = iq_cache(
+            self.k_codes.data_ptr(), self.v_codes.data_ptr(), self.k_norms.data_ptr(), self.v_norms.data_ptr(),
+            n_layers, n_kv_heads, HEAD_DIM, page_size, n_pages,
+            block_table.data_ptr() if block_table is not None else None,
+            self.max_pages_per_seq, self.status.data_ptr(),
+        )
+
+    # Views of the pools with their logical shapes (for writing oracle-made records in tests).
+    def k_code_view(self):
+        return self.k_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size, K_RECORD_BYTES)
+
+    def v_code_view(self):
+        return self.v_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // 2, V_PAIR_BYTES)
+
+    def k_norm_view(self):
+        return self.k_norms.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size)
+
+    def v_norm_view(self):
+        return self.v_norms.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size)

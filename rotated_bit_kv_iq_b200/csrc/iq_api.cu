@@ -1,0 +1,180 @@
+// extern "C" entry points of libiq: argument checks, layer views, kernel dispatch.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "iq_internal.h"
+
+namespace iq {
+
+// Centroids are handed to the kernels as binary16 values scaled by alpha.  alpha is chosen
+// so that alpha*c_k is within 2e-5 (relative) of a binary16 value for all eight levels
+// (plain binary16 rounding of c_k alone is off by up to 4.9e-4), which keeps the score and
+// value sums within ~1e-4 of the fp64 result.
+static const double kAlpha = 1.614664;
+
+static KernelConsts make_consts() {
+  const Codebook cb = compute_codebook();
+  KernelConsts kc;
+  for (int j = 0; j < 3; ++j) kc.bound_pos[j] = (float)cb.bound[4 + j];
+  uint32_t lo[2] = {0, 0}, hi[2] = {0, 0};
+  for (int k = 0; k < 8; ++k) {
+    const __half h = __float2half_rn((float)(kAlpha * cb.level[k]));
+    uint16_t bits;
+    std::memcpy(&bits, &h, 2);
+    lo[k >> 2] |= (uint32_t)(bits & 0xFF) << (8 * (k & 3));
+    hi[k >> 2] |= (uint32_t)(bits >> 8) << (8 * (k & 3));
+  }
+  kc.lut_lo[0] = lo[0];
+  kc.lut_lo[1] = lo[1];
+  kc.lut_hi[0] = hi[0];
+  kc.lut_hi[1] = hi[1];
+  kc.inv_alpha = (float)(1.0 / kAlpha);
+  return kc;
+}
+
+const KernelConsts& kernel_consts() {
+  static std::once_flag once;
+  static KernelConsts kc;
+  std::call_once(once, [] { kc = make_consts(); });
+  return kc;
+}
+
+static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static iq_status check_cache(const iq_cache* c, int32_t layer) {
+  if (!c) return IQ_ERR_INVALID_ARG;
+  if (c->head_dim != D) return IQ_ERR_UNSUPPORTED;
+  if (c->n_layers < 1 || c->n_kv_heads < 1 || c->page_size < 16 || c->page_size % 16 != 0 || c->n_pages < 1)
+    return IQ_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= c->n_layers) return IQ_ERR_INVALID_ARG;
+  if (!c->k_codes || !c->v_codes || !c->k_norms || !c->v_norms) return IQ_ERR_INVALID_ARG;
+  if (c->block_table_dev && c->max_pages_per_seq < 1) return IQ_ERR_INVALID_ARG;
+  if (!aligned(c->k_codes, 16) || !aligned(c->v_codes, 16) || !aligned(c->k_norms, 16) ||
+      !aligned(c->v_norms, 16))
+    return IQ_ERR_ALIGNMENT;
+  return IQ_OK;
+}
+
+static LayerView view(const iq_cache* c, int32_t layer) {
+  LayerView v;
+  const size_t per_layer_tokens = (size_t)c->n_pages * c->n_kv_heads * c->page_size;
+  v.k_codes = (uint8_t*)c->k_codes + per_layer_tokens * K_REC * layer;
+  v.v_codes = (uint8_t*)c->v_codes + per_layer_tokens * K_REC * layer;  // 96 B per pair = 48 B per token
+  v.k_norms = (uint16_t*)c->k_norms + per_layer_tokens * layer;
+  v.v_norms = (uint16_t*)c->v_norms + per_layer_tokens * layer;
+  v.block_table = c->block_table_dev;
+  v.max_pages = c->block_table_dev ? c->max_pages_per_seq : 1;
+  v.page_size = c->page_size;
+  v.n_pages = c->n_pages;
+  v.n_kv_heads = c->n_kv_heads;
+  v.status = c->status_dev;
+  return v;
+}
+
+static int64_t seq_capacity(const iq_cache* c) {
+  return c->block_table_dev ? (int64_t)c->page_size * c->max_pages_per_seq : (int64_t)c->page_size;
+}
+
+}  // namespace iq
+
+using namespace iq;
+
+extern "C" {
+
+const char* iq_version(void) { return "libiq 0.1 (sm_100a; packed 3-bit IsoQuant KV)"; }
+
+const char* iq_status_string(iq_status s) {
+  switch (s) {
+    case IQ_OK: return "ok";
+    case IQ_ERR_INVALID_ARG: return "invalid argument";
+    case IQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case IQ_ERR_CAPACITY: return "size exceeds cache capacity";
+    case IQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case IQ_ERR_ALIGNMENT: return "device pointer not aligned";
+    case IQ_ERR_CUDA: return "CUDA launch or runtime error";
+  }
+  return "unknown status";
+}
+
+iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
+                         size_t* code_bytes_host, size_t* norm_bytes_host) {
+  if (n_layers < 1 || n_kv_heads < 1 || page_size < 16 || page_size % 16 != 0 || n_pages < 1)
+    return IQ_ERR_INVALID_ARG;
+  const size_t tokens = (size_t)n_layers * n_pages * n_kv_heads * page_size;
+  if (code_bytes_host) *code_bytes_host = tokens * K_REC;
+  if (norm_bytes_host) *norm_bytes_host = tokens * sizeof(uint16_t);
+  return IQ_OK;
+}
+
+iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, float* params_host) {
+  if (!params_host || n_layers < 1 || n_kv_heads < 1) return IQ_ERR_INVALID_ARG;
+  init_rotation_params(seed, n_layers, n_kv_heads, params_host);
+  return IQ_OK;
+}
+
+iq_status iq_encode_append(const iq_cache* cache, int32_t layer, const void* k_dev, const void* v_dev,
+                           int32_t batch, int32_t n_new, const int32_t* start_pos_dev,
+                           const float* params_dev, iq_stream_t stream) {
+  iq_status st = check_cache(cache, layer);
+  if (st != IQ_OK) return st;
+  if (batch < 0 || n_new < 0 || !start_pos_dev || !params_dev) return IQ_ERR_INVALID_ARG;
+  if (!k_dev && !v_dev) return IQ_ERR_INVALID_ARG;
+  if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
+  if ((int64_t)n_new > seq_capacity(cache)) return IQ_ERR_CAPACITY;
+  if ((k_dev && !aligned(k_dev, 16)) || (v_dev && !aligned(v_dev, 16)) || !aligned(params_dev, 16) ||
+      !aligned(start_pos_dev, 4))
+    return IQ_ERR_ALIGNMENT;
+  const LayerView v = view(cache, layer);
+  const float* pl = params_dev + (size_t)layer * cache->n_kv_heads * NBLK * 8;
+  const int e = launch_encode(v, k_dev, v_dev, batch, n_new, start_pos_dev, pl, kernel_consts(), stream);
+  return e ? IQ_ERR_CUDA : IQ_OK;
+}
+
+size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx) {
+  if (batch < 0 || n_q_heads < 0 || n_kv_heads < 1 || max_ctx < 0) return 0;
+  return decode_workspace_bytes(batch, n_q_heads, n_kv_heads, max_ctx);
+}
+
+iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
+                              int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
+                              const float* params_dev, float* out_dev, void* workspace_dev,
+                              size_t workspace_bytes, iq_stream_t stream) {
+  iq_status st = check_cache(cache, layer);
+  if (st != IQ_OK) return st;
+  if (batch < 0 || n_q_heads < 1 || max_ctx < 0 || !q_dev || !ctx_len_dev || !params_dev || !out_dev)
+    return IQ_ERR_INVALID_ARG;
+  if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
+  if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
+  const int G = n_q_heads / cache->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
+  if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
+  if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(ctx_len_dev, 4))
+    return IQ_ERR_ALIGNMENT;
+  const size_t need = decode_workspace_bytes(batch, n_q_heads, cache->n_kv_heads, max_ctx);
+  if (!workspace_dev || workspace_bytes < need) return IQ_ERR_WORKSPACE;
+  if (!aligned(workspace_dev, 256)) return IQ_ERR_ALIGNMENT;
+  const LayerView v = view(cache, layer);
+  const float* pl = params_dev + (size_t)layer * cache->n_kv_heads * NBLK * 8;
+  const int e = launch_decode(v, q_dev, q_dtype == IQ_F32, batch, n_q_heads, ctx_len_dev, max_ctx, pl, out_dev,
+                              workspace_dev, kernel_consts(), stream);
+  return e ? IQ_ERR_CUDA : IQ_OK;
+}
+
+iq_status iq_export_codes(const iq_cache* cache, int32_t layer, int32_t kv, int32_t seq, int32_t t0, int32_t n,
+                          uint8_t* codes_dev, uint16_t* norms_dev, iq_stream_t stream) {
+  iq_status st = check_cache(cache, layer);
+  if (st != IQ_OK) return st;
+  if ((kv != 0 && kv != 1) || seq < 0 || t0 < 0 || n < 0 || !codes_dev) return IQ_ERR_INVALID_ARG;
+  if (!cache->block_table_dev && seq >= cache->n_pages) return IQ_ERR_CAPACITY;
+  if ((int64_t)t0 + n > seq_capacity(cache)) return IQ_ERR_CAPACITY;
+  const LayerView v = view(cache, layer);
+  const int e = launch_export(v, kv, seq, t0, n, codes_dev, norms_dev, kernel_consts(), stream);
+  return e ? IQ_ERR_CUDA : IQ_OK;
+}
+
+}  // extern "C"

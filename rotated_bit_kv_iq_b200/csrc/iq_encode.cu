@@ -1,0 +1,205 @@
+// Quantise-and-append kernel: fp16 K/V vectors -> packed 3-bit records + binary16 norms.
+//
+// Steps per vector follow "RotaryQuant" (rebasdaily.com, section "妙处不只是压缩，而是不再展开")
+// and its abstract (arXiv 2608.08081): Walsh-Hadamard mixing, then the block SO(4)
+// rotation, then scalar quantisation; the quantiser is the Lloyd-Max codebook of N(0,1/d)
+// ("压缩与速度的博弈" zhichai.net, sections "Beta 分布的魔力", "Lloyd-Max 最优量化").
+//
+// Mapping: one thread encodes one 128-vector entirely in registers (all seven butterfly
+// stages are register-local, no shuffles).  A CTA covers 128 consecutive positions of one
+// (sequence, kv head, K|V); the head's 32 fused block matrices live in shared memory and
+// every lane of a warp reads the same one at the same time (broadcast).  Instead of
+// normalising the vector, the rotated coordinates z = R x are compared with the
+// boundaries scaled by ||x||/sqrt(128).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "iq_device.cuh"
+
+namespace iq {
+
+constexpr int ENC_THREADS = 128;
+
+// code = #{ j : u > b_j } with u = sqrt(128) z / n, written with the three positive
+// thresholds t_j = b_j n / sqrt(128): magnitude class m = #{ |z| > t_j }, code = 4+m for
+// z > 0 and 3-m otherwise.  (Exact ties |z| = t_j are within rounding of a boundary.)
+__device__ __forceinline__ uint32_t quantise(float z, float t1, float t2, float t3) {
+  const float a = fabsf(z);
+  const uint32_t m = (uint32_t)(a > t1) + (uint32_t)(a > t2) + (uint32_t)(a > t3);
+  return z > 0.f ? 4u + m : 3u - m;
+}
+
+__global__ void __launch_bounds__(ENC_THREADS)
+encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int n_new,
+              const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
+  __shared__ float4 smat[NBLK][4];  // fused block matrices M'_k, row r as a float4
+  const int b = blockIdx.z;
+  const int head = blockIdx.y >> 1;
+  const int side = blockIdx.y & 1;  // 0 = K, 1 = V
+  const __half* src = side ? v_src : k_src;
+  if (src == nullptr) return;
+
+  if (threadIdx.x < NBLK) {
+    float Mp[4][4];
+    fused_block_matrix(params_layer + ((size_t)head * NBLK + threadIdx.x) * 8, Mp);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) smat[threadIdx.x][r] = make_float4(Mp[r][0], Mp[r][1], Mp[r][2], Mp[r][3]);
+  }
+  __syncthreads();
+
+  const int start = start_pos[b];
+  const int pos = (start & ~1) + blockIdx.x * ENC_THREADS + threadIdx.x;  // pair-aligned lanes
+  const int i_new = pos - start;
+  const bool in_range = (i_new >= 0) && (i_new < n_new);
+  // All lanes of a warp take part in the V-pair exchange below, so inactive lanes run
+  // the arithmetic on zeros and skip only the loads and stores.
+  int page = -1;
+  if (in_range) page = resolve_page(v, b, pos);
+  const bool active = in_range && page >= 0;
+
+  float y[D];
+  if (active) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + (((size_t)b * n_new + i_new) * v.n_kv_heads + head) * D);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      uint4 w = __ldg(p + q);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __half2 h = *reinterpret_cast<const __half2*>(&ws[e]);
+        float2 f = __half22float2(h);
+        y[8 * q + 2 * e] = f.x;
+        y[8 * q + 2 * e + 1] = f.y;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) y[i] = 0.f;
+  }
+
+  // ||x||^2 in fp32
+  float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < D; i += 2) {
+    ss0 = fmaf(y[i], y[i], ss0);
+    ss1 = fmaf(y[i + 1], y[i + 1], ss1);
+  }
+  const float n = sqrtf(ss0 + ss1);
+
+  // Butterfly stages on coordinate bits 2..6 (bits 0,1 are inside M').
+#pragma unroll
+  for (int bit = 2; bit < 7; ++bit) {
+    const int h = 1 << bit;
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+      if ((i & h) == 0) {
+        const float a = y[i], c = y[i + h];
+        y[i] = a + c;
+        y[i + h] = a - c;
+      }
+    }
+  }
+  // Fused SO(4) blocks.
+#pragma unroll
+  for (int k = 0; k < NBLK; ++k) {
+    const float v0 = y[4 * k], v1 = y[4 * k + 1], v2 = y[4 * k + 2], v3 = y[4 * k + 3];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 m = smat[k][r];
+      y[4 * k + r] = fmaf(m.x, v0, fmaf(m.y, v1, fmaf(m.z, v2, m.w * v3)));
+    }
+  }
+
+  const float sc = n * 0.08838834764831845f;  // n / sqrt(128)
+  const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
+
+  const size_t head_slot = (size_t)(page < 0 ? 0 : page) * v.n_kv_heads + head;
+  const int slot = pos % v.page_size;
+
+  if (side == 0) {
+    // K record: chunk c holds coordinates 32c..32c+31 in slot order.
+    uint32_t rec[12];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t spare = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) spare |= quantise(y[32 * c + 24 + j], t1, t2, t3) << (4 * j);
+#pragma unroll
+      for (int w = 0; w < 3; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) word |= quantise(y[32 * c + 8 * w + j], t1, t2, t3) << (4 * j);
+        word |= ((spare >> w) & 0x11111111u) << 3;
+        rec[3 * c + w] = word;
+      }
+    }
+    if (active) {
+      uint4* dst = reinterpret_cast<uint4*>(v.k_codes + (head_slot * v.page_size + slot) * K_REC);
+      dst[0] = make_uint4(rec[0], rec[1], rec[2], rec[3]);
+      dst[1] = make_uint4(rec[4], rec[5], rec[6], rec[7]);
+      dst[2] = make_uint4(rec[8], rec[9], rec[10], rec[11]);
+    }
+  } else {
+    // V record (token pair): this token's bytes, laid out as the first token of the pair
+    // (chunk g, word w: coordinates 16g+4w+{0,1,2,3} at nibbles {0,1,4,5}; coordinates
+    // 16g+12..15 as spare bits of nibbles {0,1,4,5}), shifted by 8 bits for the second.
+    const int par = pos & 1;
+    uint32_t part[24];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const int base = 16 * g;
+      uint32_t spare = quantise(y[base + 12], t1, t2, t3) | (quantise(y[base + 13], t1, t2, t3) << 4) |
+                       (quantise(y[base + 14], t1, t2, t3) << 16) | (quantise(y[base + 15], t1, t2, t3) << 20);
+#pragma unroll
+      for (int w = 0; w < 3; ++w) {
+        uint32_t word = quantise(y[base + 4 * w], t1, t2, t3) | (quantise(y[base + 4 * w + 1], t1, t2, t3) << 4) |
+                        (quantise(y[base + 4 * w + 2], t1, t2, t3) << 16) |
+                        (quantise(y[base + 4 * w + 3], t1, t2, t3) << 20);
+        word |= ((spare >> w) & 0x00110011u) << 3;
+        part[3 * g + w] = par ? (word << 8) : word;
+      }
+    }
+    // Merge with the partner lane (same pair).  The exchange runs on every lane (the whole
+    // warp is converged here); only the stores depend on which tokens this launch writes.
+    const unsigned lane = threadIdx.x & 31;
+    const bool partner_active = __shfl_xor_sync(0xffffffffu, (int)active, 1) != 0;
+    uint8_t* rec = v.v_codes + (head_slot * (v.page_size / 2) + (slot >> 1)) * V_REC;
+    uint32_t mine[12];  // even lane: chunks 0..3 of the record, odd lane: chunks 4..7
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const uint32_t send = (lane & 1) ? part[i] : part[12 + i];
+      const uint32_t got = __shfl_xor_sync(0xffffffffu, send, 1);
+      mine[i] = ((lane & 1) ? part[12 + i] : part[i]) | got;
+    }
+    if (active && partner_active) {
+      uint4* dst = reinterpret_cast<uint4*>(rec + (lane & 1) * 48);
+      dst[0] = make_uint4(mine[0], mine[1], mine[2], mine[3]);
+      dst[1] = make_uint4(mine[4], mine[5], mine[6], mine[7]);
+      dst[2] = make_uint4(mine[8], mine[9], mine[10], mine[11]);
+    } else if (active) {
+      // Partner token not in this launch: write only this token's bytes.
+#pragma unroll
+      for (int i = 0; i < 24; ++i) {
+        const uint32_t w = part[i];
+        rec[4 * i + par] = (uint8_t)(w >> (8 * par));
+        rec[4 * i + 2 + par] = (uint8_t)(w >> (16 + 8 * par));
+      }
+    }
+  }
+
+  if (active) {
+    uint16_t* nrm = side ? v.v_norms : v.k_norms;
+    nrm[head_slot * v.page_size + slot] = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
+  }
+}
+
+int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
+                  const int32_t* start_pos, const float* params_layer, const KernelConsts& kc, void* stream) {
+  if (batch == 0 || n_new == 0) return 0;
+  dim3 grid((n_new + 1 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * 2, batch);
+  encode_kernel<<<grid, ENC_THREADS, 0, (cudaStream_t)stream>>>(v, (const __half*)k, (const __half*)vsrc, n_new,
+                                                                start_pos, params_layer, kc);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace iq

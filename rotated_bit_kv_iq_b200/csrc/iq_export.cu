@@ -1,0 +1,67 @@
+// Export kernel: packed K/V records -> canonical codes (uint8, coordinate order) and norms.
+// One thread per (kv head, token); used to check the packed format against the oracle.
+#include <cuda_runtime.h>
+
+#include "iq_device.cuh"
+
+namespace iq {
+
+__global__ void export_kernel(LayerView v, int kv, int seq, int t0, int n, uint8_t* __restrict__ codes,
+                              uint16_t* __restrict__ norms) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int head = blockIdx.y;
+  if (i >= n) return;
+  const int pos = t0 + i;
+  const int page = resolve_page(v, seq, pos);
+  uint8_t* out = codes + ((size_t)head * n + i) * D;
+  if (page < 0) {
+    for (int c = 0; c < D; ++c) out[c] = 0xFF;
+    if (norms) norms[(size_t)head * n + i] = 0xFFFF;
+    return;
+  }
+  const int slot = pos % v.page_size;
+  const size_t hs = (size_t)page * v.n_kv_heads + head;
+  uint8_t y[D];
+  if (kv == 0) {
+    const uint32_t* rec = reinterpret_cast<const uint32_t*>(v.k_codes + (hs * v.page_size + slot) * K_REC);
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t w[3] = {rec[3 * c], rec[3 * c + 1], rec[3 * c + 2]};
+      for (int s = 0; s < 32; ++s) {
+        uint32_t code;
+        if (s < 24) code = (w[s >> 3] >> (4 * (s & 7))) & 7u;
+        else code = ((w[0] >> (4 * (s - 24) + 3)) & 1u) | (((w[1] >> (4 * (s - 24) + 3)) & 1u) << 1) |
+                    (((w[2] >> (4 * (s - 24) + 3)) & 1u) << 2);
+        y[32 * c + s] = (uint8_t)code;
+      }
+    }
+  } else {
+    const uint32_t* rec = reinterpret_cast<const uint32_t*>(v.v_codes + (hs * (v.page_size / 2) + (slot >> 1)) * V_REC);
+    const int par = slot & 1;
+    for (int gch = 0; gch < 8; ++gch) {
+      const uint32_t w[3] = {rec[3 * gch], rec[3 * gch + 1], rec[3 * gch + 2]};
+      for (int s = 0; s < 32; ++s) {
+        if (((s & 3) >= 2) != (par == 1)) continue;  // slot belongs to the other token
+        uint32_t code;
+        if (s < 24) code = (w[s >> 3] >> (4 * (s & 7))) & 7u;
+        else code = ((w[0] >> (4 * (s - 24) + 3)) & 1u) | (((w[1] >> (4 * (s - 24) + 3)) & 1u) << 1) |
+                    (((w[2] >> (4 * (s - 24) + 3)) & 1u) << 2);
+        y[16 * gch + 2 * (s >> 2) + (s & 1)] = (uint8_t)code;
+      }
+    }
+  }
+  for (int c = 0; c < D; ++c) out[c] = y[c];
+  if (norms) {
+    const uint16_t* src = (kv == 0 ? v.k_norms : v.v_norms) + hs * v.page_size + slot;
+    norms[(size_t)head * n + i] = *src;
+  }
+}
+
+int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes, uint16_t* norms,
+                  const KernelConsts&, void* stream) {
+  if (n == 0) return 0;
+  dim3 grid((n + 127) / 128, v.n_kv_heads);
+  export_kernel<<<grid, 128, 0, (cudaStream_t)stream>>>(v, kv, seq, t0, n, codes, norms);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace iq

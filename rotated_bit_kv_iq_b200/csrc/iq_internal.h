@@ -1,0 +1,67 @@
+// Internal declarations shared by the host and device translation units of libiq.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/iq.h"
+
+namespace iq {
+
+constexpr int D = 128;          // head dimension
+constexpr int NBLK = 32;        // SO(4) blocks per head
+constexpr int K_REC = 48;       // bytes of a K record (one token)
+constexpr int V_REC = 96;       // bytes of a V record (a token pair)
+constexpr int TILE = 16;        // tokens per decode tile (one mma M dimension)
+
+// Lloyd-Max quantiser of N(0,1): 8 ascending levels, 7 midpoint boundaries (double).
+struct Codebook {
+  double level[8];
+  double bound[7];
+};
+Codebook compute_codebook();
+
+// Seeded rotation parameters, [L][Hkv][32][2][4] float32, written to `out` (host).
+void init_rotation_params(uint64_t seed, int n_layers, int n_kv_heads, float* out);
+
+// Constants handed to kernels by value.
+struct KernelConsts {
+  float bound_pos[3];    // positive N(0,1) boundaries b4, b5, b6 (b3 = 0)
+  uint32_t lut_lo[2];    // low bytes of the 8 binary16 levels alpha*c_k (k = 0..3, 4..7)
+  uint32_t lut_hi[2];    // high bytes
+  float inv_alpha;       // 1 / alpha (levels are stored scaled by alpha)
+};
+const KernelConsts& kernel_consts();
+
+// Device geometry of one layer's pools, resolved on the host.
+struct LayerView {
+  uint8_t* k_codes;      // layer base of the K code pool
+  uint8_t* v_codes;
+  uint16_t* k_norms;
+  uint16_t* v_norms;
+  const int32_t* block_table;  // NULL -> sequence b uses page b
+  int32_t max_pages;     // pages per sequence in the block table (1 when table is NULL)
+  int32_t page_size;
+  int32_t n_pages;
+  int32_t n_kv_heads;
+  uint32_t* status;
+};
+
+// Kernel launchers (defined in the .cu files); return the launch error.
+int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
+                  const int32_t* start_pos, const float* params_layer, const KernelConsts& kc,
+                  void* stream);
+int launch_decode(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads,
+                  const int32_t* ctx_len, int max_ctx, const float* params_layer, float* out,
+                  void* workspace, const KernelConsts& kc, void* stream);
+int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
+                  uint16_t* norms, const KernelConsts& kc, void* stream);
+
+// Split-K geometry (host): number of splits and tokens per split for a decode call.
+struct SplitPlan {
+  int n_split;
+  int chunk;
+};
+SplitPlan plan_splits(int batch, int n_kv_heads, int max_ctx);
+size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx);
+
+}  // namespace iq

@@ -94,3 +94,41 @@ def page_permutation(seed, n_pages):
     """A random permutation of physical page ids."""
     r = _rng(seed, 5)
     return r.permutation(n_pages).astype(np.int32)
+
+
+# ------------------------------------------------------------------ device-side generator
+def _torch_gen(device, *words):
+    import torch
+
+    h = 1469598103934665603
+    for w in words:  # FNV-1a over the words -> a 63-bit seed
+        h = ((h ^ (int(w) & 0xFFFFFFFF)) * 1099511628211) & 0xFFFFFFFFFFFFFFFF
+    return torch.Generator(device=device).manual_seed(h & 0x7FFFFFFFFFFFFFFF)
+
+
+def kv_tokens_device(seed, layer, n_kv_heads, which, n, n_outliers=4, heavy_frac=0.0, device="cuda"):
+    """Same recipe as `kv_tokens`, drawn on the device with torch's generator (a different
+    stream): fp16 tensor (n, n_kv_heads, 128).  Used to fill full-size caches quickly; the
+    parity tests use the host generator."""
+    import torch
+
+    g = _torch_gen(device, seed, 6, layer, which)
+    s = torch.exp(0.5 * torch.randn((n_kv_heads, D), generator=g, device=device, dtype=torch.float32))
+    if n_outliers:
+        for h in range(n_kv_heads):
+            idx = torch.randperm(D, generator=g, device=device)[:n_outliers]
+            s[h, idx] *= 20.0
+    z = torch.randn((n, n_kv_heads, D), generator=g, device=device, dtype=torch.float32)
+    if heavy_frac > 0.0:
+        heavy = torch.rand((n, 1, 1), generator=g, device=device) < heavy_frac
+        chi2 = (torch.randn((n, n_kv_heads, D, 3), generator=g, device=device) ** 2).sum(-1)
+        t3 = torch.randn((n, n_kv_heads, D), generator=g, device=device) / torch.sqrt(chi2 / 3.0)
+        z = torch.where(heavy, t3, z)
+    return torch.clamp(z * s, -FP16_MAX, FP16_MAX).to(torch.float16)
+
+
+def queries_device(seed, layer, batch, n_q_heads, device="cuda"):
+    import torch
+
+    g = _torch_gen(device, seed, 7, layer)
+    return torch.randn((batch, n_q_heads, D), generator=g, device=device).to(torch.float16)

@@ -1,0 +1,138 @@
+"""Host-side checks of the C ABI (no GPU needed): exported symbols, host-only entry points,
+and argument validation that must reject a call before any kernel launch."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rotation
+from rotated_bit_kv_iq_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from rotated_bit_kv_iq_b200 import build
+
+    build.build()
+    return B.lib()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    hdr = open(os.path.join(ROOT, "include", "iq.h")).read()
+    names = set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(iq_\w+)\s*\(", hdr, flags=re.M))
+    assert {"iq_init_rotation", "iq_encode_append", "iq_decode_attention", "iq_decode_workspace_size",
+            "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(lib):
+    assert "libiq" in B.iq_version()
+    for s in range(7):
+        assert B.iq_status_string(s)
+    assert B.iq_status_string(99) == "unknown status"
+
+
+def test_init_rotation_is_bit_identical_to_oracle(lib):
+    got = B.iq_init_rotation(1, 3, 4)
+    want = rotation.init_rotation(1, 3, 4)
+    assert got.dtype == np.float32 and got.shape == (3, 4, 32, 2, 4)
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    got = B.iq_init_rotation(0xDEADBEEFCAFEF00D, 2, 3)
+    np.testing.assert_array_equal(got.view(np.uint32), rotation.init_rotation(0xDEADBEEFCAFEF00D, 2, 3).view(np.uint32))
+
+
+def test_cache_bytes_and_workspace(lib):
+    cb, nb = B.iq_cache_bytes(2, 4, 64, 10)
+    assert cb == 2 * 4 * 64 * 10 * 48 and nb == 2 * 4 * 64 * 10 * 2
+    with pytest.raises(B.IqError):
+        B.iq_cache_bytes(1, 1, 24, 1)  # page size not a multiple of 16
+    w1 = B.iq_decode_workspace_size(1, 32, 4, 32768)
+    w2 = B.iq_decode_workspace_size(2, 32, 4, 32768)
+    assert 0 < w1 <= w2
+    assert B.iq_decode_workspace_size(1, 32, 0, 10) == 0
+
+
+# --- validation: fake but aligned device addresses; every call below must be rejected
+# on the host.  Skipped on a GPU machine so that a validation bug can never launch a
+# kernel on these addresses.
+cpu_only = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer checks run only without a GPU")
+
+
+def _fake_cache(**kw):
+    c = B.iq_cache(0x10000, 0x20000, 0x30000, 0x40000, 2, 2, 128, 64, 4, None, 1, None)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _enc(c, layer=0, k=0x50000, v=0x60000, batch=1, n_new=4, start=0x70000, params=0x80000):
+    return B.lib().iq_encode_append(ctypes.byref(c) if c is not None else None, layer, k, v, batch, n_new, start,
+                                    params, None)
+
+
+def _dec(c, layer=0, q=0x50000, dtype=0, batch=1, hq=8, ctx=0x70000, max_ctx=32, params=0x80000, out=0x90000,
+         ws=0xA0000, ws_bytes=1 << 30):
+    return B.lib().iq_decode_attention(ctypes.byref(c) if c is not None else None, layer, q, dtype, batch, hq, ctx,
+                                       max_ctx, params, out, ws, ws_bytes, None)
+
+
+@cpu_only
+def test_encode_rejects_bad_arguments(lib):
+    assert _enc(None) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(head_dim=64)) == B.IQ_ERR_UNSUPPORTED
+    assert _enc(_fake_cache(page_size=24)) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(), layer=2) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(), layer=-1) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(k_codes=None)) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(k_codes=0x10004)) == B.IQ_ERR_ALIGNMENT
+    assert _enc(_fake_cache(), k=None, v=None) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(), start=None) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(), params=None) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(), k=0x50008) == B.IQ_ERR_ALIGNMENT
+    assert _enc(_fake_cache(), n_new=65) == B.IQ_ERR_CAPACITY          # > page_size without a block table
+    assert _enc(_fake_cache(), batch=5) == B.IQ_ERR_CAPACITY           # more sequences than pages
+    assert _enc(_fake_cache(), n_new=-1) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(block_table_dev=0xB0000, max_pages_per_seq=0)) == B.IQ_ERR_INVALID_ARG
+
+
+@cpu_only
+def test_decode_rejects_bad_arguments(lib):
+    assert _dec(None) == B.IQ_ERR_INVALID_ARG
+    assert _dec(_fake_cache(head_dim=96)) == B.IQ_ERR_UNSUPPORTED
+    assert _dec(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED          # group size 3
+    assert _dec(_fake_cache(), hq=5) == B.IQ_ERR_INVALID_ARG          # not a multiple of Hkv
+    assert _dec(_fake_cache(), dtype=7) == B.IQ_ERR_UNSUPPORTED
+    assert _dec(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
+    assert _dec(_fake_cache(), ws_bytes=16) == B.IQ_ERR_WORKSPACE
+    assert _dec(_fake_cache(), ws=None) == B.IQ_ERR_WORKSPACE
+    assert _dec(_fake_cache(), ws=0xA0010) == B.IQ_ERR_ALIGNMENT
+    assert _dec(_fake_cache(), q=0x50004) == B.IQ_ERR_ALIGNMENT
+    assert _dec(_fake_cache(), out=None) == B.IQ_ERR_INVALID_ARG
+    assert _dec(_fake_cache(), ctx=None) == B.IQ_ERR_INVALID_ARG
+    assert _dec(_fake_cache(), batch=-1) == B.IQ_ERR_INVALID_ARG
+    assert _dec(_fake_cache(), max_ctx=-1) == B.IQ_ERR_INVALID_ARG
+
+
+@cpu_only
+def test_export_rejects_bad_arguments(lib):
+    c = _fake_cache()
+    f = B.lib().iq_export_codes
+    assert f(ctypes.byref(c), 0, 2, 0, 0, 4, 0x50000, None, None) == B.IQ_ERR_INVALID_ARG
+    assert f(ctypes.byref(c), 0, 0, 4, 0, 4, 0x50000, None, None) == B.IQ_ERR_CAPACITY
+    assert f(ctypes.byref(c), 0, 0, 0, 60, 8, 0x50000, None, None) == B.IQ_ERR_CAPACITY
+    assert f(ctypes.byref(c), 0, 0, 0, 0, 4, None, None, None) == B.IQ_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        B.lib()

@@ -1,0 +1,335 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Encode: codes bit-exact except coordinates the oracle places within 1e-6 of a decision
+boundary (counted; must stay <= 0.01% of codes); norms within 1 binary16 ulp; packed
+bytes identical once those excluded codes are taken from the GPU.
+Decode: attention from the oracle's own packed cache within max relative error 2e-3
+(per output row, ||o - r||_inf / ||r||_inf)."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, encode, packing
+from rotated_bit_kv_iq_b200 import binding as B
+from rotated_bit_kv_iq_b200 import inputs
+from tests._helpers import max_rel_err, upload_sequence
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TOL = 2e-3
+EXCLUSION_CAP = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from rotated_bit_kv_iq_b200 import build
+
+    build.build()
+    B.lib()
+
+
+def _params_dev(P):
+    return torch.from_numpy(np.ascontiguousarray(P)).to(DEV)
+
+
+def _export(cache, layer, kv, seq, t0, n):
+    codes = torch.empty((cache.n_kv_heads, n, 128), dtype=torch.uint8, device=DEV)
+    norms = torch.empty((cache.n_kv_heads, n), dtype=torch.int16, device=DEV)
+    B.iq_export_codes(cache, layer, kv, seq, t0, n, codes, norms)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), norms.cpu().numpy().view(np.uint16)
+
+
+def _check_codes(gpu_codes, gpu_n16, ref, label, cap=True):
+    near = ref["near"]
+    diff = gpu_codes != ref["codes"]
+    bad = diff & ~near
+    assert not bad.any(), f"{label}: {int(bad.sum())} code mismatches outside the boundary band"
+    # the 0.01% cap is a workload-level rate; small samples may hold a single excluded code
+    if cap:
+        assert near.sum() <= max(1, EXCLUSION_CAP * near.size), f"{label}: {int(near.sum())} excluded codes"
+    # an excluded code may only differ by one cell
+    assert np.all(np.abs(gpu_codes.astype(int) - ref["codes"].astype(int))[diff] == 1)
+    ulp = np.abs(gpu_n16.astype(np.int64) - ref["norm16"].astype(np.int64))
+    assert ulp.max() <= 1, f"{label}: norm off by {ulp.max()} ulp"
+
+
+# ------------------------------------------------------------------------- encode
+def test_encode_tiny_config_matches_oracle():
+    """Single head, 512 tokens, 2 outlier channels (the tiny workload); records checked byte by byte."""
+    T, P = 512, B.iq_init_rotation(inputs.ROTATION_SEED, 1, 1)
+    cache = B.PagedCache(1, 1, 512, 1)
+    xs, refs = {}, {}
+    for which in (0, 1):
+        xs[which] = inputs.kv_tokens(inputs.DATA_SEED, 0, 0, which, 0, T, n_outliers=2)
+        refs[which] = encode.encode(xs[which], P[0, 0])
+    k = torch.from_numpy(xs[0]).view(1, T, 1, 128).to(DEV)
+    v = torch.from_numpy(xs[1]).view(1, T, 1, 128).to(DEV)
+    start = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.iq_encode_append(cache, 0, k, v, start, _params_dev(P))
+    torch.cuda.synchronize()
+    for which in (0, 1):
+        codes, n16 = _export(cache, 0, which, 0, 0, T)
+        _check_codes(codes[0], n16[0], refs[which], f"kv={which}")
+        # byte-level format check: oracle packer on the GPU's codes where they were excluded
+        expect = np.where(refs[which]["near"], codes[0], refs[which]["codes"])
+        if which == 0:
+            got = cache.k_code_view()[0, 0, 0, :T].cpu().numpy()
+            np.testing.assert_array_equal(got, packing.pack_k_fast(expect))
+        else:
+            got = cache.v_code_view()[0, 0, 0, : T // 2].cpu().numpy()
+            np.testing.assert_array_equal(got, packing.pack_v_fast(expect))
+    assert cache.status.item() == 0
+
+
+def test_encode_ragged_paged_multi_sequence():
+    """3 sequences, 2 kv heads, 64-token pages in a shuffled pool, odd start positions."""
+    Hkv, ps, n_pages, L = 2, 64, 24, 2
+    P = B.iq_init_rotation(7, L, Hkv)
+    perm = inputs.page_permutation(3, n_pages)
+    table = torch.from_numpy(perm.reshape(3, 8)).to(DEV)
+    cache = B.PagedCache(L, Hkv, ps, n_pages, block_table=table)
+    starts = np.array([0, 5, 63], dtype=np.int32)
+    n_new = 77
+    layer = 1
+    X = {}
+    for which in (0, 1):
+        arr = np.zeros((3, n_new, Hkv, 128), dtype=np.float16)
+        for b in range(3):
+            for h in range(Hkv):
+                arr[b, :, h] = inputs.kv_tokens(11 + b, layer, h, which, 0, n_new, n_outliers=4, heavy_frac=0.05)
+        X[which] = arr
+    B.iq_encode_append(cache, layer, torch.from_numpy(X[0]).to(DEV), torch.from_numpy(X[1]).to(DEV),
+                       torch.from_numpy(starts).to(DEV), _params_dev(P))
+    torch.cuda.synchronize()
+    assert cache.status.item() == 0
+    for b in range(3):
+        for which in (0, 1):
+            codes, n16 = _export(cache, layer, which, b, int(starts[b]), n_new)
+            for h in range(Hkv):
+                ref = encode.encode(X[which][b, :, h], P[layer, h])
+                _check_codes(codes[h], n16[h], ref, f"b={b} h={h} kv={which}")
+
+
+def test_encode_single_token_appends_keep_partner_bytes():
+    """Decode-style appends of one token at a time: every V write is half a pair record."""
+    Hkv, L = 2, 1
+    P = B.iq_init_rotation(5, L, Hkv)
+    cache = B.PagedCache(L, Hkv, 64, 2)
+    T = 9
+    X = {w: np.stack([inputs.kv_tokens(21, 0, h, w, 0, T) for h in range(Hkv)], axis=1) for w in (0, 1)}
+    for t in range(T):
+        start = torch.full((2,), t, dtype=torch.int32, device=DEV)
+        k = torch.from_numpy(np.stack([X[0][t:t + 1]] * 2)).to(DEV)
+        v = torch.from_numpy(np.stack([X[1][t:t + 1]] * 2)).to(DEV)
+        B.iq_encode_append(cache, 0, k, v, start, _params_dev(P))
+    torch.cuda.synchronize()
+    for seq in (0, 1):
+        for which in (0, 1):
+            codes, n16 = _export(cache, 0, which, seq, 0, T)
+            for h in range(Hkv):
+                _check_codes(codes[h], n16[h], encode.encode(X[which][:, h], P[0, h]), f"seq={seq} h={h}")
+
+
+def test_encode_edge_values():
+    """Zero vector, saturating norm, fp16 subnormals, a single hot coordinate.  Constant vectors
+    rotate to exact zeros (= the middle boundary), so the exclusion-rate cap does not apply;
+    excluded codes must still be one of the two adjacent cells."""
+    P = B.iq_init_rotation(1, 1, 1)
+    x = np.zeros((6, 128), dtype=np.float16)
+    x[1] = 60000.0
+    x[2] = np.float16(6e-8)
+    x[3, 17] = -3.0
+    x[4] = inputs.kv_tokens(0, 0, 0, 0, 0, 1)[0]
+    x[5] = -x[4]
+    cache = B.PagedCache(1, 1, 16, 1)
+    t = torch.from_numpy(x).view(1, 6, 1, 128).to(DEV)
+    B.iq_encode_append(cache, 0, t, t, torch.zeros(1, dtype=torch.int32, device=DEV), _params_dev(P))
+    torch.cuda.synchronize()
+    ref = encode.encode(x, P[0, 0])
+    for which in (0, 1):
+        codes, n16 = _export(cache, 0, which, 0, 0, 6)
+        _check_codes(codes[0], n16[0], ref, f"edge kv={which}", cap=False)
+    assert n16[0][0] == 0 and np.all(codes[0][0] == 3)
+    assert n16[0][1] == 0x7BFF
+
+
+@pytest.mark.parametrize("heavy", [0.0, 0.01])
+def test_encode_ingest_layer_sampled(heavy):
+    """Ingest shape (32768 tokens x 8 kv heads, one layer, 1% Student-t tokens) in the bench's
+    launch configuration; sampled token ranges of every head checked against the oracle."""
+    Hkv, T, L = 8, 32768, 1
+    P = B.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)
+    cache = B.PagedCache(L, Hkv, T, 1)
+    X = {w: np.stack([inputs.kv_tokens(0, 0, h, w, 0, T, heavy_frac=heavy) for h in range(Hkv)], axis=1)[None]
+         for w in (0, 1)}
+    B.iq_encode_append(cache, 0, torch.from_numpy(X[0]).to(DEV), torch.from_numpy(X[1]).to(DEV),
+                       torch.zeros(1, dtype=torch.int32, device=DEV), _params_dev(P))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    for which in (0, 1):
+        for h in range(Hkv):
+            t0 = int(rng.integers(0, T - 1024))
+            codes, n16 = _export(cache, 0, which, 0, t0, 1024)
+            ref = encode.encode(X[which][0, t0:t0 + 1024, h], P[0, h])
+            _check_codes(codes[h], n16[h], ref, f"h={h} kv={which}")
+
+
+# ------------------------------------------------------------------------- decode
+def _oracle_cache(P_layer, layer, Hkv, T, seed=0, n_outliers=4):
+    """Oracle encodings of seeded K/V for all kv heads: dict of arrays (Hkv, T, ...)."""
+    kc, kn, vc, vn = [], [], [], []
+    for h in range(Hkv):
+        ek = encode.encode(inputs.kv_tokens(seed, layer, h, 0, 0, T, n_outliers=n_outliers), P_layer[h])
+        ev = encode.encode(inputs.kv_tokens(seed, layer, h, 1, 0, T, n_outliers=n_outliers), P_layer[h])
+        kc.append(ek["codes"]); kn.append(ek["norm16"]); vc.append(ev["codes"]); vn.append(ev["norm16"])
+    return np.stack(kc), np.stack(kn), np.stack(vc), np.stack(vn)
+
+
+def _decode(cache, layer, q, ctx, max_ctx, P):
+    Bn, Hq = q.shape[0], q.shape[1]
+    out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
+    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx), dtype=torch.uint8, device=DEV)
+    B.iq_decode_attention(cache, layer, q, torch.from_numpy(np.asarray(ctx, np.int32)).to(DEV), max_ctx,
+                          _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def test_decode_tiny_config():
+    """Single head, fp32 query, context 512 (group size 1)."""
+    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, 1)
+    kc, kn, vc, vn = _oracle_cache(P[0], 0, 1, 512, n_outliers=2)
+    cache = B.PagedCache(1, 1, 512, 1)
+    upload_sequence(cache, 0, [0], 0, kc[0], kn[0], vc[0], vn[0])
+    q = inputs.queries(0, 0, 1, 1, dtype="f32")
+    out = _decode(cache, 0, torch.from_numpy(q).to(DEV), [512], 512, P)
+    ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[0])
+    assert max_rel_err(out[0], ref) < TOL
+
+
+def test_decode_gqa4_llama_8k_full():
+    """Llama-3.1-8B-shaped layer: 32 q heads / 8 kv heads, context 8192, fp16 q; all heads."""
+    Hq, Hkv, T = 32, 8, 8192
+    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, Hkv)
+    kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, T)
+    cache = B.PagedCache(1, Hkv, T, 1)
+    for h in range(Hkv):
+        upload_sequence(cache, 0, [0], h, kc[h], kn[h], vc[h], vn[h])
+    q = inputs.queries(0, 0, 1, Hq)
+    out = _decode(cache, 0, torch.from_numpy(q).to(DEV), [T], T, P)
+    ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[0])
+    err = max_rel_err(out[0], ref)
+    assert err < TOL, err
+
+
+def test_decode_gqa8_qwen_32k_layer_full():
+    """Qwen3-30B-A3B-shaped layer: 32 q heads / 4 kv heads, context 32768 (a later layer index)."""
+    Hq, Hkv, T, L, layer = 32, 4, 32768, 3, 2
+    P = B.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)
+    kc, kn, vc, vn = _oracle_cache(P[layer], layer, Hkv, T)
+    cache = B.PagedCache(L, Hkv, T, 1)
+    for h in range(Hkv):
+        upload_sequence(cache, layer, [0], h, kc[h], kn[h], vc[h], vn[h])
+    q = inputs.queries(0, layer, 1, Hq)
+    out = _decode(cache, layer, torch.from_numpy(q).to(DEV), [T], T, P)
+    ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[layer])
+    err = max_rel_err(out[0], ref)
+    assert err < TOL, err
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_decode_ragged_paged_batch(G):
+    """Ragged contexts (0, 1, 15, 17, 300, 1000) over shuffled 64-token pages, every group size."""
+    Hkv = 2
+    Hq = G * Hkv
+    ctx = [0, 1, 15, 17, 300, 1000]
+    ps, maxp = 64, 16
+    n_pages = len(ctx) * maxp
+    P = B.iq_init_rotation(3, 1, Hkv)
+    perm = inputs.page_permutation(9, n_pages)
+    table_np = perm.reshape(len(ctx), maxp)
+    cache = B.PagedCache(1, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
+    refs = []
+    q = inputs.queries(4, 0, len(ctx), Hq)
+    for b, T in enumerate(ctx):
+        if T == 0:
+            refs.append(np.zeros((Hq, 128)))
+            continue
+        kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, T, seed=100 + b)
+        for h in range(Hkv):
+            upload_sequence(cache, 0, table_np[b], h, kc[h], kn[h], vc[h], vn[h])
+        refs.append(attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[0]))
+    out = _decode(cache, 0, torch.from_numpy(q).to(DEV), ctx, 1024, P)
+    assert np.all(out[0] == 0)
+    for b in range(1, len(ctx)):
+        assert max_rel_err(out[b], refs[b]) < TOL, (b, max_rel_err(out[b], refs[b]))
+    assert cache.status.item() == 0
+
+
+def test_decode_serving_batch_sampled():
+    """Batched serving shape: 16 sequences, contexts uniform in [2048, 32768], 64-token pages in a
+    shuffled pool, 32 q / 8 kv heads, one layer of the stack, launched as the bench launches it.
+    Three sampled sequences hold oracle data and are compared in full; the others hold
+    random codes."""
+    Bn, Hq, Hkv, ps = 16, 32, 8, 64
+    cfg = inputs.CONFIGS["serve_b16"]
+    ctx = inputs.context_lengths(inputs.DATA_SEED, Bn, cfg["ctx_lo"], cfg["ctx_hi"])
+    maxp = (int(ctx.max()) + ps - 1) // ps
+    n_pages = Bn * maxp
+    perm = inputs.page_permutation(inputs.DATA_SEED, n_pages)
+    table_np = perm.reshape(Bn, maxp)
+    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, Hkv)
+    cache = B.PagedCache(1, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
+    g = torch.Generator(device=DEV).manual_seed(0)
+    cache.k_codes.copy_(torch.randint(0, 256, cache.k_codes.shape, generator=g, device=DEV, dtype=torch.uint8))
+    cache.v_codes.copy_(torch.randint(0, 256, cache.v_codes.shape, generator=g, device=DEV, dtype=torch.uint8))
+    norms = (torch.rand(cache.k_norms.shape, generator=g, device=DEV) * 40 + 1).half().view(torch.int16)
+    cache.k_norms.copy_(norms)
+    cache.v_norms.copy_(norms.flip(0))
+    sampled = [0, 7, 15]
+    q = inputs.queries(inputs.DATA_SEED, 0, Bn, Hq)
+    refs = {}
+    for b in sampled:
+        kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, int(ctx[b]), seed=50 + b)
+        for h in range(Hkv):
+            upload_sequence(cache, 0, table_np[b], h, kc[h], kn[h], vc[h], vn[h])
+        refs[b] = attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[0])
+    out = _decode(cache, 0, torch.from_numpy(q).to(DEV), ctx, int(ctx.max()), P)
+    assert np.isfinite(out).all()
+    for b in sampled:
+        assert max_rel_err(out[b], refs[b]) < TOL, (b, max_rel_err(out[b], refs[b]))
+
+
+def test_encode_then_decode_end_to_end():
+    """GPU encode followed by GPU decode vs the oracle's encode + attention of the same inputs."""
+    Hq, Hkv, T = 16, 2, 3000
+    P = B.iq_init_rotation(2, 1, Hkv)
+    cache = B.PagedCache(1, Hkv, 3008, 1)
+    X = {w: np.stack([inputs.kv_tokens(31, 0, h, w, 0, T) for h in range(Hkv)], axis=1)[None] for w in (0, 1)}
+    B.iq_encode_append(cache, 0, torch.from_numpy(X[0]).to(DEV), torch.from_numpy(X[1]).to(DEV),
+                       torch.zeros(1, dtype=torch.int32, device=DEV), _params_dev(P))
+    q = inputs.queries(31, 0, 1, Hq)
+    out = _decode(cache, 0, torch.from_numpy(q).to(DEV), [T], T, P)
+    enc = {w: [encode.encode(X[w][0, :, h], P[0, h]) for h in range(Hkv)] for w in (0, 1)}
+    ref = attention.attention_rotated(
+        q[0].astype(np.float64),
+        np.stack([e["codes"] for e in enc[0]]), np.stack([e["norm16"] for e in enc[0]]),
+        np.stack([e["codes"] for e in enc[1]]), np.stack([e["norm16"] for e in enc[1]]), P[0])
+    assert max_rel_err(out[0], ref) < TOL
+
+
+def test_decode_flags_bad_context_and_pages():
+    """ctx above max_ctx is clamped and flagged; a block-table entry outside the pool is skipped
+    and flagged; the output stays finite."""
+    Hkv, Hq = 1, 4
+    P = B.iq_init_rotation(1, 1, Hkv)
+    table = torch.tensor([[0, 1], [2, 999]], dtype=torch.int32, device=DEV)
+    cache = B.PagedCache(1, Hkv, 64, 3, block_table=table)
+    cache.k_codes.zero_(); cache.v_codes.zero_(); cache.k_norms.zero_(); cache.v_norms.zero_()
+    q = torch.from_numpy(inputs.queries(0, 0, 2, Hq)).to(DEV)
+    out = _decode(cache, 0, q, [500, 100], 128, P)
+    assert np.isfinite(out).all()
+    st = cache.status.item()
+    assert st & B.IQ_DEVERR_CTX and st & B.IQ_DEVERR_PAGE
