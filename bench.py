@@ -144,16 +144,15 @@ class DecodeStack:
             self.B * self.Hkv * 2 * self.L * BYTES_PER_VECTOR_ENCODE
 
     def layer(self, l, stream=None):
-        Bd = self.Bd
-        Bd.iq_encode_append(self.cache, l, self.knew[l], self.vnew[l], self.new_pos, self.params, stream)
-        Bd.iq_decode_attention(self.cache, l, self.q[l], self.ctx_dev, self.max_ctx, self.params, self.out[l], self.ws,
-                               stream)
+        """One layer of the decode step: append the new token and attend (iq_decode_step)."""
+        self.Bd.iq_decode_step(self.cache, l, self.q[l], self.knew[l], self.vnew[l], self.ctx_dev, self.max_ctx,
+                               self.params, self.out[l], self.ws, stream)
 
     def step(self, stream=None):
         for l in range(self.L):
             self.layer(l, stream)
 
-    launches_per_layer = 3  # encode + split-K decode + combine
+    launches_per_layer = 2  # fused append + split-K attention, combine
 
 
 def time_graph(stack, steps, warmup, stream):
@@ -166,36 +165,18 @@ def time_graph(stack, steps, warmup, stream):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         stack.step(stream)
-    for _ in range(warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        graph.replay()
-    e1.record(stream)
-    e1.synchronize()
-    return e0.elapsed_time(e1) / steps, graph
-
-
-def time_decode_kernel(stack, steps, stream):
-    """Average duration of one decode-attention call (split-K kernel + combine) per layer."""
-    torch = stack.torch
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(stack.L)]
-    tot, n = 0.0, 0
-    Bd = stack.Bd
+    # replay() launches on torch's current stream: make it the timed stream
     with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         for _ in range(steps):
-            for l in range(stack.L):
-                evs[l][0].record(stream)
-                Bd.iq_decode_attention(stack.cache, l, stack.q[l], stack.ctx_dev, stack.max_ctx, stack.params,
-                                       stack.out[l], stack.ws, stream)
-                evs[l][1].record(stream)
-            stream.synchronize()
-            for a, b in evs:
-                tot += a.elapsed_time(b)
-                n += 1
-    return tot / n
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+    return e0.elapsed_time(e1) / steps, graph
 
 
 def time_e2e(stack, steps, warmup, stream):
@@ -214,9 +195,8 @@ def time_e2e(stack, steps, warmup, stream):
             dk[l].copy_(hk[l], non_blocking=True)
             dv[l].copy_(hv[l], non_blocking=True)
             dq[l].copy_(hq[l], non_blocking=True)
-            Bd.iq_encode_append(stack.cache, l, dk[l], dv[l], stack.new_pos, stack.params, stream)
-            Bd.iq_decode_attention(stack.cache, l, dq[l], stack.ctx_dev, stack.max_ctx, stack.params, stack.out[l],
-                                   stack.ws, stream)
+            Bd.iq_decode_step(stack.cache, l, dq[l], dk[l], dv[l], stack.ctx_dev, stack.max_ctx, stack.params,
+                              stack.out[l], stack.ws, stream)
             ho[l].copy_(stack.out[l], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -292,23 +272,25 @@ def oracle_decode_sample(seconds=12.0):
         ev = encode.encode(inputs.kv_tokens(0, 0, h, 1, 0, T), P[0, h])
         slices.append((h, ek, ev))
     q = inputs.queries(0, 0, 1, 32)[0].astype(np.float64)
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        h, ek, ev = slices[n % len(slices)]
-        attention.attention_rotated(q[h * G:(h + 1) * G], ek["codes"][None], ek["norm16"][None], ev["codes"][None],
-                                    ev["norm16"][None], P[0, h:h + 1])
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=1):  # one core: the figure reported as `cores`
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            h, ek, ev = slices[n % len(slices)]
+            attention.attention_rotated(q[h * G:(h + 1) * G], ek["codes"][None], ek["norm16"][None],
+                                        ev["codes"][None], ev["norm16"][None], P[0, h:h + 1])
+            n += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
     gbs = n * T * BYTES_PER_TOKEN_HEAD / el / 1e9
     return gbs, n, el
 
 
 def reference_arm(args):
     """--impl reference: the oracle on bounded samples of the headline workload."""
-    os.environ.setdefault("OMP_NUM_THREADS", "1")
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -339,6 +321,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--layers", type=int, default=0, help="override the stack depth (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -369,7 +353,8 @@ def main():
     Bd.lib()
     stream = torch.cuda.Stream(device=dev)
     cfg = inputs.CONFIGS[HEADLINE]
-    stack = DecodeStack(cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["n_layers"], [cfg["ctx"]],
+    n_layers = args.layers or cfg["n_layers"]
+    stack = DecodeStack(cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], n_layers, [cfg["ctx"]],
                         cfg["page_size"], dev, seed=rank)
 
     def barrier():
@@ -387,7 +372,9 @@ def main():
         ms = float(t.item())
     value = world * stack.bytes_per_step / (ms * 1e-3) / 1e9
 
-    kern_ms = time_decode_kernel(stack, max(2, args.steps // 2), stream)
+    # dominant kernel: the per-layer decode step (fused append + split-K attention, then the
+    # combine), timed inside the step graph: step time / layers
+    kern_ms = ms / stack.L
     layer_bytes = int(stack.ctx.sum()) * stack.Hkv * BYTES_PER_TOKEN_HEAD
     peak, peak_kind = _peaks()
     achieved = layer_bytes / (kern_ms * 1e-3) / 1e9
@@ -400,9 +387,10 @@ def main():
         "dtype": "f16 tensor-core inputs, f32 accumulate, 3-bit codes", "data": "synthetic",
         "config": {"workload": "qwen30b_32k: decode step (append + attend) B=1, 32 q / 4 kv heads, d=128, "
                                "48 layers, ctx 32768, packed 3-bit cache", "l2": "inputs larger than L2 (629 MB/step)",
-                   "graph": "48-layer step replayed as one CUDA graph", "bytes_per_step": stack.bytes_per_step},
+                   "graph": f"{stack.L}-layer step replayed as one CUDA graph", "layers": stack.L,
+                   "bytes_per_step": stack.bytes_per_step},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "decode attention (split-K + combine) per layer",
+                     "traffic": None, "kernel": "per-layer decode step (fused append + split-K attention, combine), CUDA-graph step time / layers",
                      "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
         "e2e": {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -426,7 +414,7 @@ def main():
         result["gpu_launches"] += 32 * args.steps
         torch.cuda.empty_cache()
 
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu:
         gbs, n, el = oracle_decode_sample(args.cpu_seconds)
         result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                                   "sample": f"{n} x (1 kv head, 8 q heads, 32768 tokens) decode slices in {el:.1f} s"}

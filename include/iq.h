@@ -82,6 +82,7 @@ typedef enum { IQ_F16 = 0, IQ_F32 = 1 } iq_dtype;
 #define IQ_DEVERR_POSITION 1u /* token position outside its sequence's pages */
 #define IQ_DEVERR_PAGE 2u     /* block-table entry outside [0, n_pages) */
 #define IQ_DEVERR_CTX 4u      /* context length outside [0, max_ctx] */
+#define IQ_DEVERR_TIMEOUT 8u  /* a bounded wait inside a kernel gave up (outputs undefined) */
 
 typedef struct {
   void* k_codes;                   /* device, see layout above */
@@ -152,6 +153,23 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
                               int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
                               const float* params_dev, float* out_dev, void* workspace_dev,
                               size_t workspace_bytes, iq_stream_t stream);
+
+/* Decode step: append one new token to every sequence and attend over it, in one kernel.
+ *   k_new_dev, v_new_dev: fp16 [batch][Hkv][128], the new token's K and V; it is encoded (as by
+ *                  iq_encode_append) into position ctx_len[b]-1 of sequence b.
+ *   Other arguments and the result as for iq_decode_attention over positions [0, ctx_len[b]);
+ *   ctx_len[b] >= 1 counts the new token.  Same result as iq_encode_append(start_pos =
+ *   ctx_len-1, n_new = 1) followed by iq_decode_attention, without the separate launch.
+ * Ordering: the kernel may start while the kernel issued just before it on the stream is
+ * still running (programmatic dependent launch).  Before waiting for that kernel it reads
+ * only ctx_len_dev, the block table and the cached records of positions < ctx_len-1 (it
+ * starts their bulk loads); q, k_new, v_new, params are read, and the cache, workspace and
+ * out are written, only after the wait.  So the immediately preceding kernel must not write
+ * ctx_len, the block table or older cache positions (host copies and earlier kernels may). */
+iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
+                         const void* k_new_dev, const void* v_new_dev, int32_t batch, int32_t n_q_heads,
+                         const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
+                         void* workspace_dev, size_t workspace_bytes, iq_stream_t stream);
 
 /* Read back tokens [t0, t0+n) of sequence `seq` in layer `layer` as canonical codes:
  *   codes_dev: uint8 [Hkv][n][128] (coordinate order), norms_dev: uint16 [Hkv][n] or NULL.

@@ -25,6 +25,7 @@ IQ_F32 = 1
 IQ_DEVERR_POSITION = 1
 IQ_DEVERR_PAGE = 2
 IQ_DEVERR_CTX = 4
+IQ_DEVERR_TIMEOUT = 8
 
 HEAD_DIM = 128
 K_RECORD_BYTES = 48
@@ -80,6 +81,8 @@ def lib():
         L.iq_decode_workspace_size.argtypes = [i32, i32, i32, i32]
         L.iq_decode_attention.restype = ctypes.c_int
         L.iq_decode_attention.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp, sz, vp]
+        L.iq_decode_step.restype = ctypes.c_int
+        L.iq_decode_step.argtypes = [P, i32, vp, ctypes.c_int, vp, vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_export_codes.restype = ctypes.c_int
         L.iq_export_codes.argtypes = [P, i32, i32, i32, i32, i32, vp, vp, vp]
         _lib = L
@@ -148,6 +151,18 @@ def iq_decode_attention(cache, layer, q, ctx_len, max_ctx, params, out, workspac
     _check("iq_decode_attention", lib().iq_decode_attention(
         ctypes.byref(cache.c), layer, _ptr(q), dtype, int(q.shape[0]), int(q.shape[1]), _ptr(ctx_len), int(max_ctx),
         _ptr(params), _ptr(out), _ptr(workspace), int(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def iq_decode_step(cache, layer, q, k_new, v_new, ctx_len, max_ctx, params, out, workspace, stream=None):
+    """Append one token per sequence (k_new, v_new: fp16 [batch][Hkv][128]) at position ctx_len-1 and
+    attend over [0, ctx_len)."""
+    import torch
+
+    dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
+    _check("iq_decode_step", lib().iq_decode_step(
+        ctypes.byref(cache.c), layer, _ptr(q), dtype, _ptr(k_new), _ptr(v_new), int(q.shape[0]), int(q.shape[1]),
+        _ptr(ctx_len), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 
 def iq_export_codes(cache, layer, kv, seq, t0, n, codes, norms=None, stream=None):

@@ -5,6 +5,29 @@
 
 #include "iq_internal.h"
 
+#include <cuda_runtime.h>
+#include <utility>
+
+namespace iq {
+// Launch with programmatic stream serialization (the kernel may start while the previous
+// kernel in the stream finishes; it synchronises with griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+}  // namespace iq
+
 namespace iq {
 
 // ------------------------------------------------------------------ rotation blocks
@@ -173,6 +196,142 @@ __device__ __forceinline__ int resolve_page(const LayerView& v, int b, int pos) 
     return -1;
   }
   return page;
+}
+
+}  // namespace iq
+
+namespace iq {
+
+// ------------------------------------------------------------------ mbarrier / bulk copy
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase of the given parity to complete, for at most ~1 s; on timeout flag
+// IQ_DEVERR_TIMEOUT and return false (the caller stops using the guarded data).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      if (status) atomicOr(status, IQ_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// One bulk copy global -> this CTA's shared memory (no multicast); completes on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+}  // namespace iq
+
+namespace iq {
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel lets the next kernel in the stream launch at once; it waits for the previous
+// kernel (griddepcontrol.wait) before reading data that kernel may have written or writing
+// anything.  Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Orders this thread's view of generic-proxy global writes before later async-proxy
+// (bulk copy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// ------------------------------------------------------------------ quantiser
+// code = #{ j : u > b_j } with u = sqrt(128) z / n, written with the three positive
+// thresholds t_j = b_j n / sqrt(128): magnitude class m = #{ |z| > t_j }, code = 4+m for
+// z > 0 and 3-m otherwise.  (Exact ties |z| = t_j are within rounding of a boundary.)
+__device__ __forceinline__ uint32_t quantise(float z, float t1, float t2, float t3) {
+  const float a = fabsf(z);
+  const uint32_t m = (uint32_t)(a > t1) + (uint32_t)(a > t2) + (uint32_t)(a > t3);
+  return z > 0.f ? 4u + m : 3u - m;
+}
+
+// ------------------------------------------------------------------ one-warp vector encoder
+// One warp encodes one fp16 vector (128 values at `src`) into the K (side 0) or V (side 1)
+// record of kv head `head` at (page, slot); lane l owns coordinates 4l..4l+3 (one SO(4)
+// block).  WHT stages on coordinate bits 2..6 run as shuffles; the lane's fused block matrix
+// is passed in.  K words are assembled with two shuffles; V records are written byte by byte
+// (only this token's bytes), so the other token of the pair is never touched.
+__device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __half* __restrict__ src, int head,
+                                                   int side, int page, int slot, const float Mp[4][4],
+                                                   const KernelConsts& kc) {
+  const int lane = threadIdx.x & 31;
+  const size_t hs = (size_t)page * v.n_kv_heads + head;
+  const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+  float x[4] = {f0.x, f0.y, f1.x, f1.y};
+  float ss = x[0] * x[0] + x[1] * x[1] + x[2] * x[2] + x[3] * x[3];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float n = sqrtf(ss);
+  warp_rotate_forward(x, Mp);
+  const float sc = n * 0.08838834764831845f;
+  const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
+  const uint32_t c0 = quantise(x[0], t1, t2, t3), c1 = quantise(x[1], t1, t2, t3);
+  const uint32_t c2 = quantise(x[2], t1, t2, t3), c3 = quantise(x[3], t1, t2, t3);
+  if (side == 0) {
+    // K chunk c = lanes 8c..8c+7; word w = lanes 8c+2w (low half) and 8c+2w+1 (high half);
+    // spare slots 24..31 = lanes 8c+6, 8c+7.
+    const uint32_t v16 = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
+    const uint32_t pair = v16 | (__shfl_xor_sync(0xffffffffu, v16, 1) << 16);
+    const uint32_t spare = __shfl_sync(0xffffffffu, pair, (lane & ~7) | 6);
+    const int w = (lane & 7) >> 1;
+    if ((lane & 1) == 0 && w < 3) {
+      const uint32_t word = pair | (((spare >> w) & 0x11111111u) << 3);
+      uint32_t* rec = reinterpret_cast<uint32_t*>(v.k_codes + (hs * v.page_size + slot) * K_REC);
+      rec[3 * (lane >> 3) + w] = word;
+    }
+  } else {
+    // V chunk g = lanes 4g..4g+3; first-token layout: word w holds lane 4g+w's codes at
+    // nibbles 0,1,4,5 and lane 4g+3's codes as spare bits; shifted 8 bits for the second token.
+    const uint32_t u = c0 | (c1 << 4) | (c2 << 16) | (c3 << 20);
+    const uint32_t spare = __shfl_sync(0xffffffffu, u, (lane & ~3) | 3);
+    const int w = lane & 3;
+    if (w < 3) {
+      const int par = slot & 1;
+      const uint32_t word = (u | (((spare >> w) & 0x00110011u) << 3)) << (8 * par);
+      uint8_t* rec = v.v_codes + (hs * (v.page_size / 2) + (slot >> 1)) * V_REC + 12 * (lane >> 2) + 4 * w;
+      rec[par] = (uint8_t)(word >> (8 * par));
+      rec[2 + par] = (uint8_t)(word >> (16 + 8 * par));
+    }
+  }
+  if (lane == 0) {
+    uint16_t* nrm = side ? v.v_norms : v.k_norms;
+    nrm[hs * v.page_size + slot] = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
+  }
 }
 
 }  // namespace iq

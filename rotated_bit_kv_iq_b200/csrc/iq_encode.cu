@@ -20,19 +20,12 @@ namespace iq {
 
 constexpr int ENC_THREADS = 128;
 
-// code = #{ j : u > b_j } with u = sqrt(128) z / n, written with the three positive
-// thresholds t_j = b_j n / sqrt(128): magnitude class m = #{ |z| > t_j }, code = 4+m for
-// z > 0 and 3-m otherwise.  (Exact ties |z| = t_j are within rounding of a boundary.)
-__device__ __forceinline__ uint32_t quantise(float z, float t1, float t2, float t3) {
-  const float a = fabsf(z);
-  const uint32_t m = (uint32_t)(a > t1) + (uint32_t)(a > t2) + (uint32_t)(a > t3);
-  return z > 0.f ? 4u + m : 3u - m;
-}
-
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int n_new,
               const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
   __shared__ float4 smat[NBLK][4];  // fused block matrices M'_k, row r as a float4
+  pdl_launch_dependents();
+  pdl_wait();
   const int b = blockIdx.z;
   const int head = blockIdx.y >> 1;
   const int side = blockIdx.y & 1;  // 0 = K, 1 = V
@@ -193,13 +186,45 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   }
 }
 
+// Small appends (decode steps): one warp per vector (see warp_encode_vector).
+constexpr int APP_WARPS = 4;
+__global__ void __launch_bounds__(APP_WARPS * 32)
+append_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int batch, int n_new,
+              const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const long vid = (long)blockIdx.x * APP_WARPS + (threadIdx.x >> 5);
+  const int side = (int)(vid & 1);
+  const long rest = vid >> 1;
+  const int head = (int)(rest % v.n_kv_heads);
+  const long rest2 = rest / v.n_kv_heads;
+  const int i_new = (int)(rest2 % n_new);
+  const int b = (int)(rest2 / n_new);
+  if (b >= batch) return;  // warp-uniform
+  const __half* src = side ? v_src : k_src;
+  if (src == nullptr) return;
+  const int pos = start_pos[b] + i_new;
+  const int page = resolve_page(v, b, pos);
+  if (page < 0) return;
+  float Mp[4][4];
+  fused_block_matrix(params_layer + ((size_t)head * NBLK + lane) * 8, Mp);
+  warp_encode_vector(v, src + (((size_t)b * n_new + i_new) * v.n_kv_heads + head) * D, head, side, page,
+                     pos % v.page_size, Mp, kc);
+}
+
 int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
                   const int32_t* start_pos, const float* params_layer, const KernelConsts& kc, void* stream) {
   if (batch == 0 || n_new == 0) return 0;
+  const long vectors = (long)batch * n_new * v.n_kv_heads * 2;
+  if (n_new <= 8) {  // decode-style appends: latency matters, not throughput
+    const long blocks = (vectors + APP_WARPS - 1) / APP_WARPS;
+    return (int)launch_pdl(append_kernel, dim3((unsigned)blocks), dim3(APP_WARPS * 32), 0, (cudaStream_t)stream, v,
+                           (const __half*)k, (const __half*)vsrc, batch, n_new, start_pos, params_layer, kc);
+  }
   dim3 grid((n_new + 1 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * 2, batch);
-  encode_kernel<<<grid, ENC_THREADS, 0, (cudaStream_t)stream>>>(v, (const __half*)k, (const __half*)vsrc, n_new,
-                                                                start_pos, params_layer, kc);
-  return (int)cudaGetLastError();
+  return (int)launch_pdl(encode_kernel, grid, dim3(ENC_THREADS), 0, (cudaStream_t)stream, v, (const __half*)k,
+                         (const __half*)vsrc, n_new, start_pos, params_layer, kc);
 }
 
 }  // namespace iq

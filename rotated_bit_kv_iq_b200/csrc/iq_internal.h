@@ -53,6 +53,9 @@ int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch
 int launch_decode(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads,
                   const int32_t* ctx_len, int max_ctx, const float* params_layer, float* out,
                   void* workspace, const KernelConsts& kc, void* stream);
+int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void* k_new, const void* v_new, int batch,
+                       int n_q_heads, const int32_t* ctx_len, int max_ctx, const float* params_layer, float* out,
+                       void* workspace, const KernelConsts& kc, void* stream);
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
                   uint16_t* norms, const KernelConsts& kc, void* stream);
 

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol(lib):
     hdr = open(os.path.join(ROOT, "include", "iq.h")).read()
     names = set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(iq_\w+)\s*\(", hdr, flags=re.M))
     assert {"iq_init_rotation", "iq_encode_append", "iq_decode_attention", "iq_decode_workspace_size",
-            "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version"} <= names
+            "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version", "iq_decode_step"} <= names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -119,6 +119,24 @@ def test_decode_rejects_bad_arguments(lib):
     assert _dec(_fake_cache(), ctx=None) == B.IQ_ERR_INVALID_ARG
     assert _dec(_fake_cache(), batch=-1) == B.IQ_ERR_INVALID_ARG
     assert _dec(_fake_cache(), max_ctx=-1) == B.IQ_ERR_INVALID_ARG
+
+
+@cpu_only
+def test_decode_step_rejects_bad_arguments(lib):
+    f = B.lib().iq_decode_step
+
+    def step(c, k=0x58000, v=0x5C000, max_ctx=32, hq=8, ws_bytes=1 << 30):
+        return f(ctypes.byref(c), 0, 0x50000, 0, k, v, 1, hq, 0x70000, max_ctx, 0x80000, 0x90000, 0xA0000, ws_bytes,
+                 None)
+
+    assert step(_fake_cache(), k=None) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), v=None) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), k=0x58008) == B.IQ_ERR_ALIGNMENT
+    assert step(_fake_cache(), max_ctx=0) == B.IQ_ERR_INVALID_ARG   # the new token needs a slot
+    assert step(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
+    assert step(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert step(_fake_cache(), ws_bytes=8) == B.IQ_ERR_WORKSPACE
+    assert step(_fake_cache(head_dim=64)) == B.IQ_ERR_UNSUPPORTED
 
 
 @cpu_only

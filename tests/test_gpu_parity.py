@@ -333,3 +333,89 @@ def test_decode_flags_bad_context_and_pages():
     assert np.isfinite(out).all()
     st = cache.status.item()
     assert st & B.IQ_DEVERR_CTX and st & B.IQ_DEVERR_PAGE
+
+
+# ------------------------------------------------------------------------- fused decode step
+def _step_case(G, ctx, ps, maxp, layer=0, L=1, seed=0, graph_layers=None):
+    """Oracle-filled cache of tokens 0..ctx-2 per sequence, new token ctx-1 given as fp16 input.
+    Returns (cache, P, q, knew, vnew, refs) with refs the oracle outputs and oracle encodings."""
+    Hkv = 2
+    Hq = G * Hkv
+    Bn = len(ctx)
+    n_pages = Bn * maxp
+    P = B.iq_init_rotation(seed + 3, L, Hkv)
+    perm = inputs.page_permutation(seed + 9, n_pages)
+    table_np = perm.reshape(Bn, maxp)
+    cache = B.PagedCache(L, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
+    cases = []
+    for l in range(L):
+        q = inputs.queries(seed + 4, l, Bn, Hq)
+        knew = np.zeros((Bn, Hkv, 128), np.float16)
+        vnew = np.zeros((Bn, Hkv, 128), np.float16)
+        refs = []
+        for b, T in enumerate(ctx):
+            kc, kn, vc, vn = _oracle_cache(P[l], l, Hkv, T, seed=200 + 10 * b + seed)
+            # the last token is appended by the call: upload only 0..T-2, keep its fp16 input
+            for h in range(Hkv):
+                knew[b, h] = inputs.kv_tokens(200 + 10 * b + seed, l, h, 0, T - 1, 1)[0]
+                vnew[b, h] = inputs.kv_tokens(200 + 10 * b + seed, l, h, 1, T - 1, 1)[0]
+                if T > 1:
+                    upload_sequence(cache, l, table_np[b], h, kc[h, :T - 1], kn[h, :T - 1], vc[h, :T - 1], vn[h, :T - 1])
+            refs.append((attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[l]), kc, kn, vc, vn))
+        cases.append((q, knew, vnew, refs))
+    return cache, P, cases
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_step_matches_oracle(G):
+    """Fused append + attention: new tokens at odd and even positions, page boundaries, ctx = 1."""
+    ctx = [1, 2, 64, 65, 129, 700]
+    cache, P, cases = _step_case(G, ctx, ps=64, maxp=11)
+    q, knew, vnew, refs = cases[0]
+    Bn, Hq = q.shape[0], q.shape[1]
+    out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
+    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 704), dtype=torch.uint8, device=DEV)
+    B.iq_decode_step(cache, 0, torch.from_numpy(q).to(DEV), torch.from_numpy(knew).to(DEV), torch.from_numpy(vnew).to(DEV),
+                     torch.tensor(ctx, dtype=torch.int32, device=DEV), 704, _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    o = out.cpu().numpy()
+    for b, T in enumerate(ctx):
+        ref, kc, kn, vc, vn = refs[b]
+        assert max_rel_err(o[b], ref) < TOL, (b, max_rel_err(o[b], ref))
+        for kv, (rc, rn) in enumerate([(kc, kn), (vc, vn)]):
+            codes, n16 = _export(cache, 0, kv, b, T - 1, 1)
+            for h in range(cache.n_kv_heads):
+                e = encode.encode(np.array([knew[b, h] if kv == 0 else vnew[b, h]]), P[0, h])
+                _check_codes(codes[h], n16[h], e, f"b={b} kv={kv}", cap=False)
+    assert cache.status.item() == 0
+
+
+def test_decode_step_chain_in_cuda_graph():
+    """Three layers of steps captured in one CUDA graph and replayed (the kernels overlap through
+    programmatic dependent launch); every layer's output and appended records must match."""
+    ctx = [300, 513]
+    L = 3
+    cache, P, cases = _step_case(8, ctx, ps=64, maxp=9, L=L, seed=5)
+    Bn, Hq = cases[0][0].shape[0], cases[0][0].shape[1]
+    qs = [torch.from_numpy(c[0]).to(DEV) for c in cases]
+    ks = [torch.from_numpy(c[1]).to(DEV) for c in cases]
+    vs = [torch.from_numpy(c[2]).to(DEV) for c in cases]
+    outs = [torch.zeros((Bn, Hq, 128), dtype=torch.float32, device=DEV) for _ in range(L)]
+    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 576), dtype=torch.uint8, device=DEV)
+    ctx_d = torch.tensor(ctx, dtype=torch.int32, device=DEV)
+    Pd = _params_dev(P)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for l in range(L):
+            B.iq_decode_step(cache, l, qs[l], ks[l], vs[l], ctx_d, 576, Pd, outs[l], ws, s)
+    for _ in range(2):  # replays are idempotent: the same token is appended again
+        with torch.cuda.stream(s):
+            g.replay()
+        s.synchronize()
+    for l in range(L):
+        o = outs[l].cpu().numpy()
+        for b in range(Bn):
+            ref = cases[l][3][b][0]
+            assert max_rel_err(o[b], ref) < TOL, (l, b, max_rel_err(o[b], ref))
+    assert cache.status.item() == 0
