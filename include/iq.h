@@ -171,6 +171,26 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
                          const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
                          void* workspace_dev, size_t workspace_bytes, iq_stream_t stream);
 
+/* Size of the fixed device scratch used by iq_decode_attention_noalloc (per device). */
+#define IQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* iq_decode_attention without a caller-provided workspace.  (The method has no counterpart:
+ * this entry point only changes where the split-K scratch lives.)
+ * For callers that may not allocate device memory -- plugins whose host owns every device
+ * allocation, and services that must not allocate after start-up.  Inputs, outputs and their
+ * meaning are those of iq_decode_attention; the split-K scratch is a fixed array of
+ * IQ_NOALLOC_SCRATCH_BYTES inside the library on each device (kept until the process exits).
+ * The call allocates nothing.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before capturing a
+ * stream.  Returns IQ_ERR_WORKSPACE when iq_decode_workspace_size(batch, n_q_heads, n_kv_heads,
+ * max_ctx) exceeds IQ_NOALLOC_SCRATCH_BYTES.  All calls on a device share the one array: calls
+ * that overlap on the GPU (other streams, or a second call before the first has finished on a
+ * stream that is not ordered after it) race on it.  Nothing in the array has to start zeroed. */
+iq_status iq_decode_attention_noalloc(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
+                                      int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev,
+                                      int32_t max_ctx, const float* params_dev, float* out_dev,
+                                      iq_stream_t stream);
+
 /* Read back tokens [t0, t0+n) of sequence `seq` in layer `layer` as canonical codes:
  *   codes_dev: uint8 [Hkv][n][128] (coordinate order), norms_dev: uint16 [Hkv][n] or NULL.
  *   kv: 0 = K pool, 1 = V pool.  Host-checked against the sequence capacity. */

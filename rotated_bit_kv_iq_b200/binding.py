@@ -83,6 +83,8 @@ def lib():
         L.iq_decode_attention.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_decode_step.restype = ctypes.c_int
         L.iq_decode_step.argtypes = [P, i32, vp, ctypes.c_int, vp, vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]
+        L.iq_decode_attention_noalloc.restype = ctypes.c_int
+        L.iq_decode_attention_noalloc.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp]
         L.iq_export_codes.restype = ctypes.c_int
         L.iq_export_codes.argtypes = [P, i32, i32, i32, i32, i32, vp, vp, vp]
         _lib = L
@@ -163,6 +165,19 @@ def iq_decode_step(cache, layer, q, k_new, v_new, ctx_len, max_ctx, params, out,
         ctypes.byref(cache.c), layer, _ptr(q), dtype, _ptr(k_new), _ptr(v_new), int(q.shape[0]), int(q.shape[1]),
         _ptr(ctx_len), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace),
         int(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+IQ_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def iq_decode_attention_noalloc(cache, layer, q, ctx_len, max_ctx, params, out, stream=None):
+    """iq_decode_attention with the library's fixed device scratch instead of a caller workspace."""
+    import torch
+
+    dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
+    _check("iq_decode_attention_noalloc", lib().iq_decode_attention_noalloc(
+        ctypes.byref(cache.c), layer, _ptr(q), dtype, int(q.shape[0]), int(q.shape[1]), _ptr(ctx_len), int(max_ctx),
+        _ptr(params), _ptr(out), _stream(stream)))
 
 
 def iq_export_codes(cache, layer, kv, seq, t0, n, codes, norms=None, stream=None):

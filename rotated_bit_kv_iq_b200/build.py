@@ -7,7 +7,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libiq.so")
-CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu"]
+CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu", "iq_noalloc.cu"]
 HOST_SOURCES = ["iq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
