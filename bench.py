@@ -135,7 +135,7 @@ class DecodeStack:
             L, B, 1, Hkv, 128)
         self.q = torch.stack([inputs.queries_device(seed, l, B, Hq, device=device) for l in range(L)])
         self.out = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=device)
-        self.ws = torch.empty(Bd.iq_decode_workspace_size(B, Hq, Hkv, self.max_ctx), dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(Bd.iq_decode_workspace_size(B, Hq, Hkv, self.max_ctx), dtype=torch.uint8, device=device)
         torch.cuda.synchronize()
 
     @property

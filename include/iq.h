@@ -32,7 +32,7 @@
  *
  * Cache layout (one pool per layer stacked along the first axis):
  *   k_codes  [L][n_pages][Hkv][page_size]   x 48-byte K records
- *   v_codes  [L][n_pages][Hkv][page_size/2] x 96-byte V records (token pairs)
+ *   v_codes  [L][n_pages][Hkv][page_size/16] x 768-byte V blocks (16 tokens each)
  *   k_norms, v_norms [L][n_pages][Hkv][page_size] binary16 norms
  *   Token t of sequence b lives on page
  *       block_table_dev[b * max_pages_per_seq + t / page_size]   (paged), or
@@ -45,8 +45,11 @@
  *   32-code chunk = 12 bytes = little-endian uint32 W0,W1,W2; for j in 0..7:
  *       bits [4j,4j+3) of Ww = code of slot 8w+j; bit 4j+3 of Ww = bit w of slot 24+j
  *   K record (per token): chunk c = 0..3, slot s -> coordinate 32c+s.
- *   V record (per token pair 2p,2p+1): chunk g = 0..7, slot s -> token 2p+(s%4>=2),
- *       coordinate 16g + 2*(s/4) + (s%2); even bytes belong to token 2p, odd to 2p+1.
+ *   V block (positions 16b..16b+15 of one sequence and kv head): 64 chunks, chunk
+ *       (g, tq, h) (g 0..7, tq 0..3, h 0..1) at byte 12*(2*(4g+tq)+h); its slot
+ *       8*(m/2) + 4*(m%2) + j (m 0..7, j 0..3) holds token 8*(j/2) + 2*tq + (j%2) of the block
+ *       at coordinate 16m + g + 8h.  Token u owns nibbles j, j+4 (spare bit included) of the
+ *       words of the 16 chunks with tq = (u%8)/2, j = 2*(u/8) + u%2, and nothing else.
  *   Norm: ||x||_2 of the fp16 input, rounded to binary16 (nearest even), saturating
  *       at 65504.
  *
@@ -83,6 +86,7 @@ typedef enum { IQ_F16 = 0, IQ_F32 = 1 } iq_dtype;
 #define IQ_DEVERR_PAGE 2u     /* block-table entry outside [0, n_pages) */
 #define IQ_DEVERR_CTX 4u      /* context length outside [0, max_ctx] */
 #define IQ_DEVERR_TIMEOUT 8u  /* a bounded wait inside a kernel gave up (outputs undefined) */
+#define IQ_DEVERR_WORKSPACE 16u /* decode workspace counters were not zero (outputs undefined) */
 
 typedef struct {
   void* k_codes;                   /* device, see layout above */
@@ -123,14 +127,20 @@ iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, 
  *   params_dev   : float32 [L][Hkv][32][2][4].
  * Per vector: norm (fp32 accumulate) -> WHT -> SO(4) blocks -> threshold search against
  * the 7 Lloyd-Max boundaries -> packed record + binary16 norm written at its slot.
- * Writes only the record bytes of the tokens it encodes (the other token of a V pair is
- * preserved).  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; IQ_DEVERR_POSITION /
+ * Writes only the bits of the tokens it encodes (the other tokens of a V block keep theirs;
+ * tokens of one block may come from different calls, but calls that overlap on the GPU must
+ * not append to the same block).  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; IQ_DEVERR_POSITION /
  * IQ_DEVERR_PAGE on the device. */
 iq_status iq_encode_append(const iq_cache* cache, int32_t layer, const void* k_dev, const void* v_dev,
                            int32_t batch, int32_t n_new, const int32_t* start_pos_dev,
                            const float* params_dev, iq_stream_t stream);
 
-/* Workspace bytes iq_decode_attention needs for these sizes (split-K partials). */
+/* Workspace bytes iq_decode_attention / iq_decode_step need for these sizes on the current
+ * device: per-(sequence, kv head) arrival counters followed by the split partials.  The
+ * counters must be zero when a call starts: zero-fill a new workspace once (e.g.
+ * cudaMemsetAsync); every call leaves them zero again, so the buffer can be reused by later
+ * calls on the same stream.  A call cut short by a device error (IQ_DEVERR_TIMEOUT) may leave
+ * them set: zero-fill again after one. */
 size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx);
 
 /* Decode attention over the packed cache of layer `layer`.
@@ -142,13 +152,17 @@ size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
  *                  the per-sequence capacity (page_size, or page_size*max_pages_per_seq).
  *   params_dev   : float32 [L][Hkv][32][2][4], the parameters used when encoding.
  *   out_dev      : float32 [batch][n_q_heads][128].
- *   workspace_dev: at least iq_decode_workspace_size(...) bytes, 256-byte aligned; its
- *                  contents need no initialisation and are scratch after the call.
+ *   workspace_dev: at least iq_decode_workspace_size(...) bytes, 256-byte aligned,
+ *                  zero-filled before its first use (see iq_decode_workspace_size); calls
+ *                  that overlap on the GPU must not share one.
+ *   batch        : at most 2048 (IQ_ERR_UNSUPPORTED above).
  * q head h reads kv head h / (n_q_heads / n_kv_heads); that group size must be 1, 2, 4 or 8.
  * out[b][h] = sum_t softmax_t(<q, K_t>/sqrt(128)) V_t with K_t, V_t the dequantised
  * vectors n * R^T c[codes] / sqrt(128), computed without forming them: q is rotated once,
  * scores and the value sum are formed in the rotated basis from codes and norms,
- * split-K partials are merged, and one inverse rotation is applied per output row. */
+ * split-K partials are merged, and one inverse rotation is applied per output row.
+ * Ordering: launched with programmatic dependent launch, but the kernel waits for the
+ * preceding kernel on the stream before it reads or writes anything. */
 iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
                               int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
                               const float* params_dev, float* out_dev, void* workspace_dev,
@@ -163,9 +177,10 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
  * Ordering: the kernel may start while the kernel issued just before it on the stream is
  * still running (programmatic dependent launch).  Before waiting for that kernel it reads
  * only ctx_len_dev, the block table and the cached records of positions < ctx_len-1 (it
- * starts their bulk loads); q, k_new, v_new, params are read, and the cache, workspace and
- * out are written, only after the wait.  So the immediately preceding kernel must not write
- * ctx_len, the block table or older cache positions (host copies and earlier kernels may). */
+ * starts their bulk loads); q, k_new, v_new and params are read, and the cache, workspace
+ * and out are written, only after the wait.  So the immediately preceding kernel must not
+ * write ctx_len, the block table or older cache positions (host copies and earlier kernels
+ * may). */
 iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
                          const void* k_new_dev, const void* v_new_dev, int32_t batch, int32_t n_q_heads,
                          const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
@@ -185,7 +200,8 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
  * stream.  Returns IQ_ERR_WORKSPACE when iq_decode_workspace_size(batch, n_q_heads, n_kv_heads,
  * max_ctx) exceeds IQ_NOALLOC_SCRATCH_BYTES.  All calls on a device share the one array: calls
  * that overlap on the GPU (other streams, or a second call before the first has finished on a
- * stream that is not ordered after it) race on it.  Nothing in the array has to start zeroed. */
+ * stream that is not ordered after it) race on it.  Each call clears the array's arrival
+ * counters (cudaMemsetAsync on its stream) before the kernel; nothing else has to start zeroed. */
 iq_status iq_decode_attention_noalloc(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
                                       int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev,
                                       int32_t max_ctx, const float* params_dev, float* out_dev,

@@ -13,18 +13,21 @@ words W_0, W_1, W_2:
 K record, one per token, 48 bytes = chunks c = 0..3 at bytes [12c, 12c+12);
     slot s of chunk c holds rotated coordinate 32c + s.
 
-V record, one per token pair (2p, 2p+1), 96 bytes = chunks g = 0..7 at bytes
-[12g, 12g+12); slot s of chunk g holds
-    token  2p + (1 if s mod 4 >= 2 else 0)
-    coord  16g + 2*floor(s/4) + (s mod 2)
-so every byte belongs to one token of the pair: even bytes to token 2p, odd bytes
-to token 2p+1.
+V block, one per 16 consecutive positions 16b .. 16b+15 of a (sequence, kv head), 768 bytes
+= 64 chunks; chunk (g, tq, h) with g in 0..7, tq in 0..3, h in 0..1 sits at bytes
+[12 q, 12 q + 12) with q = 2 (4 g + tq) + h.  Slot s = 8 floor(m/2) + 4 (m mod 2) + j of
+chunk (g, tq, h), for m in 0..7 and j in 0..3, holds
+    token  u = 8 floor(j/2) + 2 tq + (j mod 2)       (position 16b + u)
+    coord  x = 16 m + g + 8 h
+so token u owns nibbles j and j+4 (all four bits, spare bit included) of the three words of
+the sixteen chunks (g, tq(u), h): no other token has a bit there.
 """
 
 import numpy as np
 
 K_BYTES = 48
-V_PAIR_BYTES = 96
+V_BLOCK_TOKENS = 16
+V_BLOCK_BYTES = 768
 
 
 def pack_chunk(y):
@@ -58,8 +61,15 @@ def k_slot_coord(c, s):
     return 32 * c + s
 
 
-def v_slot_token_coord(g, s):
-    return (1 if (s % 4) >= 2 else 0), 16 * g + 2 * (s // 4) + (s % 2)
+def v_chunk_index(g, tq, h):
+    return 2 * (4 * g + tq) + h
+
+
+def v_slot_token_coord(g, tq, h, s):
+    """(token within the block, coordinate) held by slot s of V chunk (g, tq, h)."""
+    m = 2 * (s // 8) + (s % 8) // 4
+    j = s % 4
+    return 8 * (j // 2) + 2 * tq + (j % 2), 16 * m + g + 8 * h
 
 
 def pack_k(codes):
@@ -88,45 +98,63 @@ def unpack_k(records):
 
 
 def pack_v(codes):
-    """codes (T, 128) -> (ceil(T/2), 96) uint8 V records.  For odd T the last record's
-    odd bytes (the missing partner's) are left zero."""
+    """codes (T, 128) -> (ceil(T/16), 768) uint8 V blocks; slots of positions >= T are zero."""
     codes = np.asarray(codes)
     T = codes.shape[0]
-    P = (T + 1) // 2
-    out = np.zeros((P, V_PAIR_BYTES), dtype=np.uint8)
-    for p in range(P):
-        rec = bytearray()
+    NB = (T + 15) // 16
+    out = np.zeros((NB, V_BLOCK_BYTES), dtype=np.uint8)
+    for blk in range(NB):
+        rec = bytearray(V_BLOCK_BYTES)
         for g in range(8):
-            y = []
-            for s in range(32):
-                tok, coord = v_slot_token_coord(g, s)
-                t = 2 * p + tok
-                y.append(codes[t, coord] if t < T else 0)
-            rec += pack_chunk(y)
-        out[p] = np.frombuffer(bytes(rec), dtype=np.uint8)
+            for tq in range(4):
+                for h in range(2):
+                    y = []
+                    for s in range(32):
+                        u, x = v_slot_token_coord(g, tq, h, s)
+                        t = 16 * blk + u
+                        y.append(codes[t, x] if t < T else 0)
+                    q = v_chunk_index(g, tq, h)
+                    rec[12 * q : 12 * q + 12] = pack_chunk(y)
+        out[blk] = np.frombuffer(bytes(rec), dtype=np.uint8)
     return out
 
 
 def unpack_v(records, T=None):
     records = np.asarray(records, dtype=np.uint8)
-    P = records.shape[0]
+    NB = records.shape[0]
     if T is None:
-        T = 2 * P
+        T = 16 * NB
     codes = np.zeros((T, 128), dtype=np.uint8)
-    for p in range(P):
+    for blk in range(NB):
         for g in range(8):
-            y = unpack_chunk(records[p, 12 * g : 12 * g + 12].tobytes())
-            for s in range(32):
-                tok, coord = v_slot_token_coord(g, s)
-                t = 2 * p + tok
-                if t < T:
-                    codes[t, coord] = y[s]
+            for tq in range(4):
+                for h in range(2):
+                    q = v_chunk_index(g, tq, h)
+                    y = unpack_chunk(records[blk, 12 * q : 12 * q + 12].tobytes())
+                    for s in range(32):
+                        u, x = v_slot_token_coord(g, tq, h, s)
+                        t = 16 * blk + u
+                        if t < T:
+                            codes[t, x] = y[s]
     return codes
 
 
-def v_byte_owner():
-    """For each of the 96 bytes of a V record, which token of the pair (0 or 1) owns it."""
-    return np.arange(V_PAIR_BYTES) % 2
+def v_bit_owner():
+    """For each of the 6144 bits of a V block (byte-major, bit 0 first), the token (0..15)
+    whose code it stores, from the slot map and the chunk bit layout."""
+    owner = np.full(V_BLOCK_BYTES * 8, -1)
+    for g in range(8):
+        for tq in range(4):
+            for h in range(2):
+                base = 96 * v_chunk_index(g, tq, h)
+                for w in range(3):
+                    for nib in range(8):
+                        u_direct, _ = v_slot_token_coord(g, tq, h, 8 * w + nib)
+                        u_spare, _ = v_slot_token_coord(g, tq, h, 24 + nib)
+                        for bit in range(3):
+                            owner[base + 32 * w + 4 * nib + bit] = u_direct
+                        owner[base + 32 * w + 4 * nib + 3] = u_spare
+    return owner
 
 
 # --------------------------------------------------------------------- vectorised forms
@@ -155,8 +183,14 @@ def _words_chunk(words):
     return y.astype(np.uint8)
 
 
-_V_TOK = np.array([1 if (s % 4) >= 2 else 0 for s in range(32)])
-_V_COORD = np.array([[16 * g + 2 * (s // 4) + (s % 2) for s in range(32)] for g in range(8)])
+_VB_TOK = np.zeros((64, 32), dtype=np.int64)
+_VB_COORD = np.zeros((64, 32), dtype=np.int64)
+for _g in range(8):
+    for _tq in range(4):
+        for _h in range(2):
+            for _s in range(32):
+                _VB_TOK[v_chunk_index(_g, _tq, _h), _s], _VB_COORD[v_chunk_index(_g, _tq, _h), _s] = \
+                    v_slot_token_coord(_g, _tq, _h, _s)
 
 
 def pack_k_fast(codes):
@@ -176,20 +210,20 @@ def unpack_k_fast(records):
 def pack_v_fast(codes):
     codes = np.asarray(codes)
     T = codes.shape[0]
-    P = (T + 1) // 2
-    pad = np.zeros((2 * P, 128), dtype=codes.dtype)
+    NB = (T + 15) // 16
+    pad = np.zeros((16 * NB, 128), dtype=codes.dtype)
     pad[:T] = codes
-    pairs = pad.reshape(P, 2, 128)
-    y = pairs[:, _V_TOK[None, :], _V_COORD]  # (P, 8, 32)
-    return _chunk_words(y).reshape(P, 24).view("<u4").view(np.uint8).reshape(P, V_PAIR_BYTES)
+    blocks = pad.reshape(NB, 16, 128)
+    y = blocks[:, _VB_TOK, _VB_COORD]  # (NB, 64, 32)
+    return _chunk_words(y).reshape(NB, 192).view("<u4").view(np.uint8).reshape(NB, V_BLOCK_BYTES)
 
 
 def unpack_v_fast(records, T=None):
     records = np.ascontiguousarray(np.asarray(records, dtype=np.uint8))
-    P = records.shape[0]
+    NB = records.shape[0]
     if T is None:
-        T = 2 * P
-    y = _words_chunk(records.view("<u4").reshape(P, 8, 3))  # (P, 8, 32)
-    pairs = np.zeros((P, 2, 128), dtype=np.uint8)
-    pairs[:, _V_TOK[None, :], _V_COORD] = y
-    return pairs.reshape(2 * P, 128)[:T]
+        T = 16 * NB
+    y = _words_chunk(records.view("<u4").reshape(NB, 64, 3))  # (NB, 64, 32)
+    blocks = np.zeros((NB, 16, 128), dtype=np.uint8)
+    blocks[:, _VB_TOK, _VB_COORD] = y
+    return blocks.reshape(16 * NB, 128)[:T]

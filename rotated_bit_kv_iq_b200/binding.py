@@ -26,10 +26,12 @@ IQ_DEVERR_POSITION = 1
 IQ_DEVERR_PAGE = 2
 IQ_DEVERR_CTX = 4
 IQ_DEVERR_TIMEOUT = 8
+IQ_DEVERR_WORKSPACE = 16
 
 HEAD_DIM = 128
 K_RECORD_BYTES = 48
-V_PAIR_BYTES = 96
+V_BLOCK_TOKENS = 16
+V_BLOCK_BYTES = 768
 
 
 class IqError(RuntimeError):
@@ -146,7 +148,8 @@ def iq_decode_workspace_size(batch, n_q_heads, n_kv_heads, max_ctx):
 
 
 def iq_decode_attention(cache, layer, q, ctx_len, max_ctx, params, out, workspace, stream=None):
-    """q: [batch][Hq][128] fp16|fp32; out: fp32 [batch][Hq][128]; workspace: uint8 CUDA tensor."""
+    """q: [batch][Hq][128] fp16|fp32; out: fp32 [batch][Hq][128]; workspace: uint8 CUDA tensor,
+    zero-filled before its first use (torch.zeros); calls leave it ready for the next one."""
     import torch
 
     dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
@@ -217,7 +220,8 @@ class PagedCache:
         return self.k_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size, K_RECORD_BYTES)
 
     def v_code_view(self):
-        return self.v_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // 2, V_PAIR_BYTES)
+        return self.v_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // V_BLOCK_TOKENS,
+                                 V_BLOCK_BYTES)
 
     def k_norm_view(self):
         return self.k_norms.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size)

@@ -10,29 +10,53 @@
 
 namespace iq {
 
-// Centroids are handed to the kernels as binary16 values scaled by alpha.  alpha is chosen
-// so that alpha*c_k is within 2e-5 (relative) of a binary16 value for all eight levels
-// (plain binary16 rounding of c_k alone is off by up to 4.9e-4), which keeps the score and
-// value sums within ~1e-4 of the fp64 result.
-static const double kAlpha = 1.614664;
+// Centroids reach the tensor cores as int8 pairs: alpha8 * c_k ~ hi_k + lo_k / 254 with
+// hi_k, lo_k integers in [-127, 127].  alpha8 is the scale (searched on a 1e-5 grid below the
+// largest admissible value) that minimises the worst relative error over the four centroid
+// magnitudes; for the 3-bit N(0,1) codebook it is under 3e-6, far below the fp32 rounding of
+// the products that follow.
+static void int8_levels(const Codebook& cb, double& alpha8, int hi[8], int lo[8]) {
+  const double cmax = cb.level[7];
+  double best = 1e30;
+  alpha8 = 0.0;
+  for (long i = 0;; ++i) {
+    const double a = 127.49 / cmax - 1e-5 * (double)i;
+    if (a < 0.5 * 127.49 / cmax) break;
+    double err = 0.0;
+    bool ok = true;
+    for (int k = 4; k < 8; ++k) {
+      const double v = a * cb.level[k];
+      const double h = std::nearbyint(v);
+      const double l = std::nearbyint((v - h) * 254.0);
+      if (std::fabs(h) > 127.0 || std::fabs(l) > 127.0) { ok = false; break; }
+      err = std::fmax(err, std::fabs((h + l / 254.0) / a - cb.level[k]) / cb.level[k]);
+    }
+    if (ok && err < best) { best = err; alpha8 = a; }
+  }
+  for (int k = 0; k < 8; ++k) {
+    const double v = alpha8 * cb.level[k];
+    hi[k] = (int)std::nearbyint(v);
+    lo[k] = (int)std::nearbyint((v - hi[k]) * 254.0);
+  }
+}
 
 static KernelConsts make_consts() {
   const Codebook cb = compute_codebook();
   KernelConsts kc;
   for (int j = 0; j < 3; ++j) kc.bound_pos[j] = (float)cb.bound[4 + j];
-  uint32_t lo[2] = {0, 0}, hi[2] = {0, 0};
+  double alpha8;
+  int hi[8], lo[8];
+  int8_levels(cb, alpha8, hi, lo);
+  uint32_t h4[2] = {0, 0}, l4[2] = {0, 0};
   for (int k = 0; k < 8; ++k) {
-    const __half h = __float2half_rn((float)(kAlpha * cb.level[k]));
-    uint16_t bits;
-    std::memcpy(&bits, &h, 2);
-    lo[k >> 2] |= (uint32_t)(bits & 0xFF) << (8 * (k & 3));
-    hi[k >> 2] |= (uint32_t)(bits >> 8) << (8 * (k & 3));
+    h4[k >> 2] |= (uint32_t)(uint8_t)(int8_t)hi[k] << (8 * (k & 3));
+    l4[k >> 2] |= (uint32_t)(uint8_t)(int8_t)lo[k] << (8 * (k & 3));
   }
-  kc.lut_lo[0] = lo[0];
-  kc.lut_lo[1] = lo[1];
-  kc.lut_hi[0] = hi[0];
-  kc.lut_hi[1] = hi[1];
-  kc.inv_alpha = (float)(1.0 / kAlpha);
+  kc.lut_hi[0] = h4[0];
+  kc.lut_hi[1] = h4[1];
+  kc.lut_lo[0] = l4[0];
+  kc.lut_lo[1] = l4[1];
+  kc.alpha8 = (float)alpha8;
   return kc;
 }
 
@@ -63,7 +87,7 @@ static LayerView view(const iq_cache* c, int32_t layer) {
   LayerView v;
   const size_t per_layer_tokens = (size_t)c->n_pages * c->n_kv_heads * c->page_size;
   v.k_codes = (uint8_t*)c->k_codes + per_layer_tokens * K_REC * layer;
-  v.v_codes = (uint8_t*)c->v_codes + per_layer_tokens * K_REC * layer;  // 96 B per pair = 48 B per token
+  v.v_codes = (uint8_t*)c->v_codes + per_layer_tokens * K_REC * layer;  // 768 B per 16 tokens = 48 B per token
   v.k_norms = (uint16_t*)c->k_norms + per_layer_tokens * layer;
   v.v_norms = (uint16_t*)c->v_norms + per_layer_tokens * layer;
   v.block_table = c->block_table_dev;
@@ -148,6 +172,7 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
   if (batch < 0 || n_q_heads < 1 || max_ctx < 0 || !q_dev || !ctx_len_dev || !params_dev || !out_dev)
     return IQ_ERR_INVALID_ARG;
   if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
+  if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
@@ -175,6 +200,7 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
       !v_new_dev)
     return IQ_ERR_INVALID_ARG;
   if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
+  if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;

@@ -6,19 +6,26 @@
 // full-precision K/V are never built.  "RotorQuant" (sd114.wiki, "3. V 缓存的逆旋转修复"):
 // the value sum must be mapped back with the inverse rotation.
 //
-// Kernel 1 (split): grid (split, kv head, sequence).  Each CTA rotates the G = Hq/Hkv
-// queries of its kv head once (WHT + SO(4), one warp per query), then its warps walk
-// 16-token tiles of the CTA's context range.  Per tile one warp:
-//   * loads 48-byte K records of 16 tokens and 96-byte V records of 8 token pairs,
-//   * turns codes into binary16 centroid values with byte-permute table lookups
-//     (levels are stored scaled by alpha so that all eight are within 2e-5 of a binary16),
-//   * scores all G heads at once on the tensor cores: mma.m16n8k16 with the 16 tokens as
-//     M, the 128 rotated coordinates as K and (head, hi/lo half of q) as N,
-//   * runs the online softmax (running max, rescale on increase) with warp shuffles,
-//   * accumulates sum_t p_t n_v,t c[codes] with a second mma (coordinates as M, tokens as
-//     K, heads as N); P reaches the B-operand layout through movmatrix.
-// Warps merge (m, l, acc) in shared memory; the CTA writes one partial per query head.
-// Kernel 2 (combine): merges the splits, divides by l, rescales and applies R^T.
+// One kernel per call.  The work is the list of 32-token tiles of every (sequence, kv head)
+// group, group after group; CTA c takes the contiguous run [cT/N, (c+1)T/N) of the T tiles,
+// so every CTA gets the same number of tiles whatever the context lengths.  The run is cut
+// into segments at group boundaries.  In a segment the 8 warps take the tiles round robin;
+// each warp streams its tiles through its own ring of shared-memory slots with bulk copies
+// (one mbarrier per slot) and, per tile, on the tensor cores (mma.sync int8, m16n8k32):
+//   * scores: S^T = Q' K^T with the 8 query heads' int8 hi/lo rows as M (16 rows; a third
+//     int8 term of q is a second A operand), the 32 tokens as four n-tiles and the 128
+//     rotated coordinates as K; the K codes become
+//     int8 centroid values hi_k, lo_k (alpha8 c_k = hi_k + lo_k/254) by byte-permute table
+//     lookups, two per four codes;
+//   * online softmax per head on the lane that holds the head's scores; the V norm joins the
+//     probability (P' = 2^(s - m) n_v), which is quantised to int8 hi/lo with a scale per
+//     tile and head (127 / max P'), undone when the tile's value sums are accumulated;
+//   * values: O^T += V^T P' with the 128 coordinates as eight m-tiles, the 32 tokens as K and
+//     the heads as N; V blocks are laid out so that every A register is one table lookup.
+// s32 accumulators start at a magic constant so one float subtraction converts them.
+// At a segment end the warps' (m, l, O) are merged in shared memory and written as one
+// partial per (CTA, group); the CTA that completes a group's count merges its partials,
+// normalises and applies R^T (no second kernel).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -29,529 +36,700 @@
 
 namespace iq {
 
-constexpr int DEC_WARPS = 8;                    // every warp consumes; lane 0 of warp 0 also produces
+constexpr int DEC_WARPS = 8;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
-constexpr int STAGE_TOKENS = DEC_WARPS * TILE;  // 128 tokens: one 16-token tile per consumer warp
-constexpr int TILE_K = TILE * K_REC;            // 768 B of K records per tile
-constexpr int TILE_V = TILE / 2 * V_REC;        // 768 B of V records per tile
-constexpr int TILE_N = TILE * 2;                // 32 B of norms per tile
-constexpr int STAGE_K = 0;
-constexpr int STAGE_V = STAGE_K + DEC_WARPS * TILE_K;
-constexpr int STAGE_KN = STAGE_V + DEC_WARPS * TILE_V;
-constexpr int STAGE_VN = STAGE_KN + DEC_WARPS * TILE_N;
-constexpr int STAGE_BYTES = STAGE_VN + DEC_WARPS * TILE_N;  // 12800 B
-constexpr int NSTAGE = 6;
+constexpr int TT = 32;  // tokens per tile
+constexpr int SL_K = 0;                     // 32 K records (1536 B)
+constexpr int SL_V = SL_K + TT * K_REC;     // 2 V blocks (1536 B)
+constexpr int SL_KN = SL_V + 2 * V_BLK;     // 32 K norms (64 B)
+constexpr int SL_VN = SL_KN + TT * 2;       // 32 V norms (64 B)
+constexpr int SLOT_BYTES = SL_VN + TT * 2;  // 3200 B
+constexpr int NSLOT = 3;                    // tiles in flight per warp
+constexpr int HMAX = 8;                     // query heads per kv head (layout width)
+constexpr int SO_STRIDE = 132;              // floats per (warp, head) row of the merge buffer
+constexpr int QF_WORDS = 24;                // query fragment words per lane: 16 (hi, lo) + 8 (lo2)
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int G>
 struct DecSmem {
-  // Row strides chosen for conflict-free shared-memory access (see the uses):
-  static constexpr int SQ_STRIDE = 132;                      // floats per rotated-query row
-  static constexpr int SO_STRIDE = (G == 4) ? 132 : 134;     // floats per (warp, head) partial row (>= 131)
-  static constexpr int sq = NSTAGE * STAGE_BYTES;            // float [G][SQ_STRIDE] rotated queries
-  static constexpr int sm = sq + G * SQ_STRIDE * 4;          // float [DEC_WARPS][G] warp maxima
-  static constexpr int sl = sm + DEC_WARPS * G * 4;          // float [DEC_WARPS][G] warp sums
-  static constexpr int valid = sl + DEC_WARPS * G * 4;       // uint8 [NSTAGE] tile masks
-  static constexpr int abort_flag = valid + 16;              // int
-  static constexpr int bars = (abort_flag + 4 + 7) / 8 * 8;  // uint64 full[NSTAGE], empty[NSTAGE]
-  static constexpr int bytes = bars + 2 * NSTAGE * 8;
-  static_assert(DEC_WARPS * G * SO_STRIDE * 4 <= NSTAGE * STAGE_BYTES, "merge buffer reuses the stages");
-  static_assert(SO_STRIDE >= D + D / 32 - 1 + 1, "skewed row fits its stride");
-};
-
-struct Workspace {
-  float* part_o;   // [batch][Hq][n_split][128]
-  float2* part_ml; // [batch][Hq][n_split] (max in log2 units, sum of exp2)
+  static constexpr int ring = 0;                                          // [warp][slot] tiles
+  static constexpr int so = ring + DEC_WARPS * NSLOT * SLOT_BYTES;        // float [4][head][SO_STRIDE]
+  static constexpr int sm = so + 4 * HMAX * SO_STRIDE * 4;                // float [warp][head] maxima
+  static constexpr int sl = sm + DEC_WARPS * HMAX * 4;                    // float [warp][head] sums
+  static constexpr int qfrag = sl + DEC_WARPS * HMAX * 4;                 // uint32 [lane][QF_WORDS] query fragments
+  static constexpr int kappa = qfrag + 32 * QF_WORDS * 4;                 // float [head] score scales
+  static constexpr int sparams = kappa + HMAX * 4;                        // float [32][8] one head's parameters
+  static constexpr int flags = sparams + NBLK * 8 * 4;                    // int [4]
+  static constexpr int valid = flags + 16;                                // uint8 [warp][slot] half masks
+  static constexpr int bars = (valid + DEC_WARPS * NSLOT + 7) / 8 * 8;    // uint64 [warp][slot]
+  static constexpr int plan = bars + DEC_WARPS * NSLOT * 8;               // int [batch+1] tile prefix
+  static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(batch + 1); }
 };
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-SplitPlan plan_splits(int batch, int n_kv_heads, int max_ctx) {
-  SplitPlan p;
-  const int groups = batch * n_kv_heads;
-  const int target_ctas = 2 * 148;  // two resident CTAs per SM
-  int want = (target_ctas + groups - 1) / groups;
-  if (want < 1) want = 1;
-  int chunk = (max_ctx + want - 1) / want;
-  chunk = (chunk + STAGE_TOKENS - 1) / STAGE_TOKENS * STAGE_TOKENS;
-  if (chunk < STAGE_TOKENS) chunk = STAGE_TOKENS;
-  p.chunk = chunk;
-  p.n_split = max_ctx > 0 ? (max_ctx + chunk - 1) / chunk : 1;
-  return p;
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
+
+// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else
+// one, which leaves the other half of every SM free for the next kernel's CTAs to start
+// their loads early (programmatic dependent launch).
+int decode_ctas(int batch, int n_kv_heads, int max_ctx) {
+  const int n_sm = sm_count();
+  const long long tiles = (long long)batch * n_kv_heads * ((max_ctx + TT - 1) / TT);
+  const bool fits2 = 2 * (DecSmem::bytes(batch) + 1024) <= 228 * 1024;
+  const bool big = tiles >= (long long)n_sm * 2 * DEC_WARPS * 16;
+  return n_sm * ((fits2 && big) ? 2 : 1);
+}
+
+struct Workspace {
+  uint32_t* counters;  // [groups] arrivals per group; zero between calls
+  float2* part_ml;     // [slots][HMAX] (max in log2 units, sum of 2^(s-max))
+  float* part_o;       // [slots][HMAX][128]
+};
+
+static size_t ws_slots(int batch, int n_kv_heads) { return (size_t)2 * sm_count() + (size_t)batch * n_kv_heads; }
 
 size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx) {
-  SplitPlan p = plan_splits(batch, n_kv_heads, max_ctx);
-  const size_t rows = (size_t)batch * n_q_heads * p.n_split;
-  return align256(rows * D * sizeof(float)) + align256(rows * sizeof(float2));
+  (void)n_q_heads;
+  (void)max_ctx;
+  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
+  return align256(groups * 4) + align256(slots * HMAX * sizeof(float2)) + align256(slots * HMAX * D * sizeof(float));
 }
 
-static Workspace carve(void* ws, int batch, int n_q_heads, int n_split) {
+size_t decode_counter_bytes(int batch, int n_kv_heads) { return align256((size_t)batch * n_kv_heads * 4); }
+
+static Workspace carve(void* ws, int batch, int n_kv_heads) {
+  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
   Workspace w;
-  const size_t rows = (size_t)batch * n_q_heads * n_split;
-  w.part_o = (float*)ws;
-  w.part_ml = (float2*)((char*)ws + align256(rows * D * sizeof(float)));
+  char* p = (char*)ws;
+  w.counters = (uint32_t*)p;
+  p += align256(groups * 4);
+  w.part_ml = (float2*)p;
+  p += align256(slots * HMAX * sizeof(float2));
+  w.part_o = (float*)p;
   return w;
 }
 
-__device__ __forceinline__ int clamp_ctx(int c, int max_ctx, uint32_t* status) {
-  if (c < 0 || c > max_ctx) {
-    if (status && threadIdx.x == 0) atomicOr(status, IQ_DEVERR_CTX);
-    c = c < 0 ? 0 : max_ctx;
+struct DecArgs {
+  LayerView v;
+  const void* q;
+  int q_f32, n_q_heads, g_real, batch, max_ctx;
+  const int32_t* ctx_len;
+  const float* params_layer;
+  float* out;
+  Workspace ws;
+  const __half* k_new;
+  const __half* v_new;
+  KernelConsts kc;
+};
+
+// ------------------------------------------------------------------ work plan
+// pre[b] = tiles of sequences 0..b-1 (per kv head); every CTA builds the same table.
+__device__ void build_plan(const DecArgs& a, int* pre) {
+  const int B = a.batch;
+  const int per = (B + DEC_THREADS - 1) / DEC_THREADS;
+  const int lo = threadIdx.x * per, hi = min(B, lo + per);
+  int sum = 0;
+  for (int b = lo; b < hi; ++b) {
+    int c = a.ctx_len[b];
+    if (c < 0 || c > a.max_ctx) {
+      if (a.v.status && blockIdx.x == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
+      c = c < 0 ? 0 : a.max_ctx;
+    }
+    sum += (c + TT - 1) / TT;
   }
-  return c;
+  // block-wide exclusive scan of the per-thread sums
+  __shared__ int warp_tot[DEC_WARPS];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_tot[w];
+  int run = base + incl - sum;
+  for (int b = lo; b < hi; ++b) {
+    pre[b] = run;
+    int c = a.ctx_len[b];
+    c = c < 0 ? 0 : (c > a.max_ctx ? a.max_ctx : c);
+    run += (c + TT - 1) / TT;
+  }
+  if (threadIdx.x == DEC_THREADS - 1) pre[B] = run;
+  __syncthreads();
 }
 
-// Producer side: stream stage i (up to 8 tiles of 16 tokens) of this CTA's range into ring
-// slot s with bulk copies; runs of tiles on the same page with consecutive slots share one
-// copy per component.  Tiles past the context or on invalid pages are left out of the mask.
-__device__ __forceinline__ void issue_stage(const LayerView& v, int b, int kvh, int t_stage, int t_end,
-                                            uint8_t* stage, uint8_t* valid_mask, uint64_t* full_bar) {
-  int pages[DEC_WARPS], slots[DEC_WARPS];
-  uint32_t bytes = 0, mask = 0;
+__device__ __forceinline__ int seq_ctx(const DecArgs& a, int b) {
+  int c = a.ctx_len[b];
+  return c < 0 ? 0 : (c > a.max_ctx ? a.max_ctx : c);
+}
+
+// Group holding global tile x (x < T): sequence b, kv head, first global tile of the group.
+struct Seg {
+  int b, kvh, ntiles, lo, hi;  // tiles [lo, hi) of the group's ntiles lie in this CTA
+  int ctx;                     // context length of sequence b (clamped)
+  long long gstart;
+};
+__device__ __forceinline__ Seg segment_at(const DecArgs& a, const int* pre, int B, int Hkv, long long x, long long c1) {
+  int lo = 0, hi = B - 1;  // largest b with Hkv * pre[b] <= x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)Hkv * pre[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  // the largest such b has tiles (an empty b would share its prefix with b + 1, and x < T)
+  Seg s;
+  s.b = lo;
+  s.ntiles = pre[lo + 1] - pre[lo];
+  const long long off = x - (long long)Hkv * pre[s.b];
+  s.kvh = (int)(off / s.ntiles);
+  s.gstart = (long long)Hkv * pre[s.b] + (long long)s.kvh * s.ntiles;
+  s.lo = (int)(x - s.gstart);
+  s.hi = (int)min((long long)s.ntiles, c1 - s.gstart);
+  s.ctx = seq_ctx(a, s.b);
+  return s;
+}
+
+__device__ __forceinline__ long long cta_begin(int c, long long T, int n) { return (long long)c * T / n; }
+__device__ __forceinline__ int cta_of(long long x, long long T, int n) { return (int)(((x + 1) * n - 1) / T); }
+
+// ------------------------------------------------------------------ tile loads
+// Per-warp fetch cursor over the warp's tiles (round robin inside each segment of the
+// CTA's run).  All fields are warp-uniform.
+struct Cursor {
+  Seg s;
+  int i;        // next local tile of segment s for this warp
+  bool done;
+};
+
+__device__ __forceinline__ void cursor_normalise(Cursor& c, const DecArgs& a, const int* pre, int B, int Hkv, long long c1,
+                                                 int warp) {
+  while (!c.done && c.i >= c.s.hi) {
+    const long long nx = c.s.gstart + c.s.hi;
+    if (nx >= c1) { c.done = true; break; }
+    c.s = segment_at(a, pre, B, Hkv, nx, c1);
+    c.i = c.s.lo + warp;
+  }
+}
+
+template <bool FUSED>
+__device__ __forceinline__ bool is_new_token_tile(const Seg& s, int i) {
+  return FUSED && i == s.ntiles - 1;
+}
+
+// Issue the bulk copies of tile i of group (b, kvh) into slot `st` (lane 0 only).
+__device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, int i, int ctx, uint8_t* st,
+                                           uint8_t* valid, uint64_t* bar) {
+  int page[2], slot[2];
+  uint32_t mask = 0, bytes = 0;
 #pragma unroll
-  for (int j = 0; j < DEC_WARPS; ++j) {
-    const int t = t_stage + TILE * j;
-    pages[j] = -1;
-    slots[j] = 0;
-    if (t < t_end) {
-      pages[j] = resolve_page(v, b, t);
-      slots[j] = t % v.page_size;
-      if (pages[j] >= 0) {
-        mask |= 1u << j;
-        bytes += TILE_K + TILE_V + 2 * TILE_N;
+  for (int hh = 0; hh < 2; ++hh) {
+    const int t = TT * i + 16 * hh;
+    page[hh] = -1;
+    slot[hh] = 0;
+    if (t < ctx) {
+      page[hh] = resolve_page(v, b, t);
+      slot[hh] = t % v.page_size;
+      if (page[hh] >= 0) {
+        mask |= 1u << hh;
+        bytes += 16 * K_REC + V_BLK + 64;
       }
     }
   }
-  *valid_mask = (uint8_t)mask;
-  mbar_arrive_expect_tx(full_bar, bytes);
-  int j = 0;
-  while (j < DEC_WARPS) {
-    if (pages[j] < 0) { ++j; continue; }
-    int k = j + 1;
-    while (k < DEC_WARPS && pages[k] == pages[j] && slots[k] == slots[j] + TILE * (k - j)) ++k;
-    const int n = k - j;
-    const size_t hs = (size_t)pages[j] * v.n_kv_heads + kvh;
-    bulk_g2s(stage + STAGE_K + j * TILE_K, v.k_codes + (hs * v.page_size + slots[j]) * K_REC, n * TILE_K, full_bar);
-    bulk_g2s(stage + STAGE_V + j * TILE_V, v.v_codes + (hs * (v.page_size / 2) + slots[j] / 2) * V_REC, n * TILE_V,
-             full_bar);
-    bulk_g2s(stage + STAGE_KN + j * TILE_N, v.k_norms + hs * v.page_size + slots[j], n * TILE_N, full_bar);
-    bulk_g2s(stage + STAGE_VN + j * TILE_N, v.v_norms + hs * v.page_size + slots[j], n * TILE_N, full_bar);
-    j = k;
+  *valid = (uint8_t)mask;
+  mbar_arrive_expect_tx(bar, bytes);
+  const bool joined = mask == 3u && page[0] == page[1] && slot[1] == slot[0] + 16;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if (!((mask >> hh) & 1u)) continue;
+    if (joined && hh == 1) break;
+    const int n = joined ? 2 : 1;
+    const size_t hs = (size_t)page[hh] * v.n_kv_heads + kvh;
+    bulk_g2s(st + SL_K + 16 * K_REC * hh, v.k_codes + (hs * v.page_size + slot[hh]) * K_REC, n * 16 * K_REC, bar);
+    bulk_g2s(st + SL_V + V_BLK * hh, v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + slot[hh] / V_BLK_TOKENS) * V_BLK,
+             n * V_BLK, bar);
+    bulk_g2s(st + SL_KN + 32 * hh, v.k_norms + hs * v.page_size + slot[hh], n * 32, bar);
+    bulk_g2s(st + SL_VN + 32 * hh, v.v_norms + hs * v.page_size + slot[hh], n * 32, bar);
   }
 }
 
-// G: kernel layout width (4 or 8 query heads per kv head); g_real <= G query heads exist
-// (group sizes 1 and 2 run on the 4-wide layout with the unused columns zero).
-// FUSED: decode step -- the new token of each sequence (position ctx-1; fp16 K/V in
-// k_new/v_new, [batch][Hkv][128]) is encoded into the cache by the CTA whose range holds it
-// before that tile is loaded.  The cache stages not holding it are requested before waiting
-// for the previous kernel in the stream (their contents do not depend on it), so layer l+1's
-// loads overlap layer l's tail.
-template <int G, bool FUSED>
-__global__ void __launch_bounds__(DEC_THREADS, 2)
-decode_split_kernel(LayerView v, const void* __restrict__ q, int q_f32, int n_q_heads, int g_real,
-                    const int32_t* __restrict__ ctx_len, int max_ctx, int chunk, int n_split,
-                    const float* __restrict__ params_layer, Workspace ws, KernelConsts kc,
-                    const __half* __restrict__ k_new, const __half* __restrict__ v_new) {
+// The new token of sequence b (position ctx-1): encode K and V into the cache (whole warp).
+__device__ __forceinline__ void append_new_token(const DecArgs& a, int b, int kvh, int ctx) {
+  const int p = ctx - 1;
+  const int page = resolve_page(a.v, b, p);
+  if (page < 0) return;
+  const int lane = threadIdx.x & 31;
+  float Mp[4][4];
+  fused_block_matrix(a.params_layer + ((size_t)kvh * NBLK + lane) * 8, Mp);
+  const size_t off = ((size_t)b * a.v.n_kv_heads + kvh) * D;
+  warp_encode_vector(a.v, a.k_new + off, kvh, 0, page, p % a.v.page_size, Mp, a.kc);
+  warp_encode_vector(a.v, a.v_new + off, kvh, 1, page, p % a.v.page_size, Mp, a.kc);
+}
+
+// ------------------------------------------------------------------ per-tile compute
+struct WarpState {
+  float m, l;          // head g: running max of the scores s, sum of 2^(s - m)
+  float acc[8][4];     // coordinates 16j+g (+8) x heads 2t, 2t+1 (see the mma D layout)
+};
+
+__device__ __forceinline__ uint32_t pack4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  return prmt(prmt(x0, x1, 0x0040u), prmt(x2, x3, 0x0040u), 0x5410u);
+}
+
+__device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uint32_t vmask, int tok_end,
+                                             const uint32_t (&qa)[16], const uint32_t (&q2)[8], float kappa,
+                                             const KernelConsts& kc, WarpState& ws) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t LH0 = kc.lut_hi[0], LH1 = kc.lut_hi[1], LL0 = kc.lut_lo[0], LL1 = kc.lut_lo[1];
+  // ---- scores (head g; tokens 8nt + 2t + e as entry 2nt + e).  Rows of A: q hi (g), q lo
+  // (g + 8); a third product adds the q lo2 row against the centroid hi bytes.
+  float s[8];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(st + SL_K + (8 * nt + g) * K_REC + 12 * t);
+    uint32_t sel[4];
+    chunk_selectors(kw[0], kw[1], kw[2], sel);
+    int a1[4] = {kMagicI, kMagicI, kMagicI, kMagicI}, a2[4] = {kMagicI, kMagicI, kMagicI, kMagicI};
+    int a3[4] = {kMagicI, kMagicI, kMagicI, kMagicI};
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint32_t s0 = sel[cc], s1 = sel[cc] >> 16;
+      const uint32_t bh0 = prmt(LH0, LH1, s0), bh1 = prmt(LH0, LH1, s1);
+      imma16832(a1, qa[4 * cc], qa[4 * cc + 1], qa[4 * cc + 2], qa[4 * cc + 3], bh0, bh1, a1[0], a1[1], a1[2], a1[3]);
+      imma16832(a2, qa[4 * cc], qa[4 * cc + 1], qa[4 * cc + 2], qa[4 * cc + 3], prmt(LL0, LL1, s0), prmt(LL0, LL1, s1),
+                a2[0], a2[1], a2[2], a2[3]);
+      imma16832(a3, q2[2 * cc], 0u, q2[2 * cc + 1], 0u, bh0, bh1, a3[0], a3[1], a3[2], a3[3]);
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      // hh + (lo.c_hi + hi.c_lo)/254 + (lo.c_lo + lo2.c_hi)/254^2; each pair of raw
+      // accumulators sums to 2 * 1.5 * 2^23 + x, so one subtraction removes both offsets
+      const float x1 = (__int_as_float(a1[2 + e]) + __int_as_float(a2[e])) - 2.f * kMagicF;
+      const float x2 = (__int_as_float(a2[2 + e]) + __int_as_float(a3[e])) - 2.f * kMagicF;
+      s[2 * nt + e] = fmaf(fmaf(x2, 1.0f / 254.0f, x1), 1.0f / 254.0f, magic_to_float(a1[e]));
+    }
+  }
+  // ---- norms, masks, online softmax (head g)
+  float nv[8], mx = -CUDART_INF_F;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const int tok = 8 * nt + 2 * t;
+    const float2 nk = __half22float2(*reinterpret_cast<const __half2*>(st + SL_KN + 2 * tok));
+    const float2 nvv = __half22float2(*reinterpret_cast<const __half2*>(st + SL_VN + 2 * tok));
+    s[2 * nt] *= nk.x * kappa;
+    s[2 * nt + 1] *= nk.y * kappa;
+    nv[2 * nt] = nvv.x;
+    nv[2 * nt + 1] = nvv.y;
+  }
+  if (vmask != 3u || tok_end < TT) {  // a partial tile: tokens past the context or on bad pages
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int tok = 8 * (i >> 1) + 2 * t + (i & 1);
+      if (!((vmask >> (tok >> 4)) & 1u) || tok >= tok_end) {
+        s[i] = -CUDART_INF_F;
+        nv[i] = 0.f;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx = fmaxf(mx, s[i]);
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float m_new = fmaxf(ws.m, mx);
+  if (__any_sync(0xffffffffu, m_new > ws.m)) {
+    const float r = (m_new > ws.m) ? fast_exp2(ws.m - m_new) : 1.f;
+    ws.l *= r;
+    const float r0 = __shfl_sync(0xffffffffu, r, 8 * t), r1 = __shfl_sync(0xffffffffu, r, 8 * t + 4);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ws.acc[j][0] *= r0;
+      ws.acc[j][2] *= r0;
+      ws.acc[j][1] *= r1;
+      ws.acc[j][3] *= r1;
+    }
+    ws.m = m_new;
+  }
+  // P' = 2^(s - m) n_v, quantised per (tile, head) to int8 hi/lo with scale 127 / max P'
+  float pv[8], pmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float p = (ws.m == -CUDART_INF_F) ? 0.f : fast_exp2(s[i] - ws.m);
+    ws.l += p;
+    pv[i] = p * nv[i];
+    pmax = fmaxf(pmax, pv[i]);
+  }
+  pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 1));
+  pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
+  const float gam = pmax > 0.f ? 127.f / pmax : 0.f;
+  const float ig = pmax > 0.f ? pmax * (1.0f / 127.0f) : 0.f;
+  const float ig0 = __shfl_sync(0xffffffffu, ig, 8 * t), ig1 = __shfl_sync(0xffffffffu, ig, 8 * t + 4);
+  uint32_t hb[8], lb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float x = pv[i] * gam;  // in [0, 127]
+    hb[i] = round_low_bits(x);
+    const float h = __int_as_float((int)hb[i]) - kMagicF;
+    lb[i] = round_low_bits((x - h) * 254.f);
+  }
+  const uint32_t bh0 = pack4(hb[0], hb[1], hb[2], hb[3]), bh1 = pack4(hb[4], hb[5], hb[6], hb[7]);
+  const uint32_t bl0 = pack4(lb[0], lb[1], lb[2], lb[3]), bl1 = pack4(lb[4], lb[5], lb[6], lb[7]);
+  // ---- values: lane chunk (g, t) of each V block = 24 bytes at 24 * lane
+  uint32_t sv[4][4];  // [block*2 + h][word]
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    const uint2* vw = reinterpret_cast<const uint2*>(st + SL_V + V_BLK * blk + 24 * lane);
+    const uint2 w01 = vw[0], w23 = vw[1], w45 = vw[2];
+    chunk_selectors(w01.x, w01.y, w23.x, sv[2 * blk]);
+    chunk_selectors(w23.y, w45.x, w45.y, sv[2 * blk + 1]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int sh = 16 * (j & 1), w = j >> 1;
+    const uint32_t c0 = sv[0][w] >> sh, c1 = sv[1][w] >> sh, c2 = sv[2][w] >> sh, c3 = sv[3][w] >> sh;
+    const uint32_t h0 = prmt(LH0, LH1, c0), h1 = prmt(LH0, LH1, c1), h2 = prmt(LH0, LH1, c2), h3 = prmt(LH0, LH1, c3);
+    int d1[4], d2[4];
+    imma16832(d1, h0, h1, h2, h3, bh0, bh1, kMagicI, kMagicI, kMagicI, kMagicI);
+    imma16832(d2, h0, h1, h2, h3, bl0, bl1, kMagicI, kMagicI, kMagicI, kMagicI);
+    imma16832(d2, prmt(LL0, LL1, c0), prmt(LL0, LL1, c1), prmt(LL0, LL1, c2), prmt(LL0, LL1, c3), bh0, bh1, d2[0],
+              d2[1], d2[2], d2[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float tv = fmaf(magic_to_float(d2[e]), 1.0f / 254.0f, magic_to_float(d1[e]));
+      ws.acc[j][e] = fmaf(tv, (e & 1) ? ig1 : ig0, ws.acc[j][e]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ query rotation
+// Warp h rotates query head h of group (b, kvh), quantises it to int8 hi/lo with scale
+// gamma = 127 / max|q'| and writes it in mma A-fragment order: lane l holds coordinates
+// 4l..4l+3 = k-slots of chunk cc = (l/2) mod 4, fragment row 4h + l/8.
+__device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, int h, const float* prm,
+                                             uint32_t* qfrag, float* kappa) {
+  const int lane = threadIdx.x & 31;
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool live = h < a.g_real;
+  if (live) {
+    const size_t row = ((size_t)b * a.n_q_heads + (size_t)kvh * a.g_real + h) * D + 4 * lane;
+    if (a.q_f32) {
+      const float4 f = *reinterpret_cast<const float4*>((const float*)a.q + row);
+      x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+    } else {
+      const uint2 u = *reinterpret_cast<const uint2*>((const __half*)a.q + row);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+      x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+    }
+    float Mp[4][4];
+    fused_block_matrix(prm + lane * 8, Mp);
+    warp_rotate_forward(x, Mp);
+  }
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float gam = amax > 0.f ? 127.f / amax : 1.f;
+  // q' gamma = hi + lo/254 + lo2/254^2, each an int8 (residuals stay within +-0.5 of a unit)
+  uint32_t hi[4], lo[4], lo2[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float y = x[i] * gam;
+    hi[i] = round_low_bits(y);
+    const float r1 = (y - (__int_as_float((int)hi[i]) - kMagicF)) * 254.f;
+    lo[i] = round_low_bits(r1);
+    const float r2 = (r1 - (__int_as_float((int)lo[i]) - kMagicF)) * 254.f;
+    lo2[i] = round_low_bits(r2);
+  }
+  const int tq = lane >> 3, cc = (lane >> 1) & 3, e = lane & 1;
+  uint32_t* row = qfrag + (4 * h + tq) * QF_WORDS;
+  row[4 * cc + 2 * e] = pack4(hi[0], hi[1], hi[2], hi[3]);
+  row[4 * cc + 2 * e + 1] = pack4(lo[0], lo[1], lo[2], lo[3]);
+  row[16 + 2 * cc + e] = pack4(lo2[0], lo2[1], lo2[2], lo2[3]);
+  if (lane == 0) kappa[h] = live ? kLog2e / (128.f * gam * a.kc.alpha8) : 0.f;
+}
+
+// ------------------------------------------------------------------ the kernel
+template <bool FUSED>
+__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   pdl_launch_dependents();
   if (!FUSED) pdl_wait();  // a plain call may read anything the previous kernel wrote
-  using L = DecSmem<G>;
   extern __shared__ __align__(128) uint8_t smem[];
-  float(*sq)[L::SQ_STRIDE] = reinterpret_cast<float(*)[L::SQ_STRIDE]>(smem + L::sq);
-  float(*sm)[G] = reinterpret_cast<float(*)[G]>(smem + L::sm);
-  float(*sl)[G] = reinterpret_cast<float(*)[G]>(smem + L::sl);
-  uint8_t* valid = smem + L::valid;
-  int* abort_flag = reinterpret_cast<int*>(smem + L::abort_flag);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
-  uint64_t* empty = full + NSTAGE;
+  float(*so)[HMAX][SO_STRIDE] = reinterpret_cast<float(*)[HMAX][SO_STRIDE]>(smem + DecSmem::so);
+  float(*sm)[HMAX] = reinterpret_cast<float(*)[HMAX]>(smem + DecSmem::sm);
+  float(*sl)[HMAX] = reinterpret_cast<float(*)[HMAX]>(smem + DecSmem::sl);
+  uint32_t* qfrag = reinterpret_cast<uint32_t*>(smem + DecSmem::qfrag);
+  float* kappa = reinterpret_cast<float*>(smem + DecSmem::kappa);
+  int* flags = reinterpret_cast<int*>(smem + DecSmem::flags);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DecSmem::bars);
+  int* pre = reinterpret_cast<int*>(smem + DecSmem::plan);
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, tq = lane & 3;
-  const int ctx = clamp_ctx(ctx_len[b], max_ctx, v.status);
-  const int t_begin = split * chunk;
-  if (t_begin >= ctx) return;  // uniform over the CTA
-  const int t_end = min(t_begin + chunk, ctx);
-  const int n_stage = (t_end - t_begin + STAGE_TOKENS - 1) / STAGE_TOKENS;
-  const int p_new = ctx - 1;  // FUSED: position of the token appended by this call
-  const bool owner = FUSED && p_new >= t_begin && p_new < t_end;
-  const int s_new = owner ? (p_new - t_begin) / STAGE_TOKENS : -1;  // stage holding it
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], DEC_WARPS);
-    }
-    *abort_flag = 0;
+  const int Hkv = a.v.n_kv_heads, B = a.batch;
+  uint8_t* ring = smem + DecSmem::ring + warp * NSLOT * SLOT_BYTES;
+  uint8_t* valid = smem + DecSmem::valid + warp * NSLOT;
+  uint64_t* wbar = bars + warp * NSLOT;
+  if (lane == 0) {
+    for (int s = 0; s < NSLOT; ++s) mbar_init(&wbar[s], 1);
     mbar_fence_init();
   }
-  __syncthreads();
-  const bool producer = (threadIdx.x == 0);
-  if (producer) {
-    // Fill the ring: stages 0 .. NSTAGE-1 go out before any compute (the one holding a token
-    // appended by this call only once that token is written).
-    for (int i = 0; i < n_stage && i < NSTAGE; ++i)
-      if (i != s_new)
-        issue_stage(v, b, kvh, t_begin + i * STAGE_TOKENS, t_end, smem + i * STAGE_BYTES, &valid[i], &full[i]);
-  }
-  if (FUSED) pdl_wait();
+  build_plan(a, pre);  // ends with __syncthreads (barrier inits visible)
 
-  // Rotate the G queries of this kv head (one warp per query) while the first stages land,
-  // scaled so that score_log2 = n_k * <q', alpha*c[codes]>: q' = R q log2(e) / (128 alpha).
-  {
-    float Mp[4][4];
-    fused_block_matrix(params_layer + ((size_t)kvh * NBLK + lane) * 8, Mp);
-    if (owner && warp < 2) {
-      // FUSED: warp 0 appends the new K vector, warp 1 the new V vector, of this kv head.
-      const int page = resolve_page(v, b, p_new);
-      if (page >= 0)
-        warp_encode_vector(v, (warp == 0 ? k_new : v_new) + ((size_t)b * v.n_kv_heads + kvh) * D, kvh, warp, page,
-                           p_new % v.page_size, Mp, kc);
-    }
-    for (int h = warp; h < G; h += DEC_WARPS) {
-      const size_t row = ((size_t)b * n_q_heads + (size_t)kvh * g_real + h) * D + 4 * lane;
-      float x[4] = {0.f, 0.f, 0.f, 0.f};
-      if (h >= g_real) {
-        // no such query head: zero column
-      } else if (q_f32) {
-        const float4 f = *reinterpret_cast<const float4*>((const float*)q + row);
-        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
-      } else {
-        const uint2 u = *reinterpret_cast<const uint2*>((const __half*)q + row);
-        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-        x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+  const long long T = (long long)Hkv * pre[B];
+  const int n_cta = (int)min((long long)gridDim.x, T);
+  const int cta = blockIdx.x;
+  const long long c0 = cta < n_cta ? cta_begin(cta, T, n_cta) : 0;
+  const long long c1 = cta < n_cta ? cta_begin(cta + 1, T, n_cta) : 0;
+
+  // ---- prefetch: the warp's first tiles (a tile holding this call's new token waits)
+  bool waited = !FUSED;
+  bool aborted = false;
+  Cursor fc;
+  fc.done = c0 >= c1;
+  if (!fc.done) {
+    fc.s = segment_at(a, pre, B, Hkv, c0, c1);
+    fc.i = fc.s.lo + warp;
+    cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
+  }
+  int k_fetch = 0, k_done = 0, k_wait = 0;  // tiles issued, tiles passed, slots waited for
+  auto top_up = [&]() {
+    while (!fc.done && !aborted && k_fetch < k_done + NSLOT) {
+      const int ctx = fc.s.ctx;
+      if (is_new_token_tile<FUSED>(fc.s, fc.i)) {
+        if (!waited) break;
+        append_new_token(a, fc.s.b, fc.s.kvh, ctx);
+        __syncwarp();
+        fence_proxy_async_global();  // the appended records before the bulk reads of them
       }
-      warp_rotate_forward(x, Mp);
-      const float sc = kLog2e * kc.inv_alpha * (1.0f / 128.0f);
-      *reinterpret_cast<float4*>(&sq[h][4 * lane]) = make_float4(x[0] * sc, x[1] * sc, x[2] * sc, x[3] * sc);
+      const int sl_i = k_fetch % NSLOT;
+      if (lane == 0)
+        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i]);
+      ++k_fetch;
+      fc.i += DEC_WARPS;
+      cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
     }
+  };
+  top_up();
+  // rotation parameters of the first segment's kv head into shared memory (they are not
+  // written by the kernel this one may overlap)
+  float* sprm = reinterpret_cast<float*>(smem + DecSmem::sparams);
+  int sprm_kvh = -1;
+  if (c0 < c1) {
+    sprm_kvh = segment_at(a, pre, B, Hkv, c0, c1).kvh;
+    if (threadIdx.x < NBLK * 2)
+      reinterpret_cast<float4*>(sprm)[threadIdx.x] =
+          reinterpret_cast<const float4*>(a.params_layer + (size_t)sprm_kvh * NBLK * 8)[threadIdx.x];
   }
-  __syncthreads();
-  if (owner && producer) {
-    // The appended token's record is in global memory (visible CTA-wide after the barrier);
-    // order it before the bulk-copy reads of its stage (now or in a later refill).
-    fence_proxy_async_global();
-    if (s_new < NSTAGE)
-      issue_stage(v, b, kvh, t_begin + s_new * STAGE_TOKENS, t_end, smem + s_new * STAGE_BYTES, &valid[s_new],
-                  &full[s_new]);
+  if (FUSED) {
+    pdl_wait();
+    waited = true;
+    top_up();
   }
 
-  {
-    // Query B-fragments (k16 x n8 per k-chunk c): MMA k index 2tq+e <-> coordinate
-    // 32tq+4c+e, k index 2tq+8+e <-> 32tq+4c+2+e.  Columns: G=4 -> (head n/2, hi|lo = n%2);
-    // G=8 -> tile 0 = hi halves of heads 0..7, tile 1 = lo halves.
-    constexpr int NT = G / 4;
-    uint32_t qb[NT][8][2];
+  // ---- outputs of groups with no tiles (empty context): zeros
+  const int n_groups = B * Hkv;
+  for (int gi = cta; gi < n_groups; gi += gridDim.x) {
+    const int b = gi / Hkv, kvh = gi % Hkv;
+    if (pre[b + 1] != pre[b]) continue;
+    for (int idx = threadIdx.x; idx < a.g_real * (D / 4); idx += DEC_THREADS) {
+      const int h = idx / (D / 4), c4 = idx % (D / 4);
+      float4* dst = reinterpret_cast<float4*>(a.out + ((size_t)b * a.n_q_heads + (size_t)kvh * a.g_real + h) * D) + c4;
+      *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+
+  // ---- segments of this CTA's run
+  long long x = c0;
+  while (x < c1) {
+    const Seg seg = segment_at(a, pre, B, Hkv, x, c1);
+    const int gid = seg.b * Hkv + seg.kvh;
+    __syncthreads();  // previous segment's readers of qfrag / merge buffer are done
+    if (seg.kvh != sprm_kvh) {
+      sprm_kvh = seg.kvh;
+      if (threadIdx.x < NBLK * 2)
+        reinterpret_cast<float4*>(sprm)[threadIdx.x] =
+            reinterpret_cast<const float4*>(a.params_layer + (size_t)sprm_kvh * NBLK * 8)[threadIdx.x];
+      __syncthreads();
+    }
+    rotate_query(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
+    __syncthreads();
+    uint32_t qa[16], q2[8];
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(qfrag + lane * QF_WORDS);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = src[i];
+        qa[4 * i] = u.x; qa[4 * i + 1] = u.y; qa[4 * i + 2] = u.z; qa[4 * i + 3] = u.w;
+      }
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int head = (G == 4) ? (g >> 1) : g;
-        const bool lo_part = (G == 4) ? (g & 1) : (nt == 1);
-        // float4 reads: with a 132-float row the 8 lanes of each wavefront hit distinct banks
-        const float4 x4 = *reinterpret_cast<const float4*>(&sq[head][32 * tq + 4 * c]);
-        const float xs[4] = {x4.x, x4.y, x4.z, x4.w};
-        float vals[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float hi = __half2float(__float2half_rn(xs[e]));
-          vals[e] = lo_part ? (xs[e] - hi) : xs[e];
-        }
-        qb[nt][c][0] = pack_half2(vals[0], vals[1]);
-        qb[nt][c][1] = pack_half2(vals[2], vals[3]);
+      for (int i = 0; i < 2; ++i) {
+        const uint4 u = src[4 + i];
+        q2[4 * i] = u.x; q2[4 * i + 1] = u.y; q2[4 * i + 2] = u.z; q2[4 * i + 3] = u.w;
       }
     }
-
-    constexpr int HS = G / 4;  // head slots per thread: G=4 -> head tq; G=8 -> heads 2tq, 2tq+1
-    float m_run[HS], l_run[HS];
-    float acc[8][4];
-#pragma unroll
-    for (int s = 0; s < HS; ++s) { m_run[s] = -CUDART_INF_F; l_run[s] = 0.f; }
+    const float kap = kappa[lane >> 2];
+    WarpState st;
+    st.m = -CUDART_INF_F;
+    st.l = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
-    const uint32_t lut_lo[2] = {kc.lut_lo[0], kc.lut_lo[1]};
-    const uint32_t lut_hi[2] = {kc.lut_hi[0], kc.lut_hi[1]};
+      for (int e = 0; e < 4; ++e) st.acc[j][e] = 0.f;
 
-    for (int i = 0; i < n_stage; ++i) {
-      // Refill: the slot of stage i-2 takes stage i-2+NSTAGE once every warp has left it.
-      if (producer && i >= 2 && i - 2 + NSTAGE < n_stage) {
-        const int j = i - 2, sj = j % NSTAGE;
-        if (mbar_wait(&empty[sj], (j / NSTAGE) & 1, v.status))
-          issue_stage(v, b, kvh, t_begin + (j + NSTAGE) * STAGE_TOKENS, t_end, smem + sj * STAGE_BYTES, &valid[sj],
-                      &full[sj]);
-        else
-          *abort_flag = 1;
+    const int ctx = seg.ctx;
+    for (int i = seg.lo + warp; i < seg.hi; i += DEC_WARPS) {
+      const int sl_i = k_done % NSLOT;
+      if (!aborted) {
+        const bool landed = __all_sync(0xffffffffu, mbar_wait(&wbar[sl_i], (k_done / NSLOT) & 1, a.v.status));
+        if (landed) ++k_wait; else aborted = true;
       }
-      const int s = i % NSTAGE;
-      // every lane polls; the verdict is made warp-uniform before any warp-wide instruction
-      const bool landed = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / NSTAGE) & 1, v.status));
-      if (!landed) {
-        if (lane == 0) *abort_flag = 1;
-        break;
-      }
-      const int t0 = t_begin + i * STAGE_TOKENS + TILE * warp;
-      if (t0 < t_end && ((valid[s] >> warp) & 1)) {
-        const uint8_t* st = smem + s * STAGE_BYTES;
-        const uint32_t* kA = reinterpret_cast<const uint32_t*>(st + STAGE_K + warp * TILE_K + g * K_REC + tq * 12);
-        const uint32_t* kB = kA + 8 * K_REC / 4;
-        const uint32_t* vA = reinterpret_cast<const uint32_t*>(st + STAGE_V + warp * TILE_V + tq * V_REC + g * 12);
-        const uint32_t* vB = vA + 4 * V_REC / 4;
-        const uint16_t* knp = reinterpret_cast<const uint16_t*>(st + STAGE_KN + warp * TILE_N);
-        const uint16_t* vnp = reinterpret_cast<const uint16_t*>(st + STAGE_VN + warp * TILE_N);
-        const bool okA = t0 + g < t_end, okB = t0 + g + 8 < t_end;
-        const float nkA = half_bits_to_float(knp[g]), nkB = half_bits_to_float(knp[g + 8]);
-        const float nvA = half_bits_to_float(vnp[g]), nvB = half_bits_to_float(vnp[g + 8]);
-
-        // ---- scores: S[token][col] over 8 k-chunks
-        // two independent accumulation chains (even / odd k-chunks) halve the mma latency chain
-        float sc[NT][4], sc2[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
-        {
-          uint32_t selA[4], selB[4];
-          chunk_selectors(kA[0], kA[1], kA[2], selA);
-          chunk_selectors(kB[0], kB[1], kB[2], selB);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t sA = (c & 1) ? (selA[c >> 1] >> 16) : selA[c >> 1];
-            const uint32_t sB = (c & 1) ? (selB[c >> 1] >> 16) : selB[c >> 1];
-            uint32_t lA, hA, lB, hB;
-            lut4(sA, lut_lo, lut_hi, lA, hA);
-            lut4(sB, lut_lo, lut_hi, lB, hB);
-            const uint32_t a0 = pair01(lA, hA), a2 = pair23(lA, hA);
-            const uint32_t a1 = pair01(lB, hB), a3 = pair23(lB, hB);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              mma16816((c & 1) ? sc2[nt] : sc[nt], a0, a1, a2, a3, qb[nt][c][0], qb[nt][c][1]);
-          }
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
-        }
-
-        // ---- online softmax per head slot; sv[slot][0] = token g, sv[slot][1] = token g+8
-        float sv[HS][2];
-        if (G == 4) {
-          sv[0][0] = sc[0][0] + sc[0][1];
-          sv[0][1] = sc[0][2] + sc[0][3];
-        } else {
-          sv[0][0] = sc[0][0] + sc[NT - 1][0];
-          sv[0][1] = sc[0][2] + sc[NT - 1][2];
-          sv[HS - 1][0] = sc[0][1] + sc[NT - 1][1];
-          sv[HS - 1][1] = sc[0][3] + sc[NT - 1][3];
-        }
-        float p[HS][2];
-#pragma unroll
-        for (int hsl = 0; hsl < HS; ++hsl) {
-          const float sa = okA ? sv[hsl][0] * nkA : -CUDART_INF_F;
-          const float sb = okB ? sv[hsl][1] * nkB : -CUDART_INF_F;
-          float mx = fmaxf(sa, sb);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float m_new = fmaxf(m_run[hsl], mx);
-          if (m_new > m_run[hsl]) {
-            const float r = fast_exp2(m_run[hsl] - m_new);
-            l_run[hsl] *= r;
-            if (G == 4) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[j][e] *= r;
-            } else {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                acc[j][hsl] *= r;
-                acc[j][hsl + 2] *= r;
-              }
-            }
-            m_run[hsl] = m_new;
-          }
-          const float pa = fast_exp2(sa - m_new), pb = fast_exp2(sb - m_new);
-          l_run[hsl] += pa + pb;
-          p[hsl][0] = okA ? pa * nvA : 0.f;
-          p[hsl][1] = okB ? pb * nvB : 0.f;
-        }
-
-        // ---- P in the S layout (row = token, cols 2tq, 2tq+1) -> B operand via movmatrix
-        uint32_t rowA, rowB;
-        if (G == 4) {
-          const float hiA = __half2float(__float2half_rn(p[0][0]));
-          const float hiB = __half2float(__float2half_rn(p[0][1]));
-          rowA = pack_half2(hiA, p[0][0] - hiA);
-          rowB = pack_half2(hiB, p[0][1] - hiB);
-        } else {
-          rowA = pack_half2(p[0][0], p[HS - 1][0]);
-          rowB = pack_half2(p[0][1], p[HS - 1][1]);
-        }
-        const uint32_t bp0 = movmatrix_trans(rowA), bp1 = movmatrix_trans(rowB);
-
-        // ---- values: O^T[coord][col] += V^T[coord][token] P^T[token][col]
-        {
-          uint32_t selA[4], selB[4];
-          chunk_selectors(vA[0], vA[1], vA[2], selA);
-          chunk_selectors(vB[0], vB[1], vB[2], selB);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t sA = (j & 1) ? (selA[j >> 1] >> 16) : selA[j >> 1];
-            const uint32_t sB = (j & 1) ? (selB[j >> 1] >> 16) : selB[j >> 1];
-            uint32_t lA, hA, lB, hB;
-            lut4(sA, lut_lo, lut_hi, lA, hA);
-            lut4(sB, lut_lo, lut_hi, lB, hB);
-            const uint32_t a0 = pair02(lA, hA), a1 = pair13(lA, hA);
-            const uint32_t a2 = pair02(lB, hB), a3 = pair13(lB, hB);
-            mma16816(acc[j], a0, a1, a2, a3, bp0, bp1);
-          }
-        }
-      }
+      if (!aborted) process_tile(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qa, q2, kap, a.kc, st);
+      ++k_done;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      top_up();
     }
 
-    // ---- warp partials.  Thread (g, tq) holds coordinates 16g..16g+15: acc[j][0|1] at
-    // 16g+2j, acc[j][2|3] at 16g+2j+1.  Every consumer warp has left the ring before any
-    // of them overwrites it with the merge buffer.
-    __syncthreads();
-    // Partial row of (warp, head): coordinate c at c + c/32 (a one-word skew per 32), rows
-    // SO_STRIDE floats apart; with these the strided stores below and the merge reads are
-    // free of bank conflicts.
-    float(*so)[G][L::SO_STRIDE] = reinterpret_cast<float(*)[G][L::SO_STRIDE]>(smem);
+    // ---- merge the warps (shared memory, two rounds: warp w+4 into w, then slots 0..3),
+    // then one partial per (CTA, group)
+    float lq = st.l;
+    lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+    lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+    if ((lane & 3) == 0) {
+      sm[warp][lane >> 2] = st.m;
+      sl[warp][lane >> 2] = lq;
+    }
+    {
+      const int g = lane >> 2, t = lane & 3;
+      if (warp >= 4) {
 #pragma unroll
-    for (int hsl = 0; hsl < HS; ++hsl) {
-      float l = l_run[hsl];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
-      const int head = (G == 4) ? tq : 2 * tq + hsl;
-      if (g == 0) {
-        sm[warp][head] = m_run[hsl];
-        sl[warp][head] = l;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float o0, o1;
-        if (G == 4) {
-          o0 = acc[j][0] + acc[j][1];
-          o1 = acc[j][2] + acc[j][3];
-        } else {
-          o0 = acc[j][hsl];
-          o1 = acc[j][hsl + 2];
+        for (int j = 0; j < 8; ++j) {
+          so[warp - 4][2 * t][16 * j + g] = st.acc[j][0];
+          so[warp - 4][2 * t + 1][16 * j + g] = st.acc[j][1];
+          so[warp - 4][2 * t][16 * j + g + 8] = st.acc[j][2];
+          so[warp - 4][2 * t + 1][16 * j + g + 8] = st.acc[j][3];
         }
-        const int c0 = 16 * g + 2 * j;
-        so[warp][head][c0 + (c0 >> 5)] = o0;
-        so[warp][head][c0 + 1 + (c0 >> 5)] = o1;
+      }
+      __syncthreads();
+      if (warp < 4) {
+        float f_self[2], f_oth[2], Mh[2], Lh[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hh = 2 * t + e;
+          const float m0 = sm[warp][hh], m1 = sm[warp + 4][hh];
+          const float M = fmaxf(m0, m1);
+          f_self[e] = (m0 == -CUDART_INF_F) ? 0.f : fast_exp2(m0 - M);
+          f_oth[e] = (m1 == -CUDART_INF_F) ? 0.f : fast_exp2(m1 - M);
+          Mh[e] = M;
+          Lh[e] = sl[warp][hh] * f_self[e] + sl[warp + 4][hh] * f_oth[e];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float& o = so[warp][2 * t + (e & 1)][16 * j + g + 8 * (e >> 1)];
+            o = st.acc[j][e] * f_self[e & 1] + o * f_oth[e & 1];
+          }
+        }
+        __syncwarp();
+        if (g == 0) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            sm[warp][2 * t + e] = Mh[e];
+            sl[warp][2 * t + e] = Lh[e];
+          }
+        }
       }
     }
-  }
-  __syncthreads();
-  if (*abort_flag) return;
-
-  // ---- merge warps, write this split's partial for each of the G query heads
-  const float(*so)[G][L::SO_STRIDE] = reinterpret_cast<const float(*)[G][L::SO_STRIDE]>(smem);
-  for (int idx = threadIdx.x; idx < G * D; idx += DEC_THREADS) {
-    const int h = idx / D, coord = idx % D;
-    if (h >= g_real) continue;
-    float M = -CUDART_INF_F;
+    __syncthreads();
+    const int c_first = cta_of(seg.gstart, T, n_cta);
+    const int c_last = cta_of(seg.gstart + seg.ntiles - 1, T, n_cta);
+    const int h = warp;
+    if (h < a.g_real) {
+      float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, sm[w][h]);
-    float Lsum = 0.f, O = 0.f;
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w][h]);
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int w = 0; w < DEC_WARPS; ++w) {
-      const float mw = sm[w][h];
-      const float f = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
-      Lsum = fmaf(sl[w][h], f, Lsum);
-      O = fmaf(so[w][h][coord + (coord >> 5)], f, O);
+      for (int w = 0; w < 4; ++w) {
+        const float mw = sm[w][h];
+        const float f = (mw == -CUDART_INF_F) ? 0.f : fast_exp2(mw - M);
+        L = fmaf(sl[w][h], f, L);
+        const float4 o = *reinterpret_cast<const float4*>(&so[w][h][4 * lane]);
+        O.x = fmaf(o.x, f, O.x); O.y = fmaf(o.y, f, O.y); O.z = fmaf(o.z, f, O.z); O.w = fmaf(o.w, f, O.w);
+      }
+      const size_t slot = (size_t)cta + gid;
+      reinterpret_cast<float4*>(a.ws.part_o + (slot * HMAX + h) * D)[lane] = O;
+      if (lane == 0) a.ws.part_ml[slot * HMAX + h] = make_float2(M, L);
     }
-    const size_t row = ((size_t)b * n_q_heads + (size_t)kvh * g_real + h) * n_split + split;
-    ws.part_o[row * D + coord] = O;
-    if (coord == 0) ws.part_ml[row] = make_float2(M, Lsum);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // the barrier orders the CTA's partial stores before this thread's fence and arrival
+      __threadfence();
+      const int n_parts = c_last - c_first + 1;
+      const uint32_t old = atomicAdd(&a.ws.counters[gid], 1u);
+      if ((int)old >= n_parts && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);
+      flags[0] = ((int)old == n_parts - 1);
+      __threadfence();
+    }
+    __syncthreads();
+    if (flags[0]) {
+      // ---- this CTA completed the group: merge its partials, normalise, rotate back
+      if (h < a.g_real) {
+        // one pass over the partials, sixteen partials' loads in flight at a time
+        float M = -CUDART_INF_F, L = 0.f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = c_first; c <= c_last; c += 16) {
+          float2 mk[16];
+          float4 ok[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const size_t slot = (size_t)min(c + u, c_last) + gid;
+            mk[u] = __ldcg(a.ws.part_ml + slot * HMAX + h);
+            ok[u] = __ldcg(reinterpret_cast<const float4*>(a.ws.part_o + (slot * HMAX + h) * D) + lane);
+          }
+          float Mb = M;
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (c + u <= c_last) Mb = fmaxf(Mb, mk[u].x);
+          if (Mb == -CUDART_INF_F) continue;
+          const float fo = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - Mb);
+          L *= fo;
+          O.x *= fo; O.y *= fo; O.z *= fo; O.w *= fo;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float f = (c + u > c_last || mk[u].x == -CUDART_INF_F) ? 0.f : fast_exp2(mk[u].x - Mb);
+            L = fmaf(mk[u].y, f, L);
+            O.x = fmaf(ok[u].x, f, O.x); O.y = fmaf(ok[u].y, f, O.y); O.z = fmaf(ok[u].z, f, O.z); O.w = fmaf(ok[u].w, f, O.w);
+          }
+          M = Mb;
+        }
+        float r[4] = {0.f, 0.f, 0.f, 0.f};
+        if (L > 0.f) {
+          const float sc = 0.08838834764831845f / (a.kc.alpha8 * L);  // O holds alpha8 sum P' c
+          r[0] = O.x * sc; r[1] = O.y * sc; r[2] = O.z * sc; r[3] = O.w * sc;
+          float Mp[4][4];
+          fused_block_matrix(a.params_layer + ((size_t)seg.kvh * NBLK + lane) * 8, Mp);
+          warp_rotate_inverse(r, Mp);
+        }
+        float4* dst =
+            reinterpret_cast<float4*>(a.out + ((size_t)seg.b * a.n_q_heads + (size_t)seg.kvh * a.g_real + h) * D) + lane;
+        *dst = make_float4(r[0], r[1], r[2], r[3]);
+      }
+      if (threadIdx.x == 0) a.ws.counters[gid] = 0;  // every arrival for this group is in
+    }
+    x = seg.gstart + seg.hi;
   }
-}
 
-// One CTA (8 warps) per (sequence, query head).  Phase 1: the global max M and sum L over
-// the splits (one split per thread, block reductions).  Phase 2: warp w sums splits w, w+8, ...
-// weighted by exp2(m_s - M) with independent loads; the 8 warp sums meet in shared memory and
-// warp 0 normalises, undoes the alpha and 1/sqrt(128) centroid scales and rotates back with
-// R^T = H_hat S^T.
-constexpr int CMB_WARPS = 8;
-__global__ void __launch_bounds__(CMB_WARPS * 32)
-decode_combine_kernel(int batch, int n_q_heads, int G, const int32_t* __restrict__ ctx_len, int max_ctx,
-                      int chunk, int n_split, const float* __restrict__ params_layer, Workspace ws,
-                      float* __restrict__ out, uint32_t* status, KernelConsts kc) {
-  __shared__ float4 so[CMB_WARPS][32];
-  __shared__ float red[CMB_WARPS];
-  __shared__ float sM, sL;
-  pdl_launch_dependents();
-  pdl_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x;
-  const int b = row / n_q_heads, hq = row % n_q_heads;
-  int ctx = ctx_len[b];
-  if (ctx < 0) ctx = 0;
-  if (ctx > max_ctx) ctx = max_ctx;
-  const int ns = (ctx + chunk - 1) / chunk;
-  const size_t base = (size_t)row * n_split;
-
-  float m = -CUDART_INF_F;
-  for (int s = threadIdx.x; s < ns; s += CMB_WARPS * 32) m = fmaxf(m, ws.part_ml[base + s].x);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float M = -CUDART_INF_F;
-    for (int w = 0; w < CMB_WARPS; ++w) M = fmaxf(M, red[w]);
-    sM = M;
+  // ---- leave no bulk copy in flight (only after a timed-out wait can one be pending)
+  while (k_wait < k_fetch) {
+    const int sl_i = k_wait % NSLOT;
+    mbar_wait(&wbar[sl_i], (k_wait / NSLOT) & 1, nullptr);
+    ++k_wait;
   }
-  __syncthreads();
-  const float M = sM;
-  float l = 0.f;
-  for (int s = threadIdx.x; s < ns; s += CMB_WARPS * 32) {
-    const float2 ml = ws.part_ml[base + s];
-    if (ml.x != -CUDART_INF_F) l = fmaf(ml.y, fast_exp2(ml.x - M), l);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-  __syncthreads();
-  if (lane == 0) red[warp] = l;
-
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = warp; s < ns; s += CMB_WARPS) {
-    const float2 ml = ws.part_ml[base + s];
-    const float4 po = *(reinterpret_cast<const float4*>(ws.part_o + (base + s) * D) + lane);
-    const float f = (ml.x == -CUDART_INF_F) ? 0.f : fast_exp2(ml.x - M);
-    acc.x = fmaf(po.x, f, acc.x); acc.y = fmaf(po.y, f, acc.y); acc.z = fmaf(po.z, f, acc.z); acc.w = fmaf(po.w, f, acc.w);
-  }
-  so[warp][lane] = acc;
-  __syncthreads();
-  if (warp != 0) return;
-  float L = 0.f, r[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int w = 0; w < CMB_WARPS; ++w) {
-    L += red[w];
-    const float4 x = so[w][lane];
-    r[0] += x.x; r[1] += x.y; r[2] += x.z; r[3] += x.w;
-  }
-  float4* dst = reinterpret_cast<float4*>(out + (size_t)row * D) + lane;
-  if (!(L > 0.f)) {  // empty context, or every tile on an invalid page
-    *dst = make_float4(0.f, 0.f, 0.f, 0.f);
-    return;
-  }
-  const float scale = kc.inv_alpha * 0.08838834764831845f / L;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) r[i] *= scale;
-  float Mp[4][4];
-  fused_block_matrix(params_layer + ((size_t)(hq / G) * NBLK + lane) * 8, Mp);
-  warp_rotate_inverse(r, Mp);
-  *dst = make_float4(r[0], r[1], r[2], r[3]);
 }
 
 template <bool FUSED>
@@ -560,31 +738,30 @@ static int launch_decode_impl(const LayerView& v, const void* q, int q_f32, int 
                               void* workspace, const KernelConsts& kc, void* stream, const __half* k_new,
                               const __half* v_new) {
   if (batch == 0 || n_q_heads == 0) return 0;
-  const int G = n_q_heads / v.n_kv_heads;
-  SplitPlan p = plan_splits(batch, v.n_kv_heads, max_ctx);
-  Workspace ws = carve(workspace, batch, n_q_heads, p.n_split);
-  cudaStream_t st = (cudaStream_t)stream;
+  DecArgs a;
+  a.v = v;
+  a.q = q;
+  a.q_f32 = q_f32;
+  a.n_q_heads = n_q_heads;
+  a.g_real = n_q_heads / v.n_kv_heads;
+  a.batch = batch;
+  a.max_ctx = max_ctx;
+  a.ctx_len = ctx_len;
+  a.params_layer = params_layer;
+  a.out = out;
+  a.ws = carve(workspace, batch, v.n_kv_heads);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.kc = kc;
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
-    cudaFuncSetAttribute(decode_split_kernel<4, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecSmem<4>::bytes);
-    cudaFuncSetAttribute(decode_split_kernel<8, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, DecSmem<8>::bytes);
-    cudaFuncSetAttribute(decode_split_kernel<4, FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    cudaFuncSetAttribute(decode_split_kernel<8, FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    const int maxb = (int)DecSmem::bytes(DECODE_MAX_BATCH);
+    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
-  if (max_ctx > 0) {
-    const dim3 grid(p.n_split, v.n_kv_heads, batch);
-    cudaError_t e;
-    if (G <= 4)
-      e = launch_pdl(decode_split_kernel<4, FUSED>, grid, dim3(DEC_THREADS), DecSmem<4>::bytes, st, v, q, q_f32,
-                     n_q_heads, G, ctx_len, max_ctx, p.chunk, p.n_split, params_layer, ws, kc, k_new, v_new);
-    else
-      e = launch_pdl(decode_split_kernel<8, FUSED>, grid, dim3(DEC_THREADS), DecSmem<8>::bytes, st, v, q, q_f32,
-                     n_q_heads, G, ctx_len, max_ctx, p.chunk, p.n_split, params_layer, ws, kc, k_new, v_new);
-    if (e != cudaSuccess) return (int)e;
-  }
-  const int rows = batch * n_q_heads;
-  return (int)launch_pdl(decode_combine_kernel, dim3(rows), dim3(CMB_WARPS * 32), 0, st, batch, n_q_heads, G, ctx_len,
-                         max_ctx, p.chunk, p.n_split, params_layer, ws, out, v.status, kc);
+  const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx);
+  return (int)launch_pdl(decode_kernel<FUSED>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+                         (cudaStream_t)stream, a);
 }
 
 int launch_decode(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads, const int32_t* ctx_len,

@@ -131,40 +131,27 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
-// Look up the 4 codes in the low 16 bits of `sel`: returns low and high bytes of the
-// binary16 levels in byte order of the nibbles.
-__device__ __forceinline__ void lut4(uint32_t sel, const uint32_t lo[2], const uint32_t hi[2], uint32_t& l4,
-                                     uint32_t& h4) {
-  l4 = prmt(lo[0], lo[1], sel);
-  h4 = prmt(hi[0], hi[1], sel);
-}
-// fp16x2 of (nibble0, nibble1) / (nibble2, nibble3): pairs along a K record.
-__device__ __forceinline__ uint32_t pair01(uint32_t l4, uint32_t h4) { return prmt(l4, h4, 0x5140u); }
-__device__ __forceinline__ uint32_t pair23(uint32_t l4, uint32_t h4) { return prmt(l4, h4, 0x7362u); }
-// fp16x2 of (nibble0, nibble2) / (nibble1, nibble3): pairs across the two tokens of a V record.
-__device__ __forceinline__ uint32_t pair02(uint32_t l4, uint32_t h4) { return prmt(l4, h4, 0x6240u); }
-__device__ __forceinline__ uint32_t pair13(uint32_t l4, uint32_t h4) { return prmt(l4, h4, 0x7351u); }
-
-// ------------------------------------------------------------------ tensor core (mma.sync)
-__device__ __forceinline__ void mma16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+// ------------------------------------------------------------------ tensor core (mma.sync, int8)
+// D = A B + C with A 16x32 (row), B 32x8 (col), s8 inputs, s32 accumulators.
+// Fragments (lane = 4 g + t): a0 = A[g][4t..4t+3], a1 = A[g+8][4t..], a2 = A[g][16+4t..],
+// a3 = A[g+8][16+4t..]; b0 = B[4t..4t+3][g], b1 = B[16+4t..][g]; d0,d1 = D[g][2t,2t+1],
+// d2,d3 = D[g+8][2t,2t+1] (byte i of a register = element i of its run of four).
+__device__ __forceinline__ void imma16832(int d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1, int c0, int c1, int c2, int c3) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c0), "r"(c1), "r"(c2), "r"(c3));
 }
 
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
+// Accumulators start at the bit pattern of 1.5 * 2^23: while |sum| < 2^22 the s32 result,
+// read as a float, is exactly 1.5 * 2^23 + sum, so one float subtraction converts it.
+constexpr int kMagicI = 0x4B400000;
+constexpr float kMagicF = 12582912.0f;
+__device__ __forceinline__ float magic_to_float(int x) { return __int_as_float(x) - kMagicF; }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
+// Round-to-nearest integer of |x| < 2^22 placed in the low bits of the result word
+// (two's complement): the low byte is the int8 value.
+__device__ __forceinline__ uint32_t round_low_bits(float x) { return (uint32_t)__float_as_int(x + kMagicF); }
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -282,8 +269,8 @@ __device__ __forceinline__ uint32_t quantise(float z, float t1, float t2, float 
 // One warp encodes one fp16 vector (128 values at `src`) into the K (side 0) or V (side 1)
 // record of kv head `head` at (page, slot); lane l owns coordinates 4l..4l+3 (one SO(4)
 // block).  WHT stages on coordinate bits 2..6 run as shuffles; the lane's fused block matrix
-// is passed in.  K words are assembled with two shuffles; V records are written byte by byte
-// (only this token's bytes), so the other token of the pair is never touched.
+// is passed in.  K words are assembled with two shuffles; a V block gets only this token's
+// bits (see below).
 __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __half* __restrict__ src, int head,
                                                    int side, int page, int slot, const float Mp[4][4],
                                                    const KernelConsts& kc) {
@@ -315,17 +302,35 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
       rec[3 * (lane >> 3) + w] = word;
     }
   } else {
-    // V chunk g = lanes 4g..4g+3; first-token layout: word w holds lane 4g+w's codes at
-    // nibbles 0,1,4,5 and lane 4g+3's codes as spare bits; shifted 8 bits for the second token.
-    const uint32_t u = c0 | (c1 << 4) | (c2 << 16) | (c3 << 20);
-    const uint32_t spare = __shfl_sync(0xffffffffu, u, (lane & ~3) | 3);
-    const int w = lane & 3;
-    if (w < 3) {
-      const int par = slot & 1;
-      const uint32_t word = (u | (((spare >> w) & 0x00110011u) << 3)) << (8 * par);
-      uint8_t* rec = v.v_codes + (hs * (v.page_size / 2) + (slot >> 1)) * V_REC + 12 * (lane >> 2) + 4 * w;
-      rec[par] = (uint8_t)(word >> (8 * par));
-      rec[2 + par] = (uint8_t)(word >> (16 + 8 * par));
+    // V block: this token (u = slot mod 16) owns nibbles j and j+4 of the three words of the
+    // chunks (g, tq, h) with tq = (u mod 8) / 2, j = 2 (u / 8) + (u mod 2).  Word w of chunk
+    // (g, tq, h) takes codes of coordinates 32w + g + 8h (nibble j) and 32w + 16 + g + 8h
+    // (nibble j+4), and bit w of the codes of coordinates 96 + g + 8h and 112 + g + 8h as
+    // the spare bits.  Lane l writes words k = l and l + 32 (k < 48) of the token's
+    // (g, h, w) list; the other tokens' bits are kept (atomic and/or: tokens of one block may
+    // be appended by several warps of one launch).
+    const uint32_t mine = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+    const int u = slot & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
+    uint8_t* blk = v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int k = lane + 32 * r;
+      const int kk = k < 48 ? k : 0;
+      const int gh = kk / 3, w = kk % 3;
+      const int g = gh >> 1, h = gh & 1;
+      const int x0 = 32 * w + g + 8 * h, x1 = x0 + 16, x2 = 96 + g + 8 * h, x3 = x2 + 16;
+      const uint32_t y0 = (__shfl_sync(0xffffffffu, mine, x0 >> 2) >> (8 * (x0 & 3))) & 7u;
+      const uint32_t y1 = (__shfl_sync(0xffffffffu, mine, x1 >> 2) >> (8 * (x1 & 3))) & 7u;
+      const uint32_t y2 = (__shfl_sync(0xffffffffu, mine, x2 >> 2) >> (8 * (x2 & 3))) & 7u;
+      const uint32_t y3 = (__shfl_sync(0xffffffffu, mine, x3 >> 2) >> (8 * (x3 & 3))) & 7u;
+      if (k < 48) {
+        const uint32_t n0 = y0 | (((y2 >> w) & 1u) << 3), n1 = y1 | (((y3 >> w) & 1u) << 3);
+        const uint32_t bits = (n0 << (4 * j)) | (n1 << (16 + 4 * j));
+        const uint32_t mask = (0xFu << (4 * j)) | (0xFu << (16 + 4 * j));
+        unsigned int* word = reinterpret_cast<unsigned int*>(blk + 12 * (2 * (4 * g + tq) + h) + 4 * w);
+        atomicAnd(word, ~mask);
+        atomicOr(word, bits);
+      }
     }
   }
   if (lane == 0) {

@@ -41,10 +41,10 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   __syncthreads();
 
   const int start = start_pos[b];
-  const int pos = (start & ~1) + blockIdx.x * ENC_THREADS + threadIdx.x;  // pair-aligned lanes
+  const int pos = (start & ~15) + blockIdx.x * ENC_THREADS + threadIdx.x;  // V-block-aligned lanes
   const int i_new = pos - start;
   const bool in_range = (i_new >= 0) && (i_new < n_new);
-  // All lanes of a warp take part in the V-pair exchange below, so inactive lanes run
+  // All lanes of a warp take part in the V-block exchange below, so inactive lanes run
   // the arithmetic on zeros and skip only the loads and stores.
   int page = -1;
   if (in_range) page = resolve_page(v, b, pos);
@@ -133,49 +133,55 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
       dst[2] = make_uint4(rec[8], rec[9], rec[10], rec[11]);
     }
   } else {
-    // V record (token pair): this token's bytes, laid out as the first token of the pair
-    // (chunk g, word w: coordinates 16g+4w+{0,1,2,3} at nibbles {0,1,4,5}; coordinates
-    // 16g+12..15 as spare bits of nibbles {0,1,4,5}), shifted by 8 bits for the second.
-    const int par = pos & 1;
-    uint32_t part[24];
+    // V block (16 tokens = 16 consecutive lanes): token u = lane mod 16 owns nibbles j and
+    // j+4 of the words of chunks (g, tq, h), tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2); word w
+    // takes coordinates 32w + g + 8h, 32w + 16 + g + 8h and, as spare bits (bit w), 96 + g + 8h
+    // and 112 + g + 8h.  The four tokens of a quad (lanes u, u^1, u^8, u^9) OR their words
+    // together and member j stores the chunks of g = 2j, 2j+1 (24 contiguous bytes each).
+    const unsigned lane = threadIdx.x & 31;
+    const int u = lane & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
+    uint32_t qmask = active ? ((0xFu << (4 * j)) | (0xFu << (16 + 4 * j))) : 0u;
+    qmask |= __shfl_xor_sync(0xffffffffu, qmask, 1);
+    qmask |= __shfl_xor_sync(0xffffffffu, qmask, 8);
+    // the storing member may lie outside the launch: take the block's page from an active one
+    int qpage = active ? page : -1;
+    qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 1));
+    qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 8));
+    const size_t qhs = (size_t)(qpage < 0 ? 0 : qpage) * v.n_kv_heads + head;
+    uint8_t* blk = v.v_codes + (qhs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-      const int base = 16 * g;
-      uint32_t spare = quantise(y[base + 12], t1, t2, t3) | (quantise(y[base + 13], t1, t2, t3) << 4) |
-                       (quantise(y[base + 14], t1, t2, t3) << 16) | (quantise(y[base + 15], t1, t2, t3) << 20);
+      uint32_t wd[6];
 #pragma unroll
-      for (int w = 0; w < 3; ++w) {
-        uint32_t word = quantise(y[base + 4 * w], t1, t2, t3) | (quantise(y[base + 4 * w + 1], t1, t2, t3) << 4) |
-                        (quantise(y[base + 4 * w + 2], t1, t2, t3) << 16) |
-                        (quantise(y[base + 4 * w + 3], t1, t2, t3) << 20);
-        word |= ((spare >> w) & 0x00110011u) << 3;
-        part[3 * g + w] = par ? (word << 8) : word;
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int w = 0; w < 3; ++w) {
+          const uint32_t y0 = quantise(y[32 * w + g + 8 * h], t1, t2, t3);
+          const uint32_t y1 = quantise(y[32 * w + 16 + g + 8 * h], t1, t2, t3);
+          const uint32_t y2 = quantise(y[96 + g + 8 * h], t1, t2, t3);
+          const uint32_t y3 = quantise(y[112 + g + 8 * h], t1, t2, t3);
+          const uint32_t n0 = y0 | (((y2 >> w) & 1u) << 3), n1 = y1 | (((y3 >> w) & 1u) << 3);
+          uint32_t part = active ? ((n0 << (4 * j)) | (n1 << (16 + 4 * j))) : 0u;
+          part |= __shfl_xor_sync(0xffffffffu, part, 1);
+          part |= __shfl_xor_sync(0xffffffffu, part, 8);
+          wd[3 * h + w] = part;
+        }
       }
-    }
-    // Merge with the partner lane (same pair).  The exchange runs on every lane (the whole
-    // warp is converged here); only the stores depend on which tokens this launch writes.
-    const unsigned lane = threadIdx.x & 31;
-    const bool partner_active = __shfl_xor_sync(0xffffffffu, (int)active, 1) != 0;
-    uint8_t* rec = v.v_codes + (head_slot * (v.page_size / 2) + (slot >> 1)) * V_REC;
-    uint32_t mine[12];  // even lane: chunks 0..3 of the record, odd lane: chunks 4..7
+      if (j == (g >> 1) && qmask != 0u) {
+        uint32_t* dst = reinterpret_cast<uint32_t*>(blk + 24 * (4 * g + tq));
+        if (qmask == 0xFFFFFFFFu) {
+          uint2* d2 = reinterpret_cast<uint2*>(dst);
+          d2[0] = make_uint2(wd[0], wd[1]);
+          d2[1] = make_uint2(wd[2], wd[3]);
+          d2[2] = make_uint2(wd[4], wd[5]);
+        } else {
+          // tokens of this quad outside the launch keep their bits
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
-      const uint32_t send = (lane & 1) ? part[i] : part[12 + i];
-      const uint32_t got = __shfl_xor_sync(0xffffffffu, send, 1);
-      mine[i] = ((lane & 1) ? part[12 + i] : part[i]) | got;
-    }
-    if (active && partner_active) {
-      uint4* dst = reinterpret_cast<uint4*>(rec + (lane & 1) * 48);
-      dst[0] = make_uint4(mine[0], mine[1], mine[2], mine[3]);
-      dst[1] = make_uint4(mine[4], mine[5], mine[6], mine[7]);
-      dst[2] = make_uint4(mine[8], mine[9], mine[10], mine[11]);
-    } else if (active) {
-      // Partner token not in this launch: write only this token's bytes.
-#pragma unroll
-      for (int i = 0; i < 24; ++i) {
-        const uint32_t w = part[i];
-        rec[4 * i + par] = (uint8_t)(w >> (8 * par));
-        rec[4 * i + 2 + par] = (uint8_t)(w >> (16 + 8 * par));
+          for (int i = 0; i < 6; ++i) {
+            atomicAnd(reinterpret_cast<unsigned int*>(dst + i), ~qmask);
+            atomicOr(reinterpret_cast<unsigned int*>(dst + i), wd[i]);
+          }
+        }
       }
     }
   }
@@ -222,7 +228,7 @@ int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch
     return (int)launch_pdl(append_kernel, dim3((unsigned)blocks), dim3(APP_WARPS * 32), 0, (cudaStream_t)stream, v,
                            (const __half*)k, (const __half*)vsrc, batch, n_new, start_pos, params_layer, kc);
   }
-  dim3 grid((n_new + 1 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * 2, batch);
+  dim3 grid((n_new + 15 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * 2, batch);
   return (int)launch_pdl(encode_kernel, grid, dim3(ENC_THREADS), 0, (cudaStream_t)stream, v, (const __half*)k,
                          (const __half*)vsrc, n_new, start_pos, params_layer, kc);
 }

@@ -35,17 +35,21 @@ __global__ void export_kernel(LayerView v, int kv, int seq, int t0, int n, uint8
       }
     }
   } else {
-    const uint32_t* rec = reinterpret_cast<const uint32_t*>(v.v_codes + (hs * (v.page_size / 2) + (slot >> 1)) * V_REC);
-    const int par = slot & 1;
-    for (int gch = 0; gch < 8; ++gch) {
-      const uint32_t w[3] = {rec[3 * gch], rec[3 * gch + 1], rec[3 * gch + 2]};
-      for (int s = 0; s < 32; ++s) {
-        if (((s & 3) >= 2) != (par == 1)) continue;  // slot belongs to the other token
-        uint32_t code;
-        if (s < 24) code = (w[s >> 3] >> (4 * (s & 7))) & 7u;
-        else code = ((w[0] >> (4 * (s - 24) + 3)) & 1u) | (((w[1] >> (4 * (s - 24) + 3)) & 1u) << 1) |
-                    (((w[2] >> (4 * (s - 24) + 3)) & 1u) << 2);
-        y[16 * gch + 2 * (s >> 2) + (s & 1)] = (uint8_t)code;
+    // V block: chunk (g, tq, h) at 12 (2 (4g + tq) + h); slot 8 (m/2) + 4 (m mod 2) + j holds
+    // this token (tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2)) at coordinate 16m + g + 8h.
+    const uint8_t* blk = v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
+    const int u = slot & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
+    for (int g = 0; g < 8; ++g) {
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(blk + 12 * (2 * (4 * g + tq) + h));
+        for (int m = 0; m < 8; ++m) {
+          const int s = 8 * (m >> 1) + 4 * (m & 1) + j;
+          uint32_t code;
+          if (s < 24) code = (w[s >> 3] >> (4 * (s & 7))) & 7u;
+          else code = ((w[0] >> (4 * (s - 24) + 3)) & 1u) | (((w[1] >> (4 * (s - 24) + 3)) & 1u) << 1) |
+                      (((w[2] >> (4 * (s - 24) + 3)) & 1u) << 2);
+          y[16 * m + g + 8 * h] = (uint8_t)code;
+        }
       }
     }
   }

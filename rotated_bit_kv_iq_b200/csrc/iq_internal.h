@@ -10,8 +10,8 @@ namespace iq {
 constexpr int D = 128;          // head dimension
 constexpr int NBLK = 32;        // SO(4) blocks per head
 constexpr int K_REC = 48;       // bytes of a K record (one token)
-constexpr int V_REC = 96;       // bytes of a V record (a token pair)
-constexpr int TILE = 16;        // tokens per decode tile (one mma M dimension)
+constexpr int V_BLK_TOKENS = 16;  // tokens per V block
+constexpr int V_BLK = 768;      // bytes of a V block (16 tokens x 128 codes x 3 bits)
 
 // Lloyd-Max quantiser of N(0,1): 8 ascending levels, 7 midpoint boundaries (double).
 struct Codebook {
@@ -23,12 +23,13 @@ Codebook compute_codebook();
 // Seeded rotation parameters, [L][Hkv][32][2][4] float32, written to `out` (host).
 void init_rotation_params(uint64_t seed, int n_layers, int n_kv_heads, float* out);
 
-// Constants handed to kernels by value.
+// Constants handed to kernels by value.  The eight centroids reach the tensor cores as
+// int8 pairs: alpha8 * c_k = hi_k + lo_k / 254 (hi_k, lo_k in [-127, 127]).
 struct KernelConsts {
   float bound_pos[3];    // positive N(0,1) boundaries b4, b5, b6 (b3 = 0)
-  uint32_t lut_lo[2];    // low bytes of the 8 binary16 levels alpha*c_k (k = 0..3, 4..7)
-  uint32_t lut_hi[2];    // high bytes
-  float inv_alpha;       // 1 / alpha (levels are stored scaled by alpha)
+  uint32_t lut_hi[2];    // bytes hi_k, k = 0..3 in the first word, 4..7 in the second
+  uint32_t lut_lo[2];    // bytes lo_k
+  float alpha8;          // the int8 scale
 };
 const KernelConsts& kernel_consts();
 
@@ -59,12 +60,10 @@ int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void*
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
                   uint16_t* norms, const KernelConsts& kc, void* stream);
 
-// Split-K geometry (host): number of splits and tokens per split for a decode call.
-struct SplitPlan {
-  int n_split;
-  int chunk;
-};
-SplitPlan plan_splits(int batch, int n_kv_heads, int max_ctx);
+// Decode grid (host): CTAs of one decode launch on the current device.
+int decode_ctas(int batch, int n_kv_heads, int max_ctx);
 size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx);
+size_t decode_counter_bytes(int batch, int n_kv_heads);  // leading bytes that must be zero between calls
+constexpr int DECODE_MAX_BATCH = 2048;  // sequences per decode call (per-CTA plan in shared memory)
 
 }  // namespace iq

@@ -19,8 +19,8 @@
 
 namespace {
 
-// Split-K partials of one call (maxima, sums and value sums per query head and split).
-// Nothing in it has to start at zero: every call writes what it later reads.
+// Split-K scratch of one call: per-group arrival counters (cleared by every call before its
+// kernel runs), then the partial maxima, sums and value sums.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[IQ_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -55,6 +55,10 @@ extern "C" iq_status iq_decode_attention_noalloc(const iq_cache* cache, int32_t 
   if (need > (size_t)IQ_NOALLOC_SCRATCH_BYTES) return IQ_ERR_WORKSPACE;  // problem too large for the fixed scratch
   void* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return IQ_ERR_CUDA;
+  // the arrival counters must start at zero; a call cut short by an error may leave them set
+  if (cudaMemsetAsync(scratch, 0, iq::decode_counter_bytes(batch, cache->n_kv_heads), (cudaStream_t)stream) !=
+      cudaSuccess)
+    return IQ_ERR_CUDA;
   return iq_decode_attention(cache, layer, q_dev, q_dtype, batch, n_q_heads, ctx_len_dev, max_ctx, params_dev,
                              out_dev, scratch, (size_t)IQ_NOALLOC_SCRATCH_BYTES, stream);
 }

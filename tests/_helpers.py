@@ -30,8 +30,8 @@ def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n1
         page = int(seq_pages[pi])
         lo, hi = pi * ps, min(T, (pi + 1) * ps)
         kv_k[layer, page, head, : hi - lo] = torch.from_numpy(krec[lo:hi]).to(kv_k.device)
-        plo, phi = lo // 2, (hi + 1) // 2
-        kv_v[layer, page, head, : phi - plo] = torch.from_numpy(vrec[plo:phi]).to(kv_v.device)
+        blo, bhi = lo // 16, (hi + 15) // 16  # pages hold whole 16-token V blocks
+        kv_v[layer, page, head, : bhi - blo] = torch.from_numpy(vrec[blo:bhi]).to(kv_v.device)
         kn[layer, page, head, : hi - lo] = torch.from_numpy(k_n16[lo:hi].view(np.int16)).to(kn.device)
         vn[layer, page, head, : hi - lo] = torch.from_numpy(v_n16[lo:hi].view(np.int16)).to(vn.device)
 

@@ -78,7 +78,7 @@ def test_encode_tiny_config_matches_oracle():
             got = cache.k_code_view()[0, 0, 0, :T].cpu().numpy()
             np.testing.assert_array_equal(got, packing.pack_k_fast(expect))
         else:
-            got = cache.v_code_view()[0, 0, 0, : T // 2].cpu().numpy()
+            got = cache.v_code_view()[0, 0, 0, : T // 16].cpu().numpy()
             np.testing.assert_array_equal(got, packing.pack_v_fast(expect))
     assert cache.status.item() == 0
 
@@ -112,8 +112,9 @@ def test_encode_ragged_paged_multi_sequence():
                 _check_codes(codes[h], n16[h], ref, f"b={b} h={h} kv={which}")
 
 
-def test_encode_single_token_appends_keep_partner_bytes():
-    """Decode-style appends of one token at a time: every V write is half a pair record."""
+def test_encode_single_token_appends_keep_block_neighbours():
+    """Decode-style appends of one token at a time: every V write changes only its own bits of
+    a 16-token V block (the other tokens' codes must survive)."""
     Hkv, L = 2, 1
     P = B.iq_init_rotation(5, L, Hkv)
     cache = B.PagedCache(L, Hkv, 64, 2)
@@ -190,7 +191,7 @@ def _oracle_cache(P_layer, layer, Hkv, T, seed=0, n_outliers=4):
 def _decode(cache, layer, q, ctx, max_ctx, P):
     Bn, Hq = q.shape[0], q.shape[1]
     out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
-    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx), dtype=torch.uint8, device=DEV)
     B.iq_decode_attention(cache, layer, q, torch.from_numpy(np.asarray(ctx, np.int32)).to(DEV), max_ctx,
                           _params_dev(P), out, ws)
     torch.cuda.synchronize()
@@ -374,7 +375,7 @@ def test_decode_step_matches_oracle(G):
     q, knew, vnew, refs = cases[0]
     Bn, Hq = q.shape[0], q.shape[1]
     out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
-    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 704), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 704), dtype=torch.uint8, device=DEV)
     B.iq_decode_step(cache, 0, torch.from_numpy(q).to(DEV), torch.from_numpy(knew).to(DEV), torch.from_numpy(vnew).to(DEV),
                      torch.tensor(ctx, dtype=torch.int32, device=DEV), 704, _params_dev(P), out, ws)
     torch.cuda.synchronize()
@@ -401,7 +402,7 @@ def test_decode_step_chain_in_cuda_graph():
     ks = [torch.from_numpy(c[1]).to(DEV) for c in cases]
     vs = [torch.from_numpy(c[2]).to(DEV) for c in cases]
     outs = [torch.zeros((Bn, Hq, 128), dtype=torch.float32, device=DEV) for _ in range(L)]
-    ws = torch.empty(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 576), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 576), dtype=torch.uint8, device=DEV)
     ctx_d = torch.tensor(ctx, dtype=torch.int32, device=DEV)
     Pd = _params_dev(P)
     s = torch.cuda.Stream()

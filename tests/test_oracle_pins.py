@@ -246,28 +246,59 @@ def test_chunk_golden_fixtures():
     g = _golden("packing_chunks.txt")
     ya = [s % 8 for s in range(32)]
     assert packing.pack_chunk(ya).hex() == g["chunk_mod8"][0]
-    yb = [7 if s % 4 < 2 else 0 for s in range(32)]
-    assert packing.pack_chunk(yb).hex() == g["chunk_vpair_7_0"][0]
+    yb = [7 if s % 4 == 0 else 0 for s in range(32)]
+    assert packing.pack_chunk(yb).hex() == g["chunk_slot_mod4_0_is_7"][0]
     assert packing.unpack_chunk(bytes.fromhex(g["chunk_mod8"][0])) == ya
+
+
+def test_v_block_golden_fixtures():
+    g = _golden("packing_chunks.txt")
+    c = np.zeros((16, 128), np.uint8)
+    c[0] = 7
+    rec = packing.pack_v(c)[0]
+    assert rec[:192].tobytes().hex() == g["vblock_token0_7_head"][0]
+    # chunks (g, 0, h) are the Case B chunk, every other chunk is zero
+    for q in range(64):
+        want = g["chunk_slot_mod4_0_is_7"][0] if (q // 2) % 4 == 0 else "00" * 12
+        assert rec[12 * q : 12 * q + 12].tobytes().hex() == want, q
+    m = np.tile(np.arange(128) % 8, (16, 1)).astype(np.uint8)
+    rec = packing.pack_v(m)[0]
+    for tq in range(4):
+        for h in range(2):
+            q = 2 * (4 * 5 + tq) + h
+            assert rec[12 * q : 12 * q + 12].tobytes().hex() == g["vblock_coordmod8_chunk_g5"][0]
 
 
 def test_pack_round_trip_and_ownership():
     rng = np.random.default_rng(12)
-    codes = rng.integers(0, 8, (9, 128)).astype(np.uint8)
+    codes = rng.integers(0, 8, (37, 128)).astype(np.uint8)
     np.testing.assert_array_equal(packing.unpack_k(packing.pack_k(codes)), codes)
-    np.testing.assert_array_equal(packing.unpack_v(packing.pack_v(codes), 9), codes)
-    # a V record's even bytes depend only on the first token, odd bytes only on the second
-    a = rng.integers(0, 8, (2, 128)).astype(np.uint8)
-    b = a.copy()
-    b[1] = rng.integers(0, 8, 128)
-    ra, rb = packing.pack_v(a)[0], packing.pack_v(b)[0]
-    own = packing.v_byte_owner()
-    np.testing.assert_array_equal(ra[own == 0], rb[own == 0])
+    np.testing.assert_array_equal(packing.unpack_v(packing.pack_v(codes), 37), codes)
+    np.testing.assert_array_equal(packing.pack_k_fast(codes), packing.pack_k(codes))
+    np.testing.assert_array_equal(packing.pack_v_fast(codes), packing.pack_v(codes))
+    np.testing.assert_array_equal(packing.unpack_v_fast(packing.pack_v(codes), 37), codes)
+    # the bits of a V block that change with token u are exactly the bits the owner map
+    # gives to u: nibbles j(u) and j(u)+4 of the words of chunks (g, tq(u), h)
+    own = packing.v_bit_owner()
+    assert np.all(np.bincount(own, minlength=16) == 384)
+    base = rng.integers(0, 8, (16, 128)).astype(np.uint8)
+    bits0 = np.unpackbits(packing.pack_v(base)[0], bitorder="little")
+    for u in (0, 5, 10, 15):
+        alt = base.copy()
+        alt[u] = 7 - alt[u]  # flips every code bit of token u
+        bits1 = np.unpackbits(packing.pack_v(alt)[0], bitorder="little")
+        np.testing.assert_array_equal(np.nonzero(bits0 != bits1)[0], np.nonzero(own == u)[0])
+        for t in range(16):
+            if t != u:
+                assert not np.any(bits0[own == t] != bits1[own == t])
+        j, tq = 2 * (u // 8) + (u % 2), (u % 8) // 2
+        for q in np.unique(np.nonzero(own == u)[0] // 96):
+            assert (q // 2) % 4 == tq
+        nib = (np.nonzero(own == u)[0] % 32) // 4
+        assert set(nib.tolist()) == {j, j + 4}
     # K record for codes = coordinate mod 8 is four copies of the mod-8 fixture
     k = packing.pack_k(np.array([np.arange(128) % 8], np.uint8))[0].tobytes().hex()
     assert k == _golden("packing_chunks.txt")["chunk_mod8"][0] * 4
-    v = packing.pack_v(np.array([np.full(128, 7), np.zeros(128)], np.uint8))[0].tobytes().hex()
-    assert v == "ff00" * 48
 
 
 # ------------------------------------------------------------------ attention

@@ -43,7 +43,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     cache.v_norms.copy_((torch.rand(cache.v_norms.shape, generator=g, device=DEV) * 40 + 1).half().view(torch.int16))
     need = B.iq_decode_workspace_size(Bn, Hq, Hkv, max_ctx)
     assert need <= B.IQ_NOALLOC_SCRATCH_BYTES
-    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     for call in range(2):  # the second call reuses the scratch the first one left behind
         q = torch.randn((Bn, Hq, 128), generator=g, device=DEV).half()
         ref = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
