@@ -30,14 +30,16 @@
  *   - No C++ exception crosses this interface.
  *   - head_dim is 128; every device pointer must be 16-byte aligned (workspace 256).
  *
- * Cache layout (one pool per layer stacked along the first axis):
- *   k_codes  [L][n_pages][Hkv][page_size]   x 48-byte K records
- *   v_codes  [L][n_pages][Hkv][page_size/16] x 768-byte V blocks (16 tokens each)
- *   k_norms, v_norms [L][n_pages][Hkv][page_size] binary16 norms
+ * Cache layout: one pool, [L][n_pages][Hkv][page_size/32] tile records of 3200 bytes; the
+ *   tile record of 32 consecutive slots s0..s0+31 (s0 a multiple of 32) holds
+ *       bytes [0, 1536)     the 32 K records, slot order (48 bytes each)
+ *       bytes [1536, 3072)  the two V blocks of slots s0..s0+15 and s0+16..s0+31
+ *       bytes [3072, 3136)  the 32 K norms (binary16), bytes [3136, 3200) the 32 V norms
+ *   (100 bytes per token and kv head; one tile record is one bulk copy for the decoder).
  *   Token t of sequence b lives on page
  *       block_table_dev[b * max_pages_per_seq + t / page_size]   (paged), or
  *       b                                                         (block_table_dev == NULL)
- *   at slot t % page_size.  page_size is a positive multiple of 16.
+ *   at slot t % page_size.  page_size is a positive multiple of 32.
  *
  * Record formats (this library's own; the pages fix none):
  *   code k in 0..7 = index of the ascending Lloyd-Max centroid of N(0,1):
@@ -89,14 +91,11 @@ typedef enum { IQ_F16 = 0, IQ_F32 = 1 } iq_dtype;
 #define IQ_DEVERR_WORKSPACE 16u /* decode workspace counters were not zero (outputs undefined) */
 
 typedef struct {
-  void* k_codes;                   /* device, see layout above */
-  void* v_codes;                   /* device */
-  void* k_norms;                   /* device, uint16 binary16 bits */
-  void* v_norms;                   /* device */
+  void* pool;                      /* device, tile records (see layout above), 16-byte aligned */
   int32_t n_layers;                /* L >= 1 */
   int32_t n_kv_heads;              /* Hkv >= 1 */
   int32_t head_dim;                /* must be 128 */
-  int32_t page_size;               /* tokens per page, multiple of 16 */
+  int32_t page_size;               /* tokens per page, multiple of 32 */
   int32_t n_pages;                 /* pages in the pool */
   const int32_t* block_table_dev;  /* [batch][max_pages_per_seq] or NULL */
   int32_t max_pages_per_seq;       /* ignored when block_table_dev is NULL */
@@ -109,10 +108,10 @@ const char* iq_version(void);
 /* Human-readable text of a status code (static storage; never NULL). */
 const char* iq_status_string(iq_status s);
 
-/* Bytes of one code pool (k_codes or v_codes) and of one norm pool (k_norms or v_norms)
- * for the given geometry.  Host-only; returns IQ_ERR_INVALID_ARG on bad sizes. */
+/* Bytes of the cache pool for the given geometry (100 per token slot and kv head).
+ * Host-only; returns IQ_ERR_INVALID_ARG on bad sizes (page_size not a positive multiple of 32). */
 iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
-                         size_t* code_bytes_host, size_t* norm_bytes_host);
+                         size_t* pool_bytes_host);
 
 /* Rotation parameters from a seed (host-only; writes n_layers*n_kv_heads*256 floats to
  * params_host).  Each quaternion is drawn uniformly from the unit 3-sphere by Marsaglia's

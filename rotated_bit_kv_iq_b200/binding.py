@@ -32,6 +32,8 @@ HEAD_DIM = 128
 K_RECORD_BYTES = 48
 V_BLOCK_TOKENS = 16
 V_BLOCK_BYTES = 768
+TILE_TOKENS = 32
+TILE_BYTES = 3200  # 32 K records | 2 V blocks | 32 K norms | 32 V norms
 
 
 class IqError(RuntimeError):
@@ -42,10 +44,7 @@ class IqError(RuntimeError):
 
 class iq_cache(ctypes.Structure):
     _fields_ = [
-        ("k_codes", ctypes.c_void_p),
-        ("v_codes", ctypes.c_void_p),
-        ("k_norms", ctypes.c_void_p),
-        ("v_norms", ctypes.c_void_p),
+        ("pool", ctypes.c_void_p),
         ("n_layers", ctypes.c_int32),
         ("n_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32),
@@ -74,7 +73,7 @@ def lib():
         L.iq_status_string.restype = ctypes.c_char_p
         L.iq_status_string.argtypes = [ctypes.c_int]
         L.iq_cache_bytes.restype = ctypes.c_int
-        L.iq_cache_bytes.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.iq_cache_bytes.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz)]
         L.iq_init_rotation.restype = ctypes.c_int
         L.iq_init_rotation.argtypes = [ctypes.c_uint64, i32, i32, vp]
         L.iq_encode_append.restype = ctypes.c_int
@@ -122,9 +121,9 @@ def iq_status_string(status):
 
 
 def iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages):
-    a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
-    _check("iq_cache_bytes", lib().iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, ctypes.byref(a), ctypes.byref(b)))
-    return a.value, b.value
+    a = ctypes.c_size_t(0)
+    _check("iq_cache_bytes", lib().iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, ctypes.byref(a)))
+    return a.value
 
 
 def iq_init_rotation(seed, n_layers, n_kv_heads):
@@ -191,40 +190,49 @@ def iq_export_codes(cache, layer, kv, seq, t0, n, codes, norms=None, stream=None
 
 # ----------------------------------------------------------------------- cache holder
 class PagedCache:
-    """Device pools for a packed K/V cache (torch tensors) and the iq_cache struct over them.
+    """Device pool of a packed K/V cache (one torch tensor of tile records) and the iq_cache
+    struct over it.
 
-    page_size tokens per page; with block_table None, sequence b owns page b (a contiguous
-    cache of capacity page_size tokens per sequence)."""
+    page_size tokens per page (a multiple of 32); with block_table None, sequence b owns page b
+    (a contiguous cache of capacity page_size tokens per sequence).  The k_codes, v_codes,
+    k_norms and v_norms attributes are strided views of the pool's tile records."""
 
     def __init__(self, n_layers, n_kv_heads, page_size, n_pages, block_table=None, device="cuda"):
         import torch
 
-        code_bytes, norm_bytes = iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages)
-        self.k_codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
-        self.v_codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
-        self.k_norms = torch.empty(norm_bytes // 2, dtype=torch.int16, device=device)
-        self.v_norms = torch.empty(norm_bytes // 2, dtype=torch.int16, device=device)
+        self.pool = torch.empty(iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages), dtype=torch.uint8,
+                                device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.block_table = block_table
         self.n_layers, self.n_kv_heads, self.page_size, self.n_pages = n_layers, n_kv_heads, page_size, n_pages
         self.max_pages_per_seq = int(block_table.shape[1]) if block_table is not None else 1
+        t = self.tiles()
+        self.k_codes = t[..., 0:1536]
+        self.v_codes = t[..., 1536:3072]
+        self.k_norms = t[..., 3072:3136].view(torch.int16)
+        self.v_norms = t[..., 3136:3200].view(torch.int16)
         self.c = iq_cache(
-            self.k_codes.data_ptr(), self.v_codes.data_ptr(), self.k_norms.data_ptr(), self.v_norms.data_ptr(),
-            n_layers, n_kv_heads, HEAD_DIM, page_size, n_pages,
+            self.pool.data_ptr(), n_layers, n_kv_heads, HEAD_DIM, page_size, n_pages,
             block_table.data_ptr() if block_table is not None else None,
             self.max_pages_per_seq, self.status.data_ptr(),
         )
 
-    # Views of the pools with their logical shapes (for writing oracle-made records in tests).
+    def tiles(self):
+        """[L][n_pages][Hkv][page_size/32][3200] tile records."""
+        return self.pool.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // TILE_TOKENS, TILE_BYTES)
+
+    # Views with the records' logical shapes (for writing oracle-made records in tests).
     def k_code_view(self):
-        return self.k_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size, K_RECORD_BYTES)
+        """[L][n_pages][Hkv][page_size/32][32][48]"""
+        return self.k_codes.view(*self.k_codes.shape[:-1], TILE_TOKENS, K_RECORD_BYTES)
 
     def v_code_view(self):
-        return self.v_codes.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // V_BLOCK_TOKENS,
-                                 V_BLOCK_BYTES)
+        """[L][n_pages][Hkv][page_size/32][2][768]"""
+        return self.v_codes.view(*self.v_codes.shape[:-1], 2, V_BLOCK_BYTES)
 
     def k_norm_view(self):
-        return self.k_norms.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size)
+        """[L][n_pages][Hkv][page_size/32][32] int16"""
+        return self.k_norms
 
     def v_norm_view(self):
-        return self.v_norms.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size)
+        return self.v_norms

@@ -72,24 +72,20 @@ static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 static iq_status check_cache(const iq_cache* c, int32_t layer) {
   if (!c) return IQ_ERR_INVALID_ARG;
   if (c->head_dim != D) return IQ_ERR_UNSUPPORTED;
-  if (c->n_layers < 1 || c->n_kv_heads < 1 || c->page_size < 16 || c->page_size % 16 != 0 || c->n_pages < 1)
+  if (c->n_layers < 1 || c->n_kv_heads < 1 || c->page_size < TILE_TOKENS || c->page_size % TILE_TOKENS != 0 ||
+      c->n_pages < 1)
     return IQ_ERR_INVALID_ARG;
   if (layer < 0 || layer >= c->n_layers) return IQ_ERR_INVALID_ARG;
-  if (!c->k_codes || !c->v_codes || !c->k_norms || !c->v_norms) return IQ_ERR_INVALID_ARG;
+  if (!c->pool) return IQ_ERR_INVALID_ARG;
   if (c->block_table_dev && c->max_pages_per_seq < 1) return IQ_ERR_INVALID_ARG;
-  if (!aligned(c->k_codes, 16) || !aligned(c->v_codes, 16) || !aligned(c->k_norms, 16) ||
-      !aligned(c->v_norms, 16))
-    return IQ_ERR_ALIGNMENT;
+  if (!aligned(c->pool, 16)) return IQ_ERR_ALIGNMENT;
   return IQ_OK;
 }
 
 static LayerView view(const iq_cache* c, int32_t layer) {
   LayerView v;
-  const size_t per_layer_tokens = (size_t)c->n_pages * c->n_kv_heads * c->page_size;
-  v.k_codes = (uint8_t*)c->k_codes + per_layer_tokens * K_REC * layer;
-  v.v_codes = (uint8_t*)c->v_codes + per_layer_tokens * K_REC * layer;  // 768 B per 16 tokens = 48 B per token
-  v.k_norms = (uint16_t*)c->k_norms + per_layer_tokens * layer;
-  v.v_norms = (uint16_t*)c->v_norms + per_layer_tokens * layer;
+  const size_t per_layer_tiles = (size_t)c->n_pages * c->n_kv_heads * (c->page_size / TILE_TOKENS);
+  v.pool = (uint8_t*)c->pool + per_layer_tiles * TILE_BYTES * layer;
   v.block_table = c->block_table_dev;
   v.max_pages = c->block_table_dev ? c->max_pages_per_seq : 1;
   v.page_size = c->page_size;
@@ -125,12 +121,11 @@ const char* iq_status_string(iq_status s) {
 }
 
 iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
-                         size_t* code_bytes_host, size_t* norm_bytes_host) {
-  if (n_layers < 1 || n_kv_heads < 1 || page_size < 16 || page_size % 16 != 0 || n_pages < 1)
+                         size_t* pool_bytes_host) {
+  if (n_layers < 1 || n_kv_heads < 1 || page_size < TILE_TOKENS || page_size % TILE_TOKENS != 0 || n_pages < 1)
     return IQ_ERR_INVALID_ARG;
-  const size_t tokens = (size_t)n_layers * n_pages * n_kv_heads * page_size;
-  if (code_bytes_host) *code_bytes_host = tokens * K_REC;
-  if (norm_bytes_host) *norm_bytes_host = tokens * sizeof(uint16_t);
+  if (pool_bytes_host)
+    *pool_bytes_host = (size_t)n_layers * n_pages * n_kv_heads * (page_size / TILE_TOKENS) * TILE_BYTES;
   return IQ_OK;
 }
 

@@ -39,11 +39,13 @@ namespace iq {
 constexpr int DEC_WARPS = 8;
 constexpr int DEC_THREADS = DEC_WARPS * 32;
 constexpr int TT = 32;  // tokens per tile
-constexpr int SL_K = 0;                     // 32 K records (1536 B)
-constexpr int SL_V = SL_K + TT * K_REC;     // 2 V blocks (1536 B)
-constexpr int SL_KN = SL_V + 2 * V_BLK;     // 32 K norms (64 B)
-constexpr int SL_VN = SL_KN + TT * 2;       // 32 V norms (64 B)
-constexpr int SLOT_BYTES = SL_VN + TT * 2;  // 3200 B
+// A ring slot holds one tile record as stored (one bulk copy).
+constexpr int SL_K = TR_K;
+constexpr int SL_V = TR_V;
+constexpr int SL_KN = TR_KN;
+constexpr int SL_VN = TR_VN;
+constexpr int SLOT_BYTES = TILE_BYTES;
+static_assert(TT == TILE_TOKENS, "a tile is one tile record");
 constexpr int NSLOT = 3;                    // tiles in flight per warp
 constexpr int HMAX = 8;                     // query heads per kv head (layout width)
 constexpr int SO_STRIDE = 132;              // floats per (warp, head) row of the merge buffer
@@ -85,7 +87,7 @@ int decode_ctas(int batch, int n_kv_heads, int max_ctx) {
 }
 
 struct Workspace {
-  uint32_t* counters;  // [groups] arrivals per group; zero between calls
+  uint32_t* counters;  // [2][groups]: partials written, merges finished; zero between calls
   float2* part_ml;     // [slots][HMAX] (max in log2 units, sum of 2^(s-max))
   float* part_o;       // [slots][HMAX][128]
 };
@@ -96,17 +98,17 @@ size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_
   (void)n_q_heads;
   (void)max_ctx;
   const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
-  return align256(groups * 4) + align256(slots * HMAX * sizeof(float2)) + align256(slots * HMAX * D * sizeof(float));
+  return align256(groups * 8) + align256(slots * HMAX * sizeof(float2)) + align256(slots * HMAX * D * sizeof(float));
 }
 
-size_t decode_counter_bytes(int batch, int n_kv_heads) { return align256((size_t)batch * n_kv_heads * 4); }
+size_t decode_counter_bytes(int batch, int n_kv_heads) { return align256((size_t)batch * n_kv_heads * 8); }
 
 static Workspace carve(void* ws, int batch, int n_kv_heads) {
   const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
   Workspace w;
   char* p = (char*)ws;
   w.counters = (uint32_t*)p;
-  p += align256(groups * 4);
+  p += align256(groups * 8);
   w.part_ml = (float2*)p;
   p += align256(slots * HMAX * sizeof(float2));
   w.part_o = (float*)p;
@@ -205,7 +207,20 @@ struct Cursor {
   Seg s;
   int i;        // next local tile of segment s for this warp
   bool done;
+  int pg;       // lane 0: block-table entry of the tile (loaded ahead)
 };
+
+// Lane 0 reads the block-table entries of the cursor's tile early, so that the load is in
+// flight while the warp computes (the entries are checked when the copies are issued).
+__device__ __forceinline__ void cursor_pages(Cursor& c, const LayerView& v) {
+  if (c.done || (threadIdx.x & 31) != 0) return;
+  const int t = TT * c.i;
+  c.pg = c.s.b;
+  if (v.block_table && t < c.s.ctx) {
+    const int idx = t / v.page_size;
+    c.pg = idx < v.max_pages ? __ldg(v.block_table + (size_t)c.s.b * v.max_pages + idx) : -1;
+  }
+}
 
 __device__ __forceinline__ void cursor_normalise(Cursor& c, const DecArgs& a, const int* pre, int B, int Hkv, long long c1,
                                                  int warp) {
@@ -222,40 +237,27 @@ __device__ __forceinline__ bool is_new_token_tile(const Seg& s, int i) {
   return FUSED && i == s.ntiles - 1;
 }
 
-// Issue the bulk copies of tile i of group (b, kvh) into slot `st` (lane 0 only).
-__device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, int i, int ctx, uint8_t* st,
+// Copy tile i of group (b, kvh) -- one tile record, 3200 bytes -- into slot `st` with one bulk
+// copy (lane 0).  raw_pg is the tile's block-table entry (or b without a table), validated
+// here; the half mask marks the 16-token halves that lie before ctx.
+__device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, int i, int ctx, int raw_pg, uint8_t* st,
                                            uint8_t* valid, uint64_t* bar) {
-  int page[2], slot[2];
-  uint32_t mask = 0, bytes = 0;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int t = TT * i + 16 * hh;
-    page[hh] = -1;
-    slot[hh] = 0;
-    if (t < ctx) {
-      page[hh] = resolve_page(v, b, t);
-      slot[hh] = t % v.page_size;
-      if (page[hh] >= 0) {
-        mask |= 1u << hh;
-        bytes += 16 * K_REC + V_BLK + 64;
-      }
+  const int t = TT * i;
+  int page = -1;
+  if (t < ctx) {
+    page = raw_pg;
+    if (!v.block_table && t >= v.page_size) page = -1;
+    if (page < 0 || page >= v.n_pages) {
+      if (v.status)
+        atomicOr(v.status, page < 0 && (v.block_table ? t / v.page_size >= v.max_pages : true) ? IQ_DEVERR_POSITION
+                                                                                              : IQ_DEVERR_PAGE);
+      page = -1;
     }
   }
+  const uint32_t mask = page < 0 ? 0u : (t + 16 < ctx ? 3u : 1u);
   *valid = (uint8_t)mask;
-  mbar_arrive_expect_tx(bar, bytes);
-  const bool joined = mask == 3u && page[0] == page[1] && slot[1] == slot[0] + 16;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    if (!((mask >> hh) & 1u)) continue;
-    if (joined && hh == 1) break;
-    const int n = joined ? 2 : 1;
-    const size_t hs = (size_t)page[hh] * v.n_kv_heads + kvh;
-    bulk_g2s(st + SL_K + 16 * K_REC * hh, v.k_codes + (hs * v.page_size + slot[hh]) * K_REC, n * 16 * K_REC, bar);
-    bulk_g2s(st + SL_V + V_BLK * hh, v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + slot[hh] / V_BLK_TOKENS) * V_BLK,
-             n * V_BLK, bar);
-    bulk_g2s(st + SL_KN + 32 * hh, v.k_norms + hs * v.page_size + slot[hh], n * 32, bar);
-    bulk_g2s(st + SL_VN + 32 * hh, v.v_norms + hs * v.page_size + slot[hh], n * 32, bar);
-  }
+  mbar_arrive_expect_tx(bar, mask ? TILE_BYTES : 0);
+  if (mask) bulk_g2s(st, tile_record(v, page, kvh, t % v.page_size), TILE_BYTES, bar);
 }
 
 // The new token of sequence b (position ctx-1): encode K and V into the cache (whole warp).
@@ -452,6 +454,87 @@ __device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, i
   if (lane == 0) kappa[h] = live ? kLog2e / (128.f * gam * a.kc.alpha8) : 0.f;
 }
 
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Final merge of one group's partials for the query heads this CTA was given (h = k, k + n,
+// ... with k its index among the group's n CTAs), after every partial is in.  Heads are taken
+// two at a time, four warps each, one coordinate per lane; when only one of the two exists,
+// both warp groups work on it, each over half of the partials, and meet in shared memory.
+// O = sum_c 2^(m_c - M) O_c and L likewise, then R^T per head.
+__device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, int gid, int c_first, int n_parts, int k,
+                                            float* buf, const float* prm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = warp >> 2;
+  const int coord = 32 * (warp & 3) + lane;
+  float* sacc = buf + 2 * D;                 // [128] group 1's value sums (split case)
+  float* sml = buf + 3 * D;                  // [2] group 1's (M, L)
+  for (int h0 = k; h0 < a.g_real; h0 += 2 * n_parts) {
+    const bool split = h0 + n_parts >= a.g_real;
+    const int h = split ? h0 : h0 + grp * n_parts;
+    const int half = (n_parts + 1) >> 1;
+    const int p_lo = split ? grp * half : 0, p_hi = split ? (grp ? n_parts : half) : n_parts;
+    float acc = 0.f, M = -CUDART_INF_F, L = 0.f;
+    for (int c0 = p_lo; c0 < p_hi; c0 += 32) {
+      const int nb = min(32, p_hi - c0);
+      float ov[32];
+#pragma unroll
+      for (int u = 0; u < 32; ++u)
+        ov[u] = __ldcg(a.ws.part_o + (((size_t)(c_first + c0 + min(u, nb - 1)) + gid) * HMAX + h) * D + coord);
+      const float2 ml = lane < nb ? __ldcg(a.ws.part_ml + ((size_t)(c_first + c0 + lane) + gid) * HMAX + h)
+                                  : make_float2(-CUDART_INF_F, 0.f);
+      float Mb = ml.x;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
+      Mb = fmaxf(Mb, M);
+      if (Mb == -CUDART_INF_F) continue;
+      const float fo = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - Mb);
+      const float w = (ml.x == -CUDART_INF_F) ? 0.f : fast_exp2(ml.x - Mb);
+      float lw = ml.y * w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+      acc *= fo;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) acc = fmaf(ov[u], __shfl_sync(0xffffffffu, w, u), acc);  // w = 0 past nb
+      L = L * fo + lw;
+      M = Mb;
+    }
+    if (split) {
+      if (grp == 1) {
+        sacc[coord] = acc;
+        if (warp == 4 && lane == 0) { sml[0] = M; sml[1] = L; }
+      }
+      __syncthreads();
+      if (grp == 0) {
+        const float M1 = sml[0], L1 = sml[1];
+        const float Mn = fmaxf(M, M1);
+        const float f0 = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - Mn);
+        const float f1 = (M1 == -CUDART_INF_F) ? 0.f : fast_exp2(M1 - Mn);
+        acc = acc * f0 + sacc[coord] * f1;
+        L = L * f0 + L1 * f1;
+      }
+    }
+    // normalise, gather the head in shared memory, rotate back with one warp
+    const bool live = h < a.g_real && !(split && grp == 1);
+    const int slot = split ? 0 : grp;
+    if (live) buf[slot * D + coord] = L > 0.f ? acc * (0.08838834764831845f / (a.kc.alpha8 * L)) : 0.f;
+    __syncthreads();
+    if ((warp & 3) == 0 && live) {
+      float r[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) r[i] = buf[slot * D + 4 * lane + i];
+      float Mp[4][4];
+      fused_block_matrix(prm + lane * 8, Mp);
+      warp_rotate_inverse(r, Mp);
+      reinterpret_cast<float4*>(a.out + ((size_t)seg.b * a.n_q_heads + (size_t)seg.kvh * a.g_real + h) * D)[lane] =
+          make_float4(r[0], r[1], r[2], r[3]);
+    }
+    __syncthreads();
+  }
+}
+
 // ------------------------------------------------------------------ the kernel
 template <bool FUSED>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
@@ -463,15 +546,13 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   float(*sl)[HMAX] = reinterpret_cast<float(*)[HMAX]>(smem + DecSmem::sl);
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(smem + DecSmem::qfrag);
   float* kappa = reinterpret_cast<float*>(smem + DecSmem::kappa);
-  int* flags = reinterpret_cast<int*>(smem + DecSmem::flags);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DecSmem::bars);
   int* pre = reinterpret_cast<int*>(smem + DecSmem::plan);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.v.n_kv_heads, B = a.batch;
   uint8_t* ring = smem + DecSmem::ring + warp * NSLOT * SLOT_BYTES;
   uint8_t* valid = smem + DecSmem::valid + warp * NSLOT;
-  uint64_t* wbar = bars + warp * NSLOT;
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + DecSmem::bars) + warp * NSLOT;
   if (lane == 0) {
     for (int s = 0; s < NSLOT; ++s) mbar_init(&wbar[s], 1);
     mbar_fence_init();
@@ -486,14 +567,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 
   // ---- prefetch: the warp's first tiles (a tile holding this call's new token waits)
   bool waited = !FUSED;
-  bool aborted = false;
   Cursor fc;
   fc.done = c0 >= c1;
   if (!fc.done) {
     fc.s = segment_at(a, pre, B, Hkv, c0, c1);
     fc.i = fc.s.lo + warp;
     cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
+    cursor_pages(fc, a.v);
   }
+  bool aborted = false;
   int k_fetch = 0, k_done = 0, k_wait = 0;  // tiles issued, tiles passed, slots waited for
   auto top_up = [&]() {
     while (!fc.done && !aborted && k_fetch < k_done + NSLOT) {
@@ -506,10 +588,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       }
       const int sl_i = k_fetch % NSLOT;
       if (lane == 0)
-        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i]);
+        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, fc.pg, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i]);
       ++k_fetch;
       fc.i += DEC_WARPS;
       cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
+      cursor_pages(fc, a.v);
     }
   };
   top_up();
@@ -524,6 +607,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
           reinterpret_cast<const float4*>(a.params_layer + (size_t)sprm_kvh * NBLK * 8)[threadIdx.x];
   }
   if (FUSED) {
+    // warm L2 with the first segment's queries (a prefetch is only a hint: the rows are read
+    // after the wait, so a value written meanwhile by the preceding kernel is the one used)
+    if (c0 < c1 && threadIdx.x < a.g_real * 2) {
+      const Seg s0 = segment_at(a, pre, B, Hkv, c0, c1);
+      const size_t row = ((size_t)s0.b * a.n_q_heads + (size_t)s0.kvh * a.g_real + (threadIdx.x >> 1)) * D;
+      const char* p = a.q_f32 ? (const char*)((const float*)a.q + row) : (const char*)((const __half*)a.q + row);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * (threadIdx.x & 1) * (a.q_f32 ? 2 : 1)));
+    }
     pdl_wait();
     waited = true;
     top_up();
@@ -669,57 +760,46 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     if (threadIdx.x == 0) {
       // the barrier orders the CTA's partial stores before this thread's fence and arrival
       __threadfence();
-      const int n_parts = c_last - c_first + 1;
       const uint32_t old = atomicAdd(&a.ws.counters[gid], 1u);
-      if ((int)old >= n_parts && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);
-      flags[0] = ((int)old == n_parts - 1);
-      __threadfence();
+      if ((int)old >= c_last - c_first + 1 && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);
     }
-    __syncthreads();
-    if (flags[0]) {
-      // ---- this CTA completed the group: merge its partials, normalise, rotate back
-      if (h < a.g_real) {
-        // one pass over the partials, sixteen partials' loads in flight at a time
-        float M = -CUDART_INF_F, L = 0.f;
-        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c = c_first; c <= c_last; c += 16) {
-          float2 mk[16];
-          float4 ok[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const size_t slot = (size_t)min(c + u, c_last) + gid;
-            mk[u] = __ldcg(a.ws.part_ml + slot * HMAX + h);
-            ok[u] = __ldcg(reinterpret_cast<const float4*>(a.ws.part_o + (slot * HMAX + h) * D) + lane);
+    x = seg.gstart + seg.hi;
+  }
+
+  // ---- final merges: for every group of the run, the heads given to this CTA, once all of
+  // the group's partials are in (every CTA has written all of its partials before waiting)
+  x = c0;
+  while (x < c1) {
+    const Seg seg = segment_at(a, pre, B, Hkv, x, c1);
+    const int gid = seg.b * Hkv + seg.kvh;
+    const int c_first = cta_of(seg.gstart, T, n_cta);
+    const int n_parts = cta_of(seg.gstart + seg.ntiles - 1, T, n_cta) - c_first + 1;
+    const int k = cta - c_first;
+    uint32_t* done = a.ws.counters + n_groups;
+    if (k < a.g_real) {
+      __syncthreads();
+      // this kv head's rotation parameters, loaded while the partials come in
+      if (threadIdx.x < NBLK * 2)
+        reinterpret_cast<float4*>(sprm)[threadIdx.x] =
+            reinterpret_cast<const float4*>(a.params_layer + (size_t)seg.kvh * NBLK * 8)[threadIdx.x];
+      if (threadIdx.x == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while ((int)ld_acquire(&a.ws.counters[gid]) < n_parts) {
+          if (global_timer_ns() - t0 > 1000000000ull) {
+            if (a.v.status) atomicOr(a.v.status, IQ_DEVERR_TIMEOUT);
+            break;
           }
-          float Mb = M;
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            if (c + u <= c_last) Mb = fmaxf(Mb, mk[u].x);
-          if (Mb == -CUDART_INF_F) continue;
-          const float fo = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - Mb);
-          L *= fo;
-          O.x *= fo; O.y *= fo; O.z *= fo; O.w *= fo;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float f = (c + u > c_last || mk[u].x == -CUDART_INF_F) ? 0.f : fast_exp2(mk[u].x - Mb);
-            L = fmaf(mk[u].y, f, L);
-            O.x = fmaf(ok[u].x, f, O.x); O.y = fmaf(ok[u].y, f, O.y); O.z = fmaf(ok[u].z, f, O.z); O.w = fmaf(ok[u].w, f, O.w);
-          }
-          M = Mb;
         }
-        float r[4] = {0.f, 0.f, 0.f, 0.f};
-        if (L > 0.f) {
-          const float sc = 0.08838834764831845f / (a.kc.alpha8 * L);  // O holds alpha8 sum P' c
-          r[0] = O.x * sc; r[1] = O.y * sc; r[2] = O.z * sc; r[3] = O.w * sc;
-          float Mp[4][4];
-          fused_block_matrix(a.params_layer + ((size_t)seg.kvh * NBLK + lane) * 8, Mp);
-          warp_rotate_inverse(r, Mp);
-        }
-        float4* dst =
-            reinterpret_cast<float4*>(a.out + ((size_t)seg.b * a.n_q_heads + (size_t)seg.kvh * a.g_real + h) * D) + lane;
-        *dst = make_float4(r[0], r[1], r[2], r[3]);
       }
-      if (threadIdx.x == 0) a.ws.counters[gid] = 0;  // every arrival for this group is in
+      __syncthreads();
+      merge_group(a, seg, gid, c_first, n_parts, k, reinterpret_cast<float*>(smem + DecSmem::so), sprm);
+    }
+    if (threadIdx.x == 0) {
+      // the last CTA of the group to finish clears both counters for the next call
+      if ((int)atomicAdd(&done[gid], 1u) == n_parts - 1) {
+        a.ws.counters[gid] = 0;
+        done[gid] = 0;
+      }
     }
     x = seg.gstart + seg.hi;
   }

@@ -161,6 +161,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
+// Tile record holding `slot` of (page, kv head), and the pieces of one slot inside it.
+__device__ __forceinline__ uint8_t* tile_record(const LayerView& v, int page, int head, int slot) {
+  return v.pool + (((size_t)page * v.n_kv_heads + head) * (v.page_size / TILE_TOKENS) + slot / TILE_TOKENS) * TILE_BYTES;
+}
+__device__ __forceinline__ uint8_t* k_record(const LayerView& v, int page, int head, int slot) {
+  return tile_record(v, page, head, slot) + TR_K + (slot % TILE_TOKENS) * K_REC;
+}
+__device__ __forceinline__ uint8_t* v_block(const LayerView& v, int page, int head, int slot) {
+  return tile_record(v, page, head, slot) + TR_V + ((slot % TILE_TOKENS) / V_BLK_TOKENS) * V_BLK;
+}
+__device__ __forceinline__ uint16_t* norm_slot(const LayerView& v, int page, int head, int slot, int side) {
+  return reinterpret_cast<uint16_t*>(tile_record(v, page, head, slot) + (side ? TR_VN : TR_KN)) + slot % TILE_TOKENS;
+}
+
 // Resolve the page of token `pos` of sequence `b`; returns -1 (and flags) when invalid.
 __device__ __forceinline__ int resolve_page(const LayerView& v, int b, int pos) {
   int page;
@@ -275,7 +289,6 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
                                                    int side, int page, int slot, const float Mp[4][4],
                                                    const KernelConsts& kc) {
   const int lane = threadIdx.x & 31;
-  const size_t hs = (size_t)page * v.n_kv_heads + head;
   const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
   const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
   const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
@@ -298,7 +311,7 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
     const int w = (lane & 7) >> 1;
     if ((lane & 1) == 0 && w < 3) {
       const uint32_t word = pair | (((spare >> w) & 0x11111111u) << 3);
-      uint32_t* rec = reinterpret_cast<uint32_t*>(v.k_codes + (hs * v.page_size + slot) * K_REC);
+      uint32_t* rec = reinterpret_cast<uint32_t*>(k_record(v, page, head, slot));
       rec[3 * (lane >> 3) + w] = word;
     }
   } else {
@@ -311,7 +324,7 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
     // be appended by several warps of one launch).
     const uint32_t mine = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
     const int u = slot & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
-    uint8_t* blk = v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
+    uint8_t* blk = v_block(v, page, head, slot);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       const int k = lane + 32 * r;
@@ -333,10 +346,7 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
       }
     }
   }
-  if (lane == 0) {
-    uint16_t* nrm = side ? v.v_norms : v.k_norms;
-    nrm[hs * v.page_size + slot] = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
-  }
+  if (lane == 0) *norm_slot(v, page, head, slot, side) = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
 }
 
 }  // namespace iq

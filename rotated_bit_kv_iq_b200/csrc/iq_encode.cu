@@ -106,7 +106,6 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   const float sc = n * 0.08838834764831845f;  // n / sqrt(128)
   const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
 
-  const size_t head_slot = (size_t)(page < 0 ? 0 : page) * v.n_kv_heads + head;
   const int slot = pos % v.page_size;
 
   if (side == 0) {
@@ -127,7 +126,7 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
       }
     }
     if (active) {
-      uint4* dst = reinterpret_cast<uint4*>(v.k_codes + (head_slot * v.page_size + slot) * K_REC);
+      uint4* dst = reinterpret_cast<uint4*>(k_record(v, page, head, slot));
       dst[0] = make_uint4(rec[0], rec[1], rec[2], rec[3]);
       dst[1] = make_uint4(rec[4], rec[5], rec[6], rec[7]);
       dst[2] = make_uint4(rec[8], rec[9], rec[10], rec[11]);
@@ -147,8 +146,7 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     int qpage = active ? page : -1;
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 1));
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 8));
-    const size_t qhs = (size_t)(qpage < 0 ? 0 : qpage) * v.n_kv_heads + head;
-    uint8_t* blk = v.v_codes + (qhs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
+    uint8_t* blk = v_block(v, qpage < 0 ? 0 : qpage, head, slot);
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       uint32_t wd[6];
@@ -186,10 +184,7 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     }
   }
 
-  if (active) {
-    uint16_t* nrm = side ? v.v_norms : v.k_norms;
-    nrm[head_slot * v.page_size + slot] = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
-  }
+  if (active) *norm_slot(v, page, head, slot, side) = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
 }
 
 // Small appends (decode steps): one warp per vector (see warp_encode_vector).

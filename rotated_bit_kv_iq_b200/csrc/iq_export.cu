@@ -20,10 +20,9 @@ __global__ void export_kernel(LayerView v, int kv, int seq, int t0, int n, uint8
     return;
   }
   const int slot = pos % v.page_size;
-  const size_t hs = (size_t)page * v.n_kv_heads + head;
   uint8_t y[D];
   if (kv == 0) {
-    const uint32_t* rec = reinterpret_cast<const uint32_t*>(v.k_codes + (hs * v.page_size + slot) * K_REC);
+    const uint32_t* rec = reinterpret_cast<const uint32_t*>(k_record(v, page, head, slot));
     for (int c = 0; c < 4; ++c) {
       const uint32_t w[3] = {rec[3 * c], rec[3 * c + 1], rec[3 * c + 2]};
       for (int s = 0; s < 32; ++s) {
@@ -37,7 +36,7 @@ __global__ void export_kernel(LayerView v, int kv, int seq, int t0, int n, uint8
   } else {
     // V block: chunk (g, tq, h) at 12 (2 (4g + tq) + h); slot 8 (m/2) + 4 (m mod 2) + j holds
     // this token (tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2)) at coordinate 16m + g + 8h.
-    const uint8_t* blk = v.v_codes + (hs * (v.page_size / V_BLK_TOKENS) + (slot >> 4)) * V_BLK;
+    const uint8_t* blk = v_block(v, page, head, slot);
     const int u = slot & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
     for (int g = 0; g < 8; ++g) {
       for (int h = 0; h < 2; ++h) {
@@ -54,10 +53,7 @@ __global__ void export_kernel(LayerView v, int kv, int seq, int t0, int n, uint8
     }
   }
   for (int c = 0; c < D; ++c) out[c] = y[c];
-  if (norms) {
-    const uint16_t* src = (kv == 0 ? v.k_norms : v.v_norms) + hs * v.page_size + slot;
-    norms[(size_t)head * n + i] = *src;
-  }
+  if (norms) norms[(size_t)head * n + i] = *norm_slot(v, page, head, slot, kv);
 }
 
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes, uint16_t* norms,

@@ -12,6 +12,15 @@ constexpr int NBLK = 32;        // SO(4) blocks per head
 constexpr int K_REC = 48;       // bytes of a K record (one token)
 constexpr int V_BLK_TOKENS = 16;  // tokens per V block
 constexpr int V_BLK = 768;      // bytes of a V block (16 tokens x 128 codes x 3 bits)
+// Tile record: 32 consecutive slots of one (page, kv head), 3200 bytes:
+//   [0, 1536) 32 K records | [1536, 3072) 2 V blocks | [3072, 3136) 32 K norms | [3136, 3200) 32 V norms
+constexpr int TILE_TOKENS = 32;
+constexpr int TR_K = 0;
+constexpr int TR_V = TR_K + TILE_TOKENS * K_REC;
+constexpr int TR_KN = TR_V + 2 * V_BLK;
+constexpr int TR_VN = TR_KN + TILE_TOKENS * 2;
+constexpr int TILE_BYTES = TR_VN + TILE_TOKENS * 2;
+static_assert(TILE_BYTES == 3200, "tile record size");
 
 // Lloyd-Max quantiser of N(0,1): 8 ascending levels, 7 midpoint boundaries (double).
 struct Codebook {
@@ -35,10 +44,7 @@ const KernelConsts& kernel_consts();
 
 // Device geometry of one layer's pools, resolved on the host.
 struct LayerView {
-  uint8_t* k_codes;      // layer base of the K code pool
-  uint8_t* v_codes;
-  uint16_t* k_norms;
-  uint16_t* v_norms;
+  uint8_t* pool;         // layer base of the tile-record pool
   const int32_t* block_table;  // NULL -> sequence b uses page b
   int32_t max_pages;     // pages per sequence in the block table (1 when table is NULL)
   int32_t page_size;

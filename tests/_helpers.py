@@ -13,27 +13,27 @@ def oracle_encode_stream(params_head, layer, head, which, t0, n, n_outliers=4, h
 
 
 def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n16):
-    """Write oracle-packed records of tokens 0..T-1 of one sequence/head into the device pools.
+    """Write oracle-packed records of tokens 0..T-1 of one sequence/head into the device pool.
 
     seq_pages: physical page ids of the sequence, in order."""
     import torch
 
     ps = cache.page_size
     T = k_codes.shape[0]
-    krec = packing.pack_k_fast(k_codes)
-    vrec = packing.pack_v_fast(v_codes)
-    kv_k = cache.k_code_view()
-    kv_v = cache.v_code_view()
-    kn = cache.k_norm_view()
-    vn = cache.v_norm_view()
-    for pi in range((T + ps - 1) // ps):
-        page = int(seq_pages[pi])
-        lo, hi = pi * ps, min(T, (pi + 1) * ps)
-        kv_k[layer, page, head, : hi - lo] = torch.from_numpy(krec[lo:hi]).to(kv_k.device)
-        blo, bhi = lo // 16, (hi + 15) // 16  # pages hold whole 16-token V blocks
-        kv_v[layer, page, head, : bhi - blo] = torch.from_numpy(vrec[blo:bhi]).to(kv_v.device)
-        kn[layer, page, head, : hi - lo] = torch.from_numpy(k_n16[lo:hi].view(np.int16)).to(kn.device)
-        vn[layer, page, head, : hi - lo] = torch.from_numpy(v_n16[lo:hi].view(np.int16)).to(vn.device)
+    krec = torch.from_numpy(packing.pack_k_fast(k_codes))
+    vrec = torch.from_numpy(packing.pack_v_fast(v_codes))
+    kn = torch.from_numpy(np.asarray(k_n16).view(np.int16).copy())
+    vn = torch.from_numpy(np.asarray(v_n16).view(np.int16).copy())
+    kv_k, kv_v = cache.k_code_view(), cache.v_code_view()
+    k_nv, v_nv = cache.k_norm_view(), cache.v_norm_view()
+    for t0 in range(0, T, 32):  # one tile record (32 slots of one page) at a time
+        page, slot = int(seq_pages[t0 // ps]), t0 % ps
+        tile, m = slot // 32, min(32, T - t0)
+        kv_k[layer, page, head, tile, :m] = krec[t0:t0 + m].to(kv_k.device)
+        nb = (m + 15) // 16
+        kv_v[layer, page, head, tile, :nb] = vrec[t0 // 16:t0 // 16 + nb].to(kv_v.device)
+        k_nv[layer, page, head, tile, :m] = kn[t0:t0 + m].to(k_nv.device)
+        v_nv[layer, page, head, tile, :m] = vn[t0:t0 + m].to(v_nv.device)
 
 
 def max_rel_err(out, ref):

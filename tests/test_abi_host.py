@@ -50,10 +50,10 @@ def test_init_rotation_is_bit_identical_to_oracle(lib):
 
 
 def test_cache_bytes_and_workspace(lib):
-    cb, nb = B.iq_cache_bytes(2, 4, 64, 10)
-    assert cb == 2 * 4 * 64 * 10 * 48 and nb == 2 * 4 * 64 * 10 * 2
+    pb = B.iq_cache_bytes(2, 4, 64, 10)
+    assert pb == 2 * 4 * 64 * 10 * 100  # 48 + 48 code bytes and 2 + 2 norm bytes per slot and kv head
     with pytest.raises(B.IqError):
-        B.iq_cache_bytes(1, 1, 24, 1)  # page size not a multiple of 16
+        B.iq_cache_bytes(1, 1, 48, 1)  # page size not a multiple of 32
     w1 = B.iq_decode_workspace_size(1, 32, 4, 32768)
     w2 = B.iq_decode_workspace_size(2, 32, 4, 32768)
     assert 0 < w1 <= w2
@@ -67,7 +67,7 @@ cpu_only = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer ch
 
 
 def _fake_cache(**kw):
-    c = B.iq_cache(0x10000, 0x20000, 0x30000, 0x40000, 2, 2, 128, 64, 4, None, 1, None)
+    c = B.iq_cache(0x10000, 2, 2, 128, 64, 4, None, 1, None)
     for k, v in kw.items():
         setattr(c, k, v)
     return c
@@ -91,8 +91,8 @@ def test_encode_rejects_bad_arguments(lib):
     assert _enc(_fake_cache(page_size=24)) == B.IQ_ERR_INVALID_ARG
     assert _enc(_fake_cache(), layer=2) == B.IQ_ERR_INVALID_ARG
     assert _enc(_fake_cache(), layer=-1) == B.IQ_ERR_INVALID_ARG
-    assert _enc(_fake_cache(k_codes=None)) == B.IQ_ERR_INVALID_ARG
-    assert _enc(_fake_cache(k_codes=0x10004)) == B.IQ_ERR_ALIGNMENT
+    assert _enc(_fake_cache(pool=None)) == B.IQ_ERR_INVALID_ARG
+    assert _enc(_fake_cache(pool=0x10004)) == B.IQ_ERR_ALIGNMENT
     assert _enc(_fake_cache(), k=None, v=None) == B.IQ_ERR_INVALID_ARG
     assert _enc(_fake_cache(), start=None) == B.IQ_ERR_INVALID_ARG
     assert _enc(_fake_cache(), params=None) == B.IQ_ERR_INVALID_ARG

@@ -75,10 +75,10 @@ def test_encode_tiny_config_matches_oracle():
         # byte-level format check: oracle packer on the GPU's codes where they were excluded
         expect = np.where(refs[which]["near"], codes[0], refs[which]["codes"])
         if which == 0:
-            got = cache.k_code_view()[0, 0, 0, :T].cpu().numpy()
+            got = cache.k_code_view()[0, 0, 0].reshape(-1, 48)[:T].cpu().numpy()
             np.testing.assert_array_equal(got, packing.pack_k_fast(expect))
         else:
-            got = cache.v_code_view()[0, 0, 0, : T // 16].cpu().numpy()
+            got = cache.v_code_view()[0, 0, 0].reshape(-1, 768)[: T // 16].cpu().numpy()
             np.testing.assert_array_equal(got, packing.pack_v_fast(expect))
     assert cache.status.item() == 0
 
@@ -144,7 +144,7 @@ def test_encode_edge_values():
     x[3, 17] = -3.0
     x[4] = inputs.kv_tokens(0, 0, 0, 0, 0, 1)[0]
     x[5] = -x[4]
-    cache = B.PagedCache(1, 1, 16, 1)
+    cache = B.PagedCache(1, 1, 32, 1)
     t = torch.from_numpy(x).view(1, 6, 1, 128).to(DEV)
     B.iq_encode_append(cache, 0, t, t, torch.zeros(1, dtype=torch.int32, device=DEV), _params_dev(P))
     torch.cuda.synchronize()
@@ -328,7 +328,7 @@ def test_decode_flags_bad_context_and_pages():
     P = B.iq_init_rotation(1, 1, Hkv)
     table = torch.tensor([[0, 1], [2, 999]], dtype=torch.int32, device=DEV)
     cache = B.PagedCache(1, Hkv, 64, 3, block_table=table)
-    cache.k_codes.zero_(); cache.v_codes.zero_(); cache.k_norms.zero_(); cache.v_norms.zero_()
+    cache.pool.zero_()
     q = torch.from_numpy(inputs.queries(0, 0, 2, Hq)).to(DEV)
     out = _decode(cache, 0, q, [500, 100], 128, P)
     assert np.isfinite(out).all()

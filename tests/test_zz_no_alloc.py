@@ -63,7 +63,7 @@ def test_noalloc_rejects_problems_larger_than_its_scratch():
 
     build.build()
     assert B.iq_decode_workspace_size(256, 64, 8, 1 << 20) > B.IQ_NOALLOC_SCRATCH_BYTES
-    c = B.iq_cache(0x10000, 0x20000, 0x30000, 0x40000, 1, 8, 128, 1 << 20, 256, None, 1, None)
+    c = B.iq_cache(0x10000, 1, 8, 128, 1 << 20, 256, None, 1, None)
     st = B.lib().iq_decode_attention_noalloc(ctypes.byref(c), 0, 0x50000, 0, 256, 64, 0x70000, 1 << 20, 0x80000,
                                              0x90000, None)
     assert st == B.IQ_ERR_WORKSPACE
