@@ -20,10 +20,41 @@ namespace iq {
 
 constexpr int ENC_THREADS = 128;
 
+// Packed fp32 pairs (add/sub/mul/fma .f32x2: two IEEE fp32 operations per instruction, each
+// rounded exactly as its scalar form).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2s(uint64_t r, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r)); }
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int n_new,
               const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
-  __shared__ float4 smat[NBLK][4];  // fused block matrices M'_k, row r as a float4
+  // fused block matrices M'_k as column pairs: smat[k][c][0] = (M'[0][c], M'[1][c]),
+  // smat[k][c][1] = (M'[2][c], M'[3][c])
+  __shared__ uint64_t smat[NBLK][4][2];
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.z;
@@ -36,7 +67,10 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     float Mp[4][4];
     fused_block_matrix(params_layer + ((size_t)head * NBLK + threadIdx.x) * 8, Mp);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) smat[threadIdx.x][r] = make_float4(Mp[r][0], Mp[r][1], Mp[r][2], Mp[r][3]);
+    for (int c = 0; c < 4; ++c) {
+      smat[threadIdx.x][c][0] = f2(Mp[0][c], Mp[1][c]);
+      smat[threadIdx.x][c][1] = f2(Mp[2][c], Mp[3][c]);
+    }
   }
   __syncthreads();
 
@@ -50,7 +84,7 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   if (in_range) page = resolve_page(v, b, pos);
   const bool active = in_range && page >= 0;
 
-  float y[D];
+  uint64_t y[D / 2];  // coordinate pairs (2i, 2i+1)
   if (active) {
     const uint4* p = reinterpret_cast<const uint4*>(src + (((size_t)b * n_new + i_new) * v.n_kv_heads + head) * D);
 #pragma unroll
@@ -59,73 +93,80 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        __half2 h = *reinterpret_cast<const __half2*>(&ws[e]);
-        float2 f = __half22float2(h);
-        y[8 * q + 2 * e] = f.x;
-        y[8 * q + 2 * e + 1] = f.y;
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[e]));
+        y[4 * q + e] = f2(f.x, f.y);
       }
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < D; ++i) y[i] = 0.f;
+    for (int i = 0; i < D / 2; ++i) y[i] = 0ull;
   }
 
-  // ||x||^2 in fp32
-  float ss0 = 0.f, ss1 = 0.f;
+  // ||x||^2 in fp32 (even and odd coordinates summed separately, then added)
+  uint64_t ss = 0ull;
 #pragma unroll
-  for (int i = 0; i < D; i += 2) {
-    ss0 = fmaf(y[i], y[i], ss0);
-    ss1 = fmaf(y[i + 1], y[i + 1], ss1);
-  }
+  for (int i = 0; i < D / 2; ++i) ss = fma2(y[i], y[i], ss);
+  float ss0, ss1;
+  f2s(ss, ss0, ss1);
   const float n = sqrtf(ss0 + ss1);
 
-  // Butterfly stages on coordinate bits 2..6 (bits 0,1 are inside M').
+  // Butterfly stages on coordinate bits 2..6 (bits 0,1 are inside M'), two butterflies per
+  // packed instruction.
 #pragma unroll
   for (int bit = 2; bit < 7; ++bit) {
-    const int h = 1 << bit;
+    const int h = 1 << (bit - 1);  // in pairs
 #pragma unroll
-    for (int i = 0; i < D; ++i) {
+    for (int i = 0; i < D / 2; ++i) {
       if ((i & h) == 0) {
-        const float a = y[i], c = y[i + h];
-        y[i] = a + c;
-        y[i + h] = a - c;
+        const uint64_t a = y[i], c = y[i + h];
+        y[i] = add2(a, c);
+        y[i + h] = sub2(a, c);
       }
     }
   }
-  // Fused SO(4) blocks.
+  // Fused SO(4) blocks: rows (0,1) and (2,3) as pairs, z = M' v.
 #pragma unroll
   for (int k = 0; k < NBLK; ++k) {
-    const float v0 = y[4 * k], v1 = y[4 * k + 1], v2 = y[4 * k + 2], v3 = y[4 * k + 3];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float4 m = smat[k][r];
-      y[4 * k + r] = fmaf(m.x, v0, fmaf(m.y, v1, fmaf(m.z, v2, m.w * v3)));
-    }
+    float v0, v1, v2, v3;
+    f2s(y[2 * k], v0, v1);
+    f2s(y[2 * k + 1], v2, v3);
+    const uint64_t b0 = f2(v0, v0), b1 = f2(v1, v1), b2 = f2(v2, v2), b3 = f2(v3, v3);
+    uint64_t z01 = mul2(smat[k][3][0], b3), z23 = mul2(smat[k][3][1], b3);
+    z01 = fma2(smat[k][2][0], b2, z01);
+    z23 = fma2(smat[k][2][1], b2, z23);
+    z01 = fma2(smat[k][1][0], b1, z01);
+    z23 = fma2(smat[k][1][1], b1, z23);
+    y[2 * k] = fma2(smat[k][0][0], b0, z01);
+    y[2 * k + 1] = fma2(smat[k][0][1], b0, z23);
   }
 
   const float sc = n * 0.08838834764831845f;  // n / sqrt(128)
   const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
+  // codes once: cw[r] holds coordinates 8r..8r+7 as nibbles (bit 3 clear)
+  uint32_t cw[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float za, zb;
+      f2s(y[4 * r + e], za, zb);
+      w |= quantise(za, t1, t2, t3) << (8 * e);
+      w |= quantise(zb, t1, t2, t3) << (8 * e + 4);
+    }
+    cw[r] = w;
+  }
 
   const int slot = pos % v.page_size;
-
   if (side == 0) {
-    // K record: chunk c holds coordinates 32c..32c+31 in slot order.
-    uint32_t rec[12];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t spare = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) spare |= quantise(y[32 * c + 24 + j], t1, t2, t3) << (4 * j);
-#pragma unroll
-      for (int w = 0; w < 3; ++w) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) word |= quantise(y[32 * c + 8 * w + j], t1, t2, t3) << (4 * j);
-        word |= ((spare >> w) & 0x11111111u) << 3;
-        rec[3 * c + w] = word;
-      }
-    }
+    // K record: chunk c = cw[4c..4c+3]; word w of the chunk = slots 8w..8w+7 plus bit w of
+    // slots 24..31 as the spare bits.
     if (active) {
+      uint32_t rec[12];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int w = 0; w < 3; ++w) rec[3 * c + w] = cw[4 * c + w] | (((cw[4 * c + 3] >> w) & 0x11111111u) << 3);
       uint4* dst = reinterpret_cast<uint4*>(k_record(v, page, head, slot));
       dst[0] = make_uint4(rec[0], rec[1], rec[2], rec[3]);
       dst[1] = make_uint4(rec[4], rec[5], rec[6], rec[7]);
@@ -147,18 +188,18 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 1));
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 8));
     uint8_t* blk = v_block(v, qpage < 0 ? 0 : qpage, head, slot);
-#pragma unroll
-    for (int g = 0; g < 8; ++g) {
+#pragma unroll 1
+    for (int g = 0; g < 8; ++g) {  // rolled: keeps the kernel's code small
       uint32_t wd[6];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        // codes of coordinates 16m + g + 8h: nibble g of cw[2m + h]
+        uint32_t cm[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) cm[m] = (cw[2 * m + h] >> (4 * g)) & 7u;
 #pragma unroll
         for (int w = 0; w < 3; ++w) {
-          const uint32_t y0 = quantise(y[32 * w + g + 8 * h], t1, t2, t3);
-          const uint32_t y1 = quantise(y[32 * w + 16 + g + 8 * h], t1, t2, t3);
-          const uint32_t y2 = quantise(y[96 + g + 8 * h], t1, t2, t3);
-          const uint32_t y3 = quantise(y[112 + g + 8 * h], t1, t2, t3);
-          const uint32_t n0 = y0 | (((y2 >> w) & 1u) << 3), n1 = y1 | (((y3 >> w) & 1u) << 3);
+          const uint32_t n0 = cm[2 * w] | (((cm[6] >> w) & 1u) << 3), n1 = cm[2 * w + 1] | (((cm[7] >> w) & 1u) << 3);
           uint32_t part = active ? ((n0 << (4 * j)) | (n1 << (16 + 4 * j))) : 0u;
           part |= __shfl_xor_sync(0xffffffffu, part, 1);
           part |= __shfl_xor_sync(0xffffffffu, part, 8);
