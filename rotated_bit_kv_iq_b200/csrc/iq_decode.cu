@@ -758,10 +758,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-      // the barrier orders the CTA's partial stores before this thread's fence and arrival
-      __threadfence();
-      const uint32_t old = atomicAdd(&a.ws.counters[gid], 1u);
-      if ((int)old >= c_last - c_first + 1 && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);
+      // the barrier orders the CTA's partial stores before this release-ordered arrival,
+      // which the thread does not wait for
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.ws.counters[gid]) : "memory");
     }
     x = seg.gstart + seg.hi;
   }
@@ -784,12 +783,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
             reinterpret_cast<const float4*>(a.params_layer + (size_t)seg.kvh * NBLK * 8)[threadIdx.x];
       if (threadIdx.x == 0) {
         const uint64_t t0 = global_timer_ns();
-        while ((int)ld_acquire(&a.ws.counters[gid]) < n_parts) {
+        uint32_t seen;
+        while ((int)(seen = ld_acquire(&a.ws.counters[gid])) < n_parts) {
           if (global_timer_ns() - t0 > 1000000000ull) {
             if (a.v.status) atomicOr(a.v.status, IQ_DEVERR_TIMEOUT);
             break;
           }
         }
+        if ((int)seen > n_parts && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);  // counters not zeroed
       }
       __syncthreads();
       merge_group(a, seg, gid, c_first, n_parts, k, reinterpret_cast<float*>(smem + DecSmem::so), sprm);
