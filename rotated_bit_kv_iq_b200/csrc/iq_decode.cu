@@ -616,8 +616,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * (threadIdx.x & 1) * (a.q_f32 ? 2 : 1)));
     }
     pdl_wait();
-    waited = true;
-    top_up();
   }
 
   // ---- outputs of groups with no tiles (empty context): zeros
@@ -647,6 +645,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     }
     rotate_query(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
     __syncthreads();
+    // the new token is appended by the warp that loads its tile, from here on (after the wait
+    // and outside the CTA-wide barriers, so only that warp spends the time)
+    waited = true;
     uint32_t qa[16], q2[8];
     {
       const uint4* src = reinterpret_cast<const uint4*>(qfrag + lane * QF_WORDS);
@@ -672,6 +673,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 
     const int ctx = seg.ctx;
     for (int i = seg.lo + warp; i < seg.hi; i += DEC_WARPS) {
+      top_up();  // issues this tile if it is not in flight yet, and refills the ring
       const int sl_i = k_done % NSLOT;
       if (!aborted) {
         const bool landed = __all_sync(0xffffffffu, mbar_wait(&wbar[sl_i], (k_done / NSLOT) & 1, a.v.status));
@@ -680,7 +682,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       if (!aborted) process_tile(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qa, q2, kap, a.kc, st);
       ++k_done;
       __syncwarp();
-      top_up();
     }
 
     // ---- merge the warps (shared memory, two rounds: warp w+4 into w, then slots 0..3),
