@@ -54,8 +54,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecSmem {
   static constexpr int ring = 0;                                          // [warp][slot] tiles
-  static constexpr int so = ring + DEC_WARPS * NSLOT * SLOT_BYTES;        // float [4][head][SO_STRIDE]
-  static constexpr int sm = so + 4 * HMAX * SO_STRIDE * 4;                // float [warp][head] maxima
+  static constexpr int so = ring + DEC_WARPS * NSLOT * SLOT_BYTES;        // float [warp-4][head][SO_STRIDE]
+  static constexpr int sm = so + (DEC_WARPS - 4) * HMAX * SO_STRIDE * 4;  // float [warp][head] maxima
   static constexpr int sl = sm + DEC_WARPS * HMAX * 4;                    // float [warp][head] sums
   static constexpr int qfrag = sl + DEC_WARPS * HMAX * 4;                 // uint32 [lane][QF_WORDS] query fragments
   static constexpr int kappa = qfrag + 32 * QF_WORDS * 4;                 // float [head] score scales
@@ -75,9 +75,9 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else
-// one, which leaves the other half of every SM free for the next kernel's CTAs to start
-// their loads early (programmatic dependent launch).
+// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else one
+// CTA per SM, compiled for up to 255 registers a thread: the tile loop then runs with more
+// instruction-level parallelism, which matters more than early starts of the next kernel.
 int decode_ctas(int batch, int n_kv_heads, int max_ctx) {
   const int n_sm = sm_count();
   const long long tiles = (long long)batch * n_kv_heads * ((max_ctx + TT - 1) / TT);
@@ -467,7 +467,7 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 // O = sum_c 2^(m_c - M) O_c and L likewise, then R^T per head.
 __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, int gid, int c_first, int n_parts, int k,
                                             float* buf, const float* prm) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = warp >> 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = warp >> 2;  // groups 0, 1 work
   const int coord = 32 * (warp & 3) + lane;
   float* sacc = buf + 2 * D;                 // [128] group 1's value sums (split case)
   float* sml = buf + 3 * D;                  // [2] group 1's (M, L)
@@ -477,7 +477,7 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
     const int half = (n_parts + 1) >> 1;
     const int p_lo = split ? grp * half : 0, p_hi = split ? (grp ? n_parts : half) : n_parts;
     float acc = 0.f, M = -CUDART_INF_F, L = 0.f;
-    for (int c0 = p_lo; c0 < p_hi; c0 += 32) {
+    for (int c0 = p_lo; c0 < p_hi && grp < 2; c0 += 32) {
       const int nb = min(32, p_hi - c0);
       float ov[32];
 #pragma unroll
@@ -517,7 +517,7 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
       }
     }
     // normalise, gather the head in shared memory, rotate back with one warp
-    const bool live = h < a.g_real && !(split && grp == 1);
+    const bool live = grp < 2 && h < a.g_real && !(split && grp == 1);
     const int slot = split ? 0 : grp;
     if (live) buf[slot * D + coord] = L > 0.f ? acc * (0.08838834764831845f / (a.kc.alpha8 * L)) : 0.f;
     __syncthreads();
@@ -536,8 +536,8 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
 }
 
 // ------------------------------------------------------------------ the kernel
-template <bool FUSED>
-__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
+template <bool FUSED, int MINB>
+__global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(DecArgs a) {
   pdl_launch_dependents();
   if (!FUSED) pdl_wait();  // a plain call may read anything the previous kernel wrote
   extern __shared__ __align__(128) uint8_t smem[];
@@ -573,6 +573,13 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     fc.s = segment_at(a, pre, B, Hkv, c0, c1);
     fc.i = fc.s.lo + warp;
     cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
+    // lanes 1.. request the block-table entries of the warp's next tiles now, so that the
+    // dependent lookups of the first copies below find them in L1
+    if (!fc.done && a.v.block_table && lane > 0 && lane < NSLOT) {
+      const int t = TT * (fc.i + lane * DEC_WARPS);
+      if (fc.i + lane * DEC_WARPS < fc.s.hi && t < fc.s.ctx && t / a.v.page_size < a.v.max_pages)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(a.v.block_table + (size_t)fc.s.b * a.v.max_pages + t / a.v.page_size));
+    }
     cursor_pages(fc, a.v);
   }
   bool aborted = false;
@@ -643,7 +650,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
             reinterpret_cast<const float4*>(a.params_layer + (size_t)sprm_kvh * NBLK * 8)[threadIdx.x];
       __syncthreads();
     }
-    rotate_query(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
+    if (warp < HMAX) rotate_query(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
     __syncthreads();
     // the new token is appended by the warp that loads its tile, from here on (after the wait
     // and outside the CTA-wide barriers, so only that warp spends the time)
@@ -684,8 +691,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       __syncwarp();
     }
 
-    // ---- merge the warps (shared memory, two rounds: warp w+4 into w, then slots 0..3),
-    // then one partial per (CTA, group)
+    // ---- merge the warps (shared memory, two rounds: warps w+4, w+8, ... into w, then
+    // slots 0..3), then one partial per (CTA, group)
     float lq = st.l;
     lq += __shfl_xor_sync(0xffffffffu, lq, 1);
     lq += __shfl_xor_sync(0xffffffffu, lq, 2);
@@ -706,23 +713,35 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       }
       __syncthreads();
       if (warp < 4) {
-        float f_self[2], f_oth[2], Mh[2], Lh[2];
+        constexpr int NO = DEC_WARPS / 4 - 1;  // other warps merged into this one
+        float f_self[2], f_oth[NO][2], Mh[2], Lh[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int hh = 2 * t + e;
-          const float m0 = sm[warp][hh], m1 = sm[warp + 4][hh];
-          const float M = fmaxf(m0, m1);
+          const float m0 = sm[warp][hh];
+          float M = m0;
+#pragma unroll
+          for (int k = 0; k < NO; ++k) M = fmaxf(M, sm[warp + 4 * (k + 1)][hh]);
           f_self[e] = (m0 == -CUDART_INF_F) ? 0.f : fast_exp2(m0 - M);
-          f_oth[e] = (m1 == -CUDART_INF_F) ? 0.f : fast_exp2(m1 - M);
+          float L = sl[warp][hh] * f_self[e];
+#pragma unroll
+          for (int k = 0; k < NO; ++k) {
+            const float mk = sm[warp + 4 * (k + 1)][hh];
+            f_oth[k][e] = (mk == -CUDART_INF_F) ? 0.f : fast_exp2(mk - M);
+            L = fmaf(sl[warp + 4 * (k + 1)][hh], f_oth[k][e], L);
+          }
           Mh[e] = M;
-          Lh[e] = sl[warp][hh] * f_self[e] + sl[warp + 4][hh] * f_oth[e];
+          Lh[e] = L;
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float& o = so[warp][2 * t + (e & 1)][16 * j + g + 8 * (e >> 1)];
-            o = st.acc[j][e] * f_self[e & 1] + o * f_oth[e & 1];
+            const int hh = 2 * t + (e & 1), c = 16 * j + g + 8 * (e >> 1);
+            float o = st.acc[j][e] * f_self[e & 1];
+#pragma unroll
+            for (int k = 0; k < NO; ++k) o = fmaf(so[warp + 4 * k][hh][c], f_oth[k][e & 1], o);
+            so[warp][hh][c] = o;
           }
         }
         __syncwarp();
@@ -776,6 +795,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     const int n_parts = cta_of(seg.gstart + seg.ntiles - 1, T, n_cta) - c_first + 1;
     const int k = cta - c_first;
     uint32_t* done = a.ws.counters + n_groups;
+    const int n_mergers = min(a.g_real, n_parts);
     if (k < a.g_real) {
       __syncthreads();
       // this kv head's rotation parameters, loaded while the partials come in
@@ -793,12 +813,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
         }
         if ((int)seen > n_parts && a.v.status) atomicOr(a.v.status, IQ_DEVERR_WORKSPACE);  // counters not zeroed
       }
+      // the group's mergers count themselves once they have seen every partial; the last
+      // one clears both counters for the next call (nothing reads them again in this one).
+      // The count is taken before the merge so that its round trip overlaps the merge.
+      uint32_t seen_by = 0;
+      if (threadIdx.x == 0) seen_by = atomicAdd(&done[gid], 1u);
       __syncthreads();
       merge_group(a, seg, gid, c_first, n_parts, k, reinterpret_cast<float*>(smem + DecSmem::so), sprm);
-    }
-    if (threadIdx.x == 0) {
-      // the last CTA of the group to finish clears both counters for the next call
-      if ((int)atomicAdd(&done[gid], 1u) == n_parts - 1) {
+      if (threadIdx.x == 0 && (int)seen_by == n_mergers - 1) {
         a.ws.counters[gid] = 0;
         done[gid] = 0;
       }
@@ -838,11 +860,16 @@ static int launch_decode_impl(const LayerView& v, const void* q, int q_f32, int 
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     const int maxb = (int)DecSmem::bytes(DECODE_MAX_BATCH);
-    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(decode_kernel<FUSED, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED, 1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(decode_kernel<FUSED, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED, 2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx);
-  return (int)launch_pdl(decode_kernel<FUSED>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+  if (ctas > sm_count())
+    return (int)launch_pdl(decode_kernel<FUSED, 2>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+                           (cudaStream_t)stream, a);
+  return (int)launch_pdl(decode_kernel<FUSED, 1>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
                          (cudaStream_t)stream, a);
 }
 
