@@ -49,7 +49,7 @@ static_assert(TT == TILE_TOKENS, "a tile is one tile record");
 constexpr int NSLOT = 3;                    // tiles in flight per warp
 constexpr int HMAX = 8;                     // query heads per kv head (layout width)
 constexpr int SO_STRIDE = 132;              // floats per (warp, head) row of the merge buffer
-constexpr int QF_WORDS = 24;                // query fragment words per lane: 16 (hi, lo) + 8 (lo2)
+constexpr int QF_WORDS = 28;  // query fragment words per lane: 16 (hi, lo) + 8 (lo2) + 4 (bank skew)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecSmem {
@@ -75,9 +75,9 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else one
-// CTA per SM, compiled for up to 255 registers a thread: the tile loop then runs with more
-// instruction-level parallelism, which matters more than early starts of the next kernel.
+// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else
+// one, which leaves the other half of every SM free for the next kernel's CTAs to start their
+// loads early (programmatic dependent launch).
 int decode_ctas(int batch, int n_kv_heads, int max_ctx) {
   const int n_sm = sm_count();
   const long long tiles = (long long)batch * n_kv_heads * ((max_ctx + TT - 1) / TT);
@@ -284,7 +284,7 @@ __device__ __forceinline__ uint32_t pack4(uint32_t x0, uint32_t x1, uint32_t x2,
 }
 
 __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uint32_t vmask, int tok_end,
-                                             const uint32_t (&qa)[16], const uint32_t (&q2)[8], float kappa,
+                                             const uint32_t* __restrict__ qf, float kappa,
                                              const KernelConsts& kc, WarpState& ws) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint32_t LH0 = kc.lut_hi[0], LH1 = kc.lut_hi[1], LL0 = kc.lut_lo[0], LL1 = kc.lut_lo[1];
@@ -302,10 +302,12 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
     for (int cc = 0; cc < 4; ++cc) {
       const uint32_t s0 = sel[cc], s1 = sel[cc] >> 16;
       const uint32_t bh0 = prmt(LH0, LH1, s0), bh1 = prmt(LH0, LH1, s1);
-      imma16832(a1, qa[4 * cc], qa[4 * cc + 1], qa[4 * cc + 2], qa[4 * cc + 3], bh0, bh1, a1[0], a1[1], a1[2], a1[3]);
-      imma16832(a2, qa[4 * cc], qa[4 * cc + 1], qa[4 * cc + 2], qa[4 * cc + 3], prmt(LL0, LL1, s0), prmt(LL0, LL1, s1),
+      const uint4 qv = reinterpret_cast<const uint4*>(qf)[cc];
+      const uint2 qw = reinterpret_cast<const uint2*>(qf + 16)[cc];
+      imma16832(a1, qv.x, qv.y, qv.z, qv.w, bh0, bh1, a1[0], a1[1], a1[2], a1[3]);
+      imma16832(a2, qv.x, qv.y, qv.z, qv.w, prmt(LL0, LL1, s0), prmt(LL0, LL1, s1),
                 a2[0], a2[1], a2[2], a2[3]);
-      imma16832(a3, q2[2 * cc], 0u, q2[2 * cc + 1], 0u, bh0, bh1, a3[0], a3[1], a3[2], a3[3]);
+      imma16832(a3, qw.x, 0u, qw.y, 0u, bh0, bh1, a3[0], a3[1], a3[2], a3[3]);
     }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -536,8 +538,8 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
 }
 
 // ------------------------------------------------------------------ the kernel
-template <bool FUSED, int MINB>
-__global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(DecArgs a) {
+template <bool FUSED>
+__global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   pdl_launch_dependents();
   if (!FUSED) pdl_wait();  // a plain call may read anything the previous kernel wrote
   extern __shared__ __align__(128) uint8_t smem[];
@@ -655,20 +657,6 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(DecArgs a) {
     // the new token is appended by the warp that loads its tile, from here on (after the wait
     // and outside the CTA-wide barriers, so only that warp spends the time)
     waited = true;
-    uint32_t qa[16], q2[8];
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(qfrag + lane * QF_WORDS);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 u = src[i];
-        qa[4 * i] = u.x; qa[4 * i + 1] = u.y; qa[4 * i + 2] = u.z; qa[4 * i + 3] = u.w;
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint4 u = src[4 + i];
-        q2[4 * i] = u.x; q2[4 * i + 1] = u.y; q2[4 * i + 2] = u.z; q2[4 * i + 3] = u.w;
-      }
-    }
     const float kap = kappa[lane >> 2];
     WarpState st;
     st.m = -CUDART_INF_F;
@@ -686,7 +674,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(DecArgs a) {
         const bool landed = __all_sync(0xffffffffu, mbar_wait(&wbar[sl_i], (k_done / NSLOT) & 1, a.v.status));
         if (landed) ++k_wait; else aborted = true;
       }
-      if (!aborted) process_tile(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qa, q2, kap, a.kc, st);
+      if (!aborted) process_tile(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qfrag + lane * QF_WORDS, kap, a.kc, st);
       ++k_done;
       __syncwarp();
     }
@@ -860,16 +848,11 @@ static int launch_decode_impl(const LayerView& v, const void* q, int q_f32, int 
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     const int maxb = (int)DecSmem::bytes(DECODE_MAX_BATCH);
-    cudaFuncSetAttribute(decode_kernel<FUSED, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-    cudaFuncSetAttribute(decode_kernel<FUSED, 1>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    cudaFuncSetAttribute(decode_kernel<FUSED, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-    cudaFuncSetAttribute(decode_kernel<FUSED, 2>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx);
-  if (ctas > sm_count())
-    return (int)launch_pdl(decode_kernel<FUSED, 2>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
-                           (cudaStream_t)stream, a);
-  return (int)launch_pdl(decode_kernel<FUSED, 1>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+  return (int)launch_pdl(decode_kernel<FUSED>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
                          (cudaStream_t)stream, a);
 }
 
