@@ -175,11 +175,11 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
  *   ctx_len-1, n_new = 1) followed by iq_decode_attention, without the separate launch.
  * Ordering: the kernel may start while the kernel issued just before it on the stream is
  * still running (programmatic dependent launch).  Before waiting for that kernel it reads
- * only ctx_len_dev, the block table and the cached records of positions < ctx_len-1 (it
- * starts their bulk loads); q, k_new, v_new and params are read, and the cache, workspace
- * and out are written, only after the wait.  So the immediately preceding kernel must not
- * write ctx_len, the block table or older cache positions (host copies and earlier kernels
- * may). */
+ * only ctx_len_dev, the block table, params (the rotation of one kv head) and the cached
+ * records of positions < ctx_len-1 (it starts their bulk loads); q, k_new and v_new are
+ * read, and the cache, workspace and out are written, only after the wait.  So the
+ * immediately preceding kernel must not write ctx_len, the block table, params or older
+ * cache positions (host copies and earlier kernels may). */
 iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
                          const void* k_new_dev, const void* v_new_dev, int32_t batch, int32_t n_q_heads,
                          const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
