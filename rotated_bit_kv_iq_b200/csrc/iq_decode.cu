@@ -63,8 +63,8 @@ struct DecSmem {
   static constexpr int flags = sparams + NBLK * 8 * 4;                    // int [4]
   static constexpr int valid = flags + 16;                                // uint8 [warp][slot] half masks
   static constexpr int bars = (valid + DEC_WARPS * NSLOT + 7) / 8 * 8;    // uint64 [warp][slot]
-  static constexpr int plan = bars + DEC_WARPS * NSLOT * 8;               // int [batch+1] tile prefix
-  static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(batch + 1); }
+  static constexpr int plan = bars + DEC_WARPS * NSLOT * 8;               // int [batch+1] tile prefix, [batch] ctx
+  static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(2 * batch + 1); }
 };
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -129,7 +129,8 @@ struct DecArgs {
 };
 
 // ------------------------------------------------------------------ work plan
-// pre[b] = tiles of sequences 0..b-1 (per kv head); every CTA builds the same table.
+// pre[b] = tiles of sequences 0..b-1 (per kv head) and pre[B + 1 + b] = the clamped context
+// length of sequence b; every CTA builds the same table.
 __device__ void build_plan(const DecArgs& a, int* pre) {
   const int B = a.batch;
   const int per = (B + DEC_THREADS - 1) / DEC_THREADS;
@@ -161,15 +162,11 @@ __device__ void build_plan(const DecArgs& a, int* pre) {
     pre[b] = run;
     int c = a.ctx_len[b];
     c = c < 0 ? 0 : (c > a.max_ctx ? a.max_ctx : c);
+    pre[B + 1 + b] = c;
     run += (c + TT - 1) / TT;
   }
   if (threadIdx.x == DEC_THREADS - 1) pre[B] = run;
   __syncthreads();
-}
-
-__device__ __forceinline__ int seq_ctx(const DecArgs& a, int b) {
-  int c = a.ctx_len[b];
-  return c < 0 ? 0 : (c > a.max_ctx ? a.max_ctx : c);
 }
 
 // Group holding global tile x (x < T): sequence b, kv head, first global tile of the group.
@@ -193,7 +190,7 @@ __device__ __forceinline__ Seg segment_at(const DecArgs& a, const int* pre, int 
   s.gstart = (long long)Hkv * pre[s.b] + (long long)s.kvh * s.ntiles;
   s.lo = (int)(x - s.gstart);
   s.hi = (int)min((long long)s.ntiles, c1 - s.gstart);
-  s.ctx = seq_ctx(a, s.b);
+  s.ctx = pre[B + 1 + s.b];
   return s;
 }
 
