@@ -63,7 +63,8 @@ struct DecSmem {
   static constexpr int flags = sparams + NBLK * 8 * 4;                    // int [4]
   static constexpr int valid = flags + 16;                                // uint8 [warp][slot] half masks
   static constexpr int bars = (valid + DEC_WARPS * NSLOT + 7) / 8 * 8;    // uint64 [warp][slot]
-  static constexpr int plan = bars + DEC_WARPS * NSLOT * 8;               // int [batch+1] tile prefix, [batch] ctx
+  static constexpr int cursors = bars + DEC_WARPS * NSLOT * 8;           // Cursor [warp]
+  static constexpr int plan = cursors + DEC_WARPS * 48;                   // int [batch+1] tile prefix, [batch] ctx
   static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(2 * batch + 1); }
 };
 
@@ -199,24 +200,28 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int n) { return 
 
 // ------------------------------------------------------------------ tile loads
 // Per-warp fetch cursor over the warp's tiles (round robin inside each segment of the
-// CTA's run).  All fields are warp-uniform.
+// CTA's run).  All fields are warp-uniform.  It lives in shared memory between refills: it
+// is used once per tile, and registers held across the tile loop would be spilled to local
+// memory, whose reloads miss the small L1 left next to a full shared-memory carve-out.
 struct Cursor {
   Seg s;
-  int i;        // next local tile of segment s for this warp
-  bool done;
-  int pg;       // lane 0: block-table entry of the tile (loaded ahead)
+  int i;     // next local tile of segment s for this warp
+  int done;
 };
 
-// Lane 0 reads the block-table entries of the cursor's tile early, so that the load is in
-// flight while the warp computes (the entries are checked when the copies are issued).
-__device__ __forceinline__ void cursor_pages(Cursor& c, const LayerView& v) {
-  if (c.done || (threadIdx.x & 31) != 0) return;
+static_assert(sizeof(Cursor) <= 48, "one cursor slot per warp");
+
+// Lane 0 reads the block-table entry of the cursor's tile early, so that the load is in
+// flight while the warp computes (the entry is checked when the copy is issued).
+__device__ __forceinline__ int cursor_page(const Cursor& c, const LayerView& v) {
+  if (c.done || (threadIdx.x & 31) != 0) return -1;
   const int t = TT * c.i;
-  c.pg = c.s.b;
+  int pg = c.s.b;
   if (v.block_table && t < c.s.ctx) {
     const int idx = t / v.page_size;
-    c.pg = idx < v.max_pages ? __ldg(v.block_table + (size_t)c.s.b * v.max_pages + idx) : -1;
+    pg = idx < v.max_pages ? __ldg(v.block_table + (size_t)c.s.b * v.max_pages + idx) : -1;
   }
+  return pg;
 }
 
 __device__ __forceinline__ void cursor_normalise(Cursor& c, const DecArgs& a, const int* pre, int B, int Hkv, long long c1,
@@ -566,7 +571,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 
   // ---- prefetch: the warp's first tiles (a tile holding this call's new token waits)
   bool waited = !FUSED;
+  Cursor* curs = reinterpret_cast<Cursor*>(smem + DecSmem::cursors) + warp;
   Cursor fc;
+  int pg = -1;  // lane 0: block-table entry of the cursor's tile
   fc.done = c0 >= c1;
   if (!fc.done) {
     fc.s = segment_at(a, pre, B, Hkv, c0, c1);
@@ -579,12 +586,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       if (fc.i + lane * DEC_WARPS < fc.s.hi && t < fc.s.ctx && t / a.v.page_size < a.v.max_pages)
         asm volatile("prefetch.global.L1 [%0];" ::"l"(a.v.block_table + (size_t)fc.s.b * a.v.max_pages + t / a.v.page_size));
     }
-    cursor_pages(fc, a.v);
+    pg = cursor_page(fc, a.v);
   }
+  if (lane == 0) *curs = fc;
+  __syncwarp();
   bool aborted = false;
   int k_fetch = 0, k_done = 0, k_wait = 0;  // tiles issued, tiles passed, slots waited for
   auto top_up = [&]() {
-    while (!fc.done && !aborted && k_fetch < k_done + NSLOT) {
+    if (aborted || k_fetch >= k_done + NSLOT) return;
+    Cursor fc = *curs;
+    if (fc.done) return;
+    while (!fc.done && k_fetch < k_done + NSLOT) {
       const int ctx = fc.s.ctx;
       if (is_new_token_tile<FUSED>(fc.s, fc.i)) {
         if (!waited) break;
@@ -594,12 +606,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       }
       const int sl_i = k_fetch % NSLOT;
       if (lane == 0)
-        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, fc.pg, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i]);
+        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, pg, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i]);
       ++k_fetch;
       fc.i += DEC_WARPS;
       cursor_normalise(fc, a, pre, B, Hkv, c1, warp);
-      cursor_pages(fc, a.v);
+      pg = cursor_page(fc, a.v);
     }
+    __syncwarp();
+    if (lane == 0) *curs = fc;
+    __syncwarp();
   };
   top_up();
   // rotation parameters of the first segment's kv head into shared memory (they are not
