@@ -30,6 +30,29 @@ if ROOT not in sys.path:
 
 BYTES_PER_TOKEN_HEAD = 100  # 48 B K codes + 2 B K norm + 48 B V codes + 2 B V norm
 BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
+# DRAM bytes (read + write) of one decode_kernel launch of the headline layer, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum, one 13.1 MB layer), valid only for the
+# kernel sources it was taken on: reported as roofline.traffic while their hash matches.
+DECODE_TRAFFIC = {"sources": ["rotated_bit_kv_iq_b200/csrc/iq_decode.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
+                              "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"],
+                  "sha256": "0983cb34aaa81bbbd0a64c8cf446e82010b6c25e3943cc32c2dac88ec05c3722",
+                  "bytes": 13216512}
+
+
+def decode_traffic():
+    """Captured DRAM bytes per decode launch, or None once the kernel sources have changed."""
+    import hashlib
+    h = hashlib.sha256()
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        for f in DECODE_TRAFFIC["sources"]:
+            with open(os.path.join(here, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return DECODE_TRAFFIC["bytes"] if h.hexdigest() == DECODE_TRAFFIC["sha256"] else None
+
+
 HEADLINE = "qwen30b_32k"
 METRIC = "packed-KV decode attention GB/s & % HBM peak at 32K ctx; encode Mvec/s"
 
@@ -425,7 +448,8 @@ def main():
                    "graph": f"{stack.L}-layer step replayed as one CUDA graph", "layers": stack.L,
                    "bytes_per_step": stack.bytes_per_step},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "decode_kernel (one launch per layer: append + split attention + merge), CUDA-graph step time / layers",
+                     "traffic": decode_traffic(),
+                     "kernel": "decode_kernel (one launch per layer: append + split attention + merge), CUDA-graph step time / layers",
                      "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
         "e2e": {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
