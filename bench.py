@@ -279,7 +279,26 @@ def bench_encode(steps, warmup, device, stream):
             "bytes_per_launch": T * Hkv * 2 * BYTES_PER_VECTOR_ENCODE}
 
 
-def bench_serving(steps, warmup, device, stream, seed=0):
+def max_over_ranks(x, device=None):
+    """Max of a float over the ranks of the default process group (x itself without one).
+    Every timed quantity of a multi-rank run goes through this, so that the job's time is
+    that of its slowest rank."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_rank_step, ms):
+    """Whole-job rate: every rank moves bytes_per_rank_step per step; ms is the max over ranks."""
+    return world * bytes_per_rank_step / (ms * 1e-3) / 1e9
+
+
+def bench_serving(steps, warmup, device, stream, seed=0, world=1):
     """Batched serving workload: one decode step of a 32-layer stack for 16 sequences with
     seeded contexts uniform in [2048, 32768], 64-token pages in a shuffled pool, 32 q / 8 kv
     heads; replayed as one CUDA graph."""
@@ -296,6 +315,7 @@ def bench_serving(steps, warmup, device, stream, seed=0):
                         block_table=table, n_pages=B * maxp)
     ms, graph = time_graph(stack, steps, warmup, stream)
     del graph
+    ms = max_over_ranks(ms, device)
     peak, peak_kind = _peaks()
     layer_bytes = int(stack.ctx.sum()) * stack.Hkv * BYTES_PER_TOKEN_HEAD
     kern_ms = ms / stack.L
@@ -303,7 +323,7 @@ def bench_serving(steps, warmup, device, stream, seed=0):
     out = {
         "workload": f"serve_b16: decode step of 16 paged sequences (contexts {int(ctx.min())}..{int(ctx.max())}, "
                     f"sum {int(ctx.sum())}), 32 q / 8 kv heads, d=128, 32 layers, 64-token pages",
-        "value": stack.bytes_per_step / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+        "value": job_gbs(world, stack.bytes_per_step, ms), "unit": "GB/s", "ms_per_step": ms,
         "bytes_per_step": stack.bytes_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": None, "kernel": "decode_kernel, CUDA-graph step time / layers",
@@ -424,11 +444,8 @@ def main():
     with ClockSampler(local) as clk:
         ms, graph = time_graph(stack, args.steps, args.warmup, stream)
     barrier()
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * stack.bytes_per_step / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(ms, dev)
+    value = job_gbs(world, stack.bytes_per_step, ms)
 
     # dominant kernel: the per-layer decode step (one kernel: append, split attention, merge,
     # inverse rotation), timed inside the step graph: step time / layers
@@ -437,6 +454,7 @@ def main():
     peak, peak_kind = _peaks()
     achieved = layer_bytes / (kern_ms * 1e-3) / 1e9
     e2e_ms, h2d, d2h = time_e2e(stack, args.steps, args.warmup, stream)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     del graph
 
     result = {
@@ -451,7 +469,7 @@ def main():
                      "traffic": decode_traffic(),
                      "kernel": "decode_kernel (one launch per layer: append + split attention + merge), CUDA-graph step time / layers",
                      "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
-        "e2e": {"value": world * stack.bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": job_gbs(world, stack.bytes_per_step, e2e_ms), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": stack.L * DecodeStack.launches_per_layer * args.steps,
         "clocks": clk.summary(),
@@ -460,11 +478,13 @@ def main():
     torch.cuda.empty_cache()
 
     if not args.no_extras:
-        srv = bench_serving(args.steps, args.warmup, dev, stream, seed=rank)
+        srv = bench_serving(args.steps, args.warmup, dev, stream, seed=rank, world=world)
         result["serving"] = srv
         result["gpu_launches"] += srv["launches"]
         torch.cuda.empty_cache()
         enc = bench_encode(args.steps, args.warmup, dev, stream)
+        enc["ms_per_step"] = max_over_ranks(enc["ms_per_step"], dev)
+        enc["launch_ms"] = max_over_ranks(enc["launch_ms"], dev)
         mvec = world * enc["vectors_per_step"] / (enc["ms_per_step"] * 1e-3) / 1e6
         enc_ach = enc["bytes_per_launch"] / (enc["launch_ms"] * 1e-3) / 1e9
         result["encode"] = {
