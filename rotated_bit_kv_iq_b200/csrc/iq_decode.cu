@@ -285,6 +285,13 @@ __device__ __forceinline__ uint32_t pack4(uint32_t x0, uint32_t x1, uint32_t x2,
   return prmt(prmt(x0, x1, 0x0040u), prmt(x2, x3, 0x0040u), 0x5410u);
 }
 
+// P4 (at most four query heads per kv head): the mma rows and columns left free by the
+// small group carry the query's and the probabilities' lower terms, so the third score mma
+// and the third value mma disappear.  Score rows: g < 4 = q hi of head g with q lo2 at row
+// g + 8; g >= 4 = q lo of head g - 4 (rows 12..15 zero).  Value columns: n < 4 = P' hi of
+// head n, n >= 4 = P' lo of head n - 4; lanes t < 2 accumulate the hi columns, t >= 2 the
+// lo columns of the same heads (added together at the segment end).
+template <bool P4>
 __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uint32_t vmask, int tok_end,
                                              const uint32_t* __restrict__ qf, float kappa,
                                              const KernelConsts& kc, WarpState& ws) {
@@ -305,19 +312,33 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
       const uint32_t s0 = sel[cc], s1 = sel[cc] >> 16;
       const uint32_t bh0 = prmt(LH0, LH1, s0), bh1 = prmt(LH0, LH1, s1);
       const uint4 qv = reinterpret_cast<const uint4*>(qf)[cc];
-      const uint2 qw = reinterpret_cast<const uint2*>(qf + 16)[cc];
       imma16832(a1, qv.x, qv.y, qv.z, qv.w, bh0, bh1, a1[0], a1[1], a1[2], a1[3]);
       imma16832(a2, qv.x, qv.y, qv.z, qv.w, prmt(LL0, LL1, s0), prmt(LL0, LL1, s1),
                 a2[0], a2[1], a2[2], a2[3]);
-      imma16832(a3, qw.x, 0u, qw.y, 0u, bh0, bh1, a3[0], a3[1], a3[2], a3[3]);
+      if (!P4) {
+        const uint2 qw = reinterpret_cast<const uint2*>(qf + 16)[cc];
+        imma16832(a3, qw.x, 0u, qw.y, 0u, bh0, bh1, a3[0], a3[1], a3[2], a3[3]);
+      }
     }
+    if (P4) {
+      // rows g >= 4 hold lo.c_hi (a1) and lo.c_lo (a2) of head g - 4: scaled here and added by
+      // lane g - 4 (lane - 16); rows g + 8 of lanes g < 4 hold lo2.c_hi
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      // hh + (lo.c_hi + hi.c_lo)/254 + (lo.c_lo + lo2.c_hi)/254^2; each pair of raw
-      // accumulators sums to 2 * 1.5 * 2^23 + x, so one subtraction removes both offsets
-      const float x1 = (__int_as_float(a1[2 + e]) + __int_as_float(a2[e])) - 2.f * kMagicF;
-      const float x2 = (__int_as_float(a2[2 + e]) + __int_as_float(a3[e])) - 2.f * kMagicF;
-      s[2 * nt + e] = fmaf(fmaf(x2, 1.0f / 254.0f, x1), 1.0f / 254.0f, magic_to_float(a1[e]));
+      for (int e = 0; e < 2; ++e) {
+        const float w = fmaf(magic_to_float(a2[e]), 1.0f / (254.0f * 254.0f), magic_to_float(a1[e]) * (1.0f / 254.0f));
+        const float w_lo = __shfl_xor_sync(0xffffffffu, w, 16);
+        s[2 * nt + e] = fmaf(magic_to_float(a1[2 + e]), 1.0f / (254.0f * 254.0f),
+                             fmaf(magic_to_float(a2[e]), 1.0f / 254.0f, magic_to_float(a1[e]))) + w_lo;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        // hh + (lo.c_hi + hi.c_lo)/254 + (lo.c_lo + lo2.c_hi)/254^2; each pair of raw
+        // accumulators sums to 2 * 1.5 * 2^23 + x, so one subtraction removes both offsets
+        const float x1 = (__int_as_float(a1[2 + e]) + __int_as_float(a2[e])) - 2.f * kMagicF;
+        const float x2 = (__int_as_float(a2[2 + e]) + __int_as_float(a3[e])) - 2.f * kMagicF;
+        s[2 * nt + e] = fmaf(fmaf(x2, 1.0f / 254.0f, x1), 1.0f / 254.0f, magic_to_float(a1[e]));
+      }
     }
   }
   // ---- norms, masks, online softmax (head g)
@@ -350,7 +371,8 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
   if (__any_sync(0xffffffffu, m_new > ws.m)) {
     const float r = (m_new > ws.m) ? fast_exp2(ws.m - m_new) : 1.f;
     ws.l *= r;
-    const float r0 = __shfl_sync(0xffffffffu, r, 8 * t), r1 = __shfl_sync(0xffffffffu, r, 8 * t + 4);
+    const int hl = P4 ? 8 * (t & 1) : 8 * t;  // lane of the head of columns 2t, 2t+1
+    const float r0 = __shfl_sync(0xffffffffu, r, hl), r1 = __shfl_sync(0xffffffffu, r, hl + 4);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       ws.acc[j][0] *= r0;
@@ -373,7 +395,9 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
   pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
   const float gam = pmax > 0.f ? 127.f / pmax : 0.f;
   const float ig = pmax > 0.f ? pmax * (1.0f / 127.0f) : 0.f;
-  const float ig0 = __shfl_sync(0xffffffffu, ig, 8 * t), ig1 = __shfl_sync(0xffffffffu, ig, 8 * t + 4);
+  const int hl = P4 ? 8 * (t & 1) : 8 * t;
+  const float igs = (P4 && t >= 2) ? 1.0f / 254.0f : 1.0f;  // P4: lo columns carry P' lo
+  const float ig0 = __shfl_sync(0xffffffffu, ig, hl) * igs, ig1 = __shfl_sync(0xffffffffu, ig, hl + 4) * igs;
   uint32_t hb[8], lb[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -382,8 +406,12 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
     const float h = __int_as_float((int)hb[i]) - kMagicF;
     lb[i] = round_low_bits((x - h) * 254.f);
   }
-  const uint32_t bh0 = pack4(hb[0], hb[1], hb[2], hb[3]), bh1 = pack4(hb[4], hb[5], hb[6], hb[7]);
+  uint32_t bh0 = pack4(hb[0], hb[1], hb[2], hb[3]), bh1 = pack4(hb[4], hb[5], hb[6], hb[7]);
   const uint32_t bl0 = pack4(lb[0], lb[1], lb[2], lb[3]), bl1 = pack4(lb[4], lb[5], lb[6], lb[7]);
+  if (P4) {  // columns g >= 4: P' lo of head g - 4, from lane - 16
+    const uint32_t x0 = __shfl_xor_sync(0xffffffffu, bl0, 16), x1 = __shfl_xor_sync(0xffffffffu, bl1, 16);
+    if (g >= 4) { bh0 = x0; bh1 = x1; }
+  }
   // ---- values: lane chunk (g, t) of each V block = 24 bytes at 24 * lane
   uint32_t sv[4][4];  // [block*2 + h][word]
 #pragma unroll
@@ -400,9 +428,14 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
     const uint32_t h0 = prmt(LH0, LH1, c0), h1 = prmt(LH0, LH1, c1), h2 = prmt(LH0, LH1, c2), h3 = prmt(LH0, LH1, c3);
     int d1[4], d2[4];
     imma16832(d1, h0, h1, h2, h3, bh0, bh1, kMagicI, kMagicI, kMagicI, kMagicI);
-    imma16832(d2, h0, h1, h2, h3, bl0, bl1, kMagicI, kMagicI, kMagicI, kMagicI);
-    imma16832(d2, prmt(LL0, LL1, c0), prmt(LL0, LL1, c1), prmt(LL0, LL1, c2), prmt(LL0, LL1, c3), bh0, bh1, d2[0],
-              d2[1], d2[2], d2[3]);
+    if (P4) {
+      imma16832(d2, prmt(LL0, LL1, c0), prmt(LL0, LL1, c1), prmt(LL0, LL1, c2), prmt(LL0, LL1, c3), bh0, bh1,
+                kMagicI, kMagicI, kMagicI, kMagicI);
+    } else {
+      imma16832(d2, h0, h1, h2, h3, bl0, bl1, kMagicI, kMagicI, kMagicI, kMagicI);
+      imma16832(d2, prmt(LL0, LL1, c0), prmt(LL0, LL1, c1), prmt(LL0, LL1, c2), prmt(LL0, LL1, c3), bh0, bh1,
+                d2[0], d2[1], d2[2], d2[3]);
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float tv = fmaf(magic_to_float(d2[e]), 1.0f / 254.0f, magic_to_float(d1[e]));
@@ -415,6 +448,9 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
 // Warp h rotates query head h of group (b, kvh), quantises it to int8 hi/lo with scale
 // gamma = 127 / max|q'| and writes it in mma A-fragment order: lane l holds coordinates
 // 4l..4l+3 = k-slots of chunk cc = (l/2) mod 4, fragment row 4h + l/8.
+// P4: head h < 4 fills the fragment rows of lanes g = h (hi, with lo2 as row g + 8) and
+// g = h + 4 (lo, row g + 8 zero); see process_tile.
+template <bool P4>
 __device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, int h, const float* prm,
                                              uint32_t* qfrag, float* kappa) {
   const int lane = threadIdx.x & 31;
@@ -452,9 +488,17 @@ __device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, i
   }
   const int tq = lane >> 3, cc = (lane >> 1) & 3, e = lane & 1;
   uint32_t* row = qfrag + (4 * h + tq) * QF_WORDS;
-  row[4 * cc + 2 * e] = pack4(hi[0], hi[1], hi[2], hi[3]);
-  row[4 * cc + 2 * e + 1] = pack4(lo[0], lo[1], lo[2], lo[3]);
-  row[16 + 2 * cc + e] = pack4(lo2[0], lo2[1], lo2[2], lo2[3]);
+  if (P4) {
+    uint32_t* row_lo = qfrag + (4 * (h + 4) + tq) * QF_WORDS;
+    row[4 * cc + 2 * e] = pack4(hi[0], hi[1], hi[2], hi[3]);
+    row[4 * cc + 2 * e + 1] = pack4(lo2[0], lo2[1], lo2[2], lo2[3]);
+    row_lo[4 * cc + 2 * e] = pack4(lo[0], lo[1], lo[2], lo[3]);
+    row_lo[4 * cc + 2 * e + 1] = 0u;
+  } else {
+    row[4 * cc + 2 * e] = pack4(hi[0], hi[1], hi[2], hi[3]);
+    row[4 * cc + 2 * e + 1] = pack4(lo[0], lo[1], lo[2], lo[3]);
+    row[16 + 2 * cc + e] = pack4(lo2[0], lo2[1], lo2[2], lo2[3]);
+  }
   if (lane == 0) kappa[h] = live ? kLog2e / (128.f * gam * a.kc.alpha8) : 0.f;
 }
 
@@ -540,7 +584,7 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
 }
 
 // ------------------------------------------------------------------ the kernel
-template <bool FUSED>
+template <bool FUSED, bool P4>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   pdl_launch_dependents();
   if (!FUSED) pdl_wait();  // a plain call may read anything the previous kernel wrote
@@ -664,7 +708,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
             reinterpret_cast<const float4*>(a.params_layer + (size_t)sprm_kvh * NBLK * 8)[threadIdx.x];
       __syncthreads();
     }
-    if (warp < HMAX) rotate_query(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
+    if (warp < (P4 ? 4 : HMAX))
+      rotate_query<P4>(a, seg.b, seg.kvh, warp, sprm, qfrag, kappa);
+    else if (P4 && warp < HMAX && lane == 0)
+      kappa[warp] = 0.f;  // rows of lo terms: their lanes' scores are not used
     __syncthreads();
     // the new token is appended by the warp that loads its tile, from here on (after the wait
     // and outside the CTA-wide barriers, so only that warp spends the time)
@@ -686,13 +733,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
         const bool landed = __all_sync(0xffffffffu, mbar_wait(&wbar[sl_i], (k_done / NSLOT) & 1, a.v.status));
         if (landed) ++k_wait; else aborted = true;
       }
-      if (!aborted) process_tile(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qfrag + lane * QF_WORDS, kap, a.kc, st);
+      if (!aborted) process_tile<P4>(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qfrag + lane * QF_WORDS, kap, a.kc, st);
       ++k_done;
       __syncwarp();
     }
 
     // ---- merge the warps (shared memory, two rounds: warps w+4, w+8, ... into w, then
     // slots 0..3), then one partial per (CTA, group)
+    if (P4) {  // add the lo columns (lanes t >= 2) into the hi columns of the same heads
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) st.acc[j][e] += __shfl_xor_sync(0xffffffffu, st.acc[j][e], 2);
+    }
     float lq = st.l;
     lq += __shfl_xor_sync(0xffffffffu, lq, 1);
     lq += __shfl_xor_sync(0xffffffffu, lq, 2);
@@ -860,11 +913,16 @@ static int launch_decode_impl(const LayerView& v, const void* q, int q_f32, int 
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     const int maxb = (int)DecSmem::bytes(DECODE_MAX_BATCH);
-    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-    cudaFuncSetAttribute(decode_kernel<FUSED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(decode_kernel<FUSED, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED, false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaFuncSetAttribute(decode_kernel<FUSED, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
+    cudaFuncSetAttribute(decode_kernel<FUSED, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx);
-  return (int)launch_pdl(decode_kernel<FUSED>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+  if (a.g_real <= 4)
+    return (int)launch_pdl(decode_kernel<FUSED, true>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
+                           (cudaStream_t)stream, a);
+  return (int)launch_pdl(decode_kernel<FUSED, false>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
                          (cudaStream_t)stream, a);
 }
 
