@@ -35,8 +35,8 @@ BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
 # kernel sources it was taken on: reported as roofline.traffic while their hash matches.
 DECODE_TRAFFIC = {"sources": ["rotated_bit_kv_iq_b200/csrc/iq_decode.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
                               "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"],
-                  "sha256": "0983cb34aaa81bbbd0a64c8cf446e82010b6c25e3943cc32c2dac88ec05c3722",
-                  "bytes": 13216512}
+                  "sha256": "928159a9458a1feaacb1bab5a75908973e6523ea1766d9f500d84dabf44ffb28",
+                  "bytes": 13215744}
 
 
 def decode_traffic():
