@@ -203,26 +203,38 @@ def time_graph(stack, steps, warmup, stream):
 
 
 def time_e2e(stack, steps, warmup, stream):
-    """Same step through the public API with host buffers: per layer the new K/V and the
-    queries come from pinned host memory and the attention output goes back to it."""
+    """Same step through the public API with host buffers: every step copies the new K/V and
+    the queries of all layers from pinned host memory (one copy per tensor), runs the
+    layers' iq_decode_step calls (captured once as a CUDA graph, like the device-timed
+    step) and copies all attention outputs back to pinned host memory."""
     torch = stack.torch
     hk = stack.knew.cpu().pin_memory()
     hv = stack.vnew.cpu().pin_memory()
     hq = stack.q.cpu().pin_memory()
     ho = torch.empty(stack.out.shape, dtype=torch.float32).pin_memory()
     dk, dv, dq = torch.empty_like(stack.knew), torch.empty_like(stack.vnew), torch.empty_like(stack.q)
+    dout = torch.empty_like(stack.out)
     Bd = stack.Bd
 
-    def step():
+    def layers():
         for l in range(stack.L):
-            dk[l].copy_(hk[l], non_blocking=True)
-            dv[l].copy_(hv[l], non_blocking=True)
-            dq[l].copy_(hq[l], non_blocking=True)
             Bd.iq_decode_step(stack.cache, l, dq[l], dk[l], dv[l], stack.ctx_dev, stack.max_ctx, stack.params,
-                              stack.out[l], stack.ws, stream)
-            ho[l].copy_(stack.out[l], non_blocking=True)
+                              dout[l], stack.ws, stream)
 
     with torch.cuda.stream(stream):
+        layers()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            layers()
+
+        def step():
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            graph.replay()
+            ho.copy_(dout, non_blocking=True)
+
         for _ in range(max(1, warmup)):
             step()
         stream.synchronize()
@@ -232,6 +244,7 @@ def time_e2e(stack, steps, warmup, stream):
             step()
         e1.record(stream)
         e1.synchronize()
+    del graph
     ms = e0.elapsed_time(e1) / steps
     h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
     d2h = ho.numel() * 4
