@@ -32,25 +32,37 @@ BYTES_PER_TOKEN_HEAD = 100  # 48 B K codes + 2 B K norm + 48 B V codes + 2 B V n
 BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
 # DRAM bytes (read + write) of one decode_kernel launch of the headline layer, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum, one 13.1 MB layer), valid only for the
-# kernel sources it was taken on: reported as roofline.traffic while their hash matches.
+# kernel sources it was taken on: reported as roofline.traffic while their code hash matches.
 DECODE_TRAFFIC = {"sources": ["rotated_bit_kv_iq_b200/csrc/iq_decode.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
                               "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"],
-                  "sha256": "928159a9458a1feaacb1bab5a75908973e6523ea1766d9f500d84dabf44ffb28",
+                  "sha256": "b66e8e08151dd41a269d3d625650ec35aa53c10118573fe62a728c3915db9035",
                   "bytes": 13215744}
+
+
+def kernel_source_hash(paths):
+    """SHA-256 of the code in the given C/C++/CUDA sources, comments and blank space removed
+    (a comment edit does not change the kernel the counters were taken on)."""
+    import hashlib
+    import re
+
+    h = hashlib.sha256()
+    here = os.path.dirname(os.path.abspath(__file__))
+    for f in paths:
+        with open(os.path.join(here, f), encoding="utf-8") as fh:
+            txt = fh.read()
+        txt = re.sub(r"/\*.*?\*/", " ", txt, flags=re.S)
+        txt = re.sub(r"//[^\n]*", " ", txt)
+        h.update(" ".join(txt.split()).encode())
+    return h.hexdigest()
 
 
 def decode_traffic():
     """Captured DRAM bytes per decode launch, or None once the kernel sources have changed."""
-    import hashlib
-    h = hashlib.sha256()
-    here = os.path.dirname(os.path.abspath(__file__))
     try:
-        for f in DECODE_TRAFFIC["sources"]:
-            with open(os.path.join(here, f), "rb") as fh:
-                h.update(fh.read())
+        digest = kernel_source_hash(DECODE_TRAFFIC["sources"])
     except OSError:
         return None
-    return DECODE_TRAFFIC["bytes"] if h.hexdigest() == DECODE_TRAFFIC["sha256"] else None
+    return DECODE_TRAFFIC["bytes"] if digest == DECODE_TRAFFIC["sha256"] else None
 
 
 HEADLINE = "qwen30b_32k"

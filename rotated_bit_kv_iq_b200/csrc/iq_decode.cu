@@ -22,10 +22,13 @@
 //     tile and head (127 / max P'), undone when the tile's value sums are accumulated;
 //   * values: O^T += V^T P' with the 128 coordinates as eight m-tiles, the 32 tokens as K and
 //     the heads as N; V blocks are laid out so that every A register is one table lookup.
-// s32 accumulators start at a magic constant so one float subtraction converts them.
+// s32 accumulators start at a magic constant so one float subtraction converts them.  With
+// at most four query heads per kv head the lower terms of q and P' ride in the mma rows and
+// columns the group leaves free (template P4), so a tile takes 48 mma instead of 72.
 // At a segment end the warps' (m, l, O) are merged in shared memory and written as one
-// partial per (CTA, group); the CTA that completes a group's count merges its partials,
-// normalises and applies R^T (no second kernel).
+// partial per (CTA, group), announced by a release-ordered count.  After its run, the k-th
+// CTA of a group (k < heads per kv head) waits for the group's count, merges head k (and
+// k + n, ... for n CTAs) over all partials, normalises and applies R^T: no second kernel.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
