@@ -240,10 +240,10 @@ def test_decode_gqa8_qwen_32k_layer_full():
     assert err < TOL, err
 
 
-@pytest.mark.parametrize("G", [1, 2, 3, 4, 6, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_ragged_paged_batch(G):
-    """Ragged contexts (0, 1, 15, 17, 300, 1000) over shuffled 64-token pages, group sizes of both
-    mma layouts (G <= 4 packs the lower terms into the free rows and columns), odd ones too."""
+    """Ragged contexts (0, 1, 15, 17, 300, 1000) over shuffled 64-token pages, every supported
+    group size (both mma layouts: G <= 4 packs the lower terms into the free rows and columns)."""
     Hkv = 2
     Hq = G * Hkv
     ctx = [0, 1, 15, 17, 300, 1000]
@@ -368,7 +368,7 @@ def _step_case(G, ctx, ps, maxp, layer=0, L=1, seed=0, graph_layers=None):
     return cache, P, cases
 
 
-@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_step_matches_oracle(G):
     """Fused append + attention: new tokens at odd and even positions, page boundaries, ctx = 1."""
     ctx = [1, 2, 64, 65, 129, 700]
