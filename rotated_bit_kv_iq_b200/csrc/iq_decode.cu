@@ -834,8 +834,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-      // the barrier orders the CTA's partial stores before this release-ordered arrival,
-      // which the thread does not wait for
+      // the barrier orders the CTA's partial stores before this release-ordered arrival (a
+      // reduction: no value comes back, so nothing waits for the counter itself)
       asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.ws.counters[gid]) : "memory");
     }
     x = seg.gstart + seg.hi;
