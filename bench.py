@@ -217,8 +217,10 @@ def time_graph(stack, steps, warmup, stream):
 def time_e2e(stack, steps, warmup, stream):
     """Same step through the public API with host buffers: every step copies the new K/V and
     the queries of all layers from pinned host memory (one copy per tensor), runs the
-    layers' iq_decode_step calls (captured once as a CUDA graph, like the device-timed
-    step) and copies all attention outputs back to pinned host memory."""
+    layers' iq_decode_step calls and copies all attention outputs back to pinned host memory.
+    Returned twice: with the layers' calls captured once as a CUDA graph (like the device-timed
+    step), and with every call made through the C ABI each step (host marshalling and argument
+    checks of 48 calls inside the timed region)."""
     torch = stack.torch
     hk = stack.knew.cpu().pin_memory()
     hv = stack.vnew.cpu().pin_memory()
@@ -233,20 +235,7 @@ def time_e2e(stack, steps, warmup, stream):
             Bd.iq_decode_step(stack.cache, l, dq[l], dk[l], dv[l], stack.ctx_dev, stack.max_ctx, stack.params,
                               dout[l], stack.ws, stream)
 
-    with torch.cuda.stream(stream):
-        layers()
-        stream.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            layers()
-
-        def step():
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dq.copy_(hq, non_blocking=True)
-            graph.replay()
-            ho.copy_(dout, non_blocking=True)
-
+    def timed(step):
         for _ in range(max(1, warmup)):
             step()
         stream.synchronize()
@@ -256,11 +245,36 @@ def time_e2e(stack, steps, warmup, stream):
             step()
         e1.record(stream)
         e1.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    with torch.cuda.stream(stream):
+        layers()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            layers()
+
+        def copy_in():
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+
+        def step_graph():
+            copy_in()
+            graph.replay()
+            ho.copy_(dout, non_blocking=True)
+
+        def step_direct():
+            copy_in()
+            layers()
+            ho.copy_(dout, non_blocking=True)
+
+        ms = timed(step_graph)
+        ms_direct = timed(step_direct)
     del graph
-    ms = e0.elapsed_time(e1) / steps
     h2d = hk.numel() * 2 + hv.numel() * 2 + hq.numel() * 2
     d2h = ho.numel() * 4
-    return ms, h2d, d2h
+    return ms, ms_direct, h2d, d2h
 
 
 def bench_encode(steps, warmup, device, stream):
@@ -323,7 +337,7 @@ def job_gbs(world, bytes_per_rank_step, ms):
     return world * bytes_per_rank_step / (ms * 1e-3) / 1e9
 
 
-def bench_serving(steps, warmup, device, stream, seed=0, world=1):
+def bench_serving(steps, warmup, device, stream, seed=0, world=1, n_layers=0):
     """Batched serving workload: one decode step of a 32-layer stack for 16 sequences with
     seeded contexts uniform in [2048, 32768], 64-token pages in a shuffled pool, 32 q / 8 kv
     heads; replayed as one CUDA graph."""
@@ -336,8 +350,8 @@ def bench_serving(steps, warmup, device, stream, seed=0, world=1):
     ctx = inputs.context_lengths(inputs.DATA_SEED, B, cfg["ctx_lo"], cfg["ctx_hi"])
     maxp = (int(ctx.max()) + ps - 1) // ps
     table = torch.from_numpy(inputs.page_permutation(inputs.DATA_SEED, B * maxp).reshape(B, maxp)).to(device)
-    stack = DecodeStack(B, cfg["n_q_heads"], cfg["n_kv_heads"], cfg["n_layers"], ctx, ps, device, seed=seed,
-                        block_table=table, n_pages=B * maxp)
+    stack = DecodeStack(B, cfg["n_q_heads"], cfg["n_kv_heads"], n_layers or cfg["n_layers"], ctx, ps, device,
+                        seed=seed, block_table=table, n_pages=B * maxp)
     ms, graph = time_graph(stack, steps, warmup, stream)
     del graph
     ms = max_over_ranks(ms, device)
@@ -347,7 +361,7 @@ def bench_serving(steps, warmup, device, stream, seed=0, world=1):
     achieved = layer_bytes / (kern_ms * 1e-3) / 1e9
     out = {
         "workload": f"serve_b16: decode step of 16 paged sequences (contexts {int(ctx.min())}..{int(ctx.max())}, "
-                    f"sum {int(ctx.sum())}), 32 q / 8 kv heads, d=128, 32 layers, 64-token pages",
+                    f"sum {int(ctx.sum())}), 32 q / 8 kv heads, d=128, {stack.L} layers, 64-token pages",
         "value": job_gbs(world, stack.bytes_per_step, ms), "unit": "GB/s", "ms_per_step": ms,
         "bytes_per_step": stack.bytes_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
@@ -360,15 +374,33 @@ def bench_serving(steps, warmup, device, stream, seed=0, world=1):
 
 
 # ------------------------------------------------------------------ oracle baseline
+def _cpu_info():
+    """CPU model and the cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except AttributeError:
+        affinity = os.cpu_count()
+    return model, affinity
+
+
 def oracle_decode_sample(seconds=12.0):
     """fp64 oracle decode attention on slices of the headline workload (one kv head, 8 query
-    heads, 32768 tokens per slice) until about `seconds` of CPU time; returns GB/s."""
-    from oracle import attention, encode
-    from rotated_bit_kv_iq_b200 import binding as Bd
+    heads, 32768 tokens per slice) until about `seconds` of CPU time; returns GB/s.  The oracle
+    draws its own rotation parameters and encodes the host generator's tokens itself."""
+    from oracle import attention, encode, rotation
     from rotated_bit_kv_iq_b200 import inputs
 
     T, G = 32768, 8
-    P = Bd.iq_init_rotation(inputs.ROTATION_SEED, 1, 4)
+    P = rotation.init_rotation(inputs.ROTATION_SEED, 1, 4)
     slices = []
     for h in range(2):  # encode outside the timed part
         ek = encode.encode(inputs.kv_tokens(0, 0, h, 0, 0, T), P[0, h])
@@ -392,6 +424,102 @@ def oracle_decode_sample(seconds=12.0):
     return gbs, n, el
 
 
+def oracle_config_rates():
+    """The oracle, single-threaded, on bounded samples of the other workloads (a few seconds):
+    encode Mvec/s on the tiny workload (512 tokens x K,V) and on one (layer, kv head) slice of the
+    ingest workload (32768 tokens x K,V = 65536 vectors, 1% Student-t tokens); decode attention
+    microseconds per layer on the tiny workload, one llama8b_8k layer (8 kv heads x 8192 tokens,
+    4 q heads each) and one qwen30b_32k layer (4 kv heads x 32768 tokens, 8 q heads each), each
+    extrapolated to the stack depth."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attention, encode, rotation
+    from rotated_bit_kv_iq_b200 import inputs
+
+    out = {"encode_mvec_s": {}, "decode_us_per_layer": {}}
+    with threadpool_limits(limits=1):
+        P1 = rotation.init_rotation(inputs.ROTATION_SEED, 1, 8)
+        # encode: tiny workload in full
+        x = [inputs.kv_tokens(0, 0, 0, w, 0, 512, n_outliers=2) for w in (0, 1)]
+        t0 = time.perf_counter()
+        enc_tiny = [encode.encode(xi, P1[0, 0]) for xi in x]
+        out["encode_mvec_s"]["tiny (1024 vectors)"] = 1024 / (time.perf_counter() - t0) / 1e6
+        # encode: one (layer, kv head) slice of the ingest workload
+        x = [inputs.kv_tokens(0, 0, 0, w, 0, 32768, heavy_frac=0.01) for w in (0, 1)]
+        t0 = time.perf_counter()
+        for xi in x:
+            encode.encode(xi, P1[0, 0])
+        el = time.perf_counter() - t0
+        out["encode_mvec_s"]["ingest_32k slice (65536 vectors)"] = 65536 / el / 1e6
+        out["encode_full_ingest_s_extrapolated"] = 16777216 / (65536 / el)
+        # decode: tiny
+        q = inputs.queries(0, 0, 1, 1, dtype="f32")[0].astype(np.float64)
+        t0 = time.perf_counter()
+        attention.attention_rotated(q, enc_tiny[0]["codes"][None], enc_tiny[0]["norm16"][None],
+                                    enc_tiny[1]["codes"][None], enc_tiny[1]["norm16"][None], P1[0, :1])
+        out["decode_us_per_layer"]["tiny (ctx 512, 1 head)"] = (time.perf_counter() - t0) * 1e6
+        # decode: one layer of the 8K and 32K workloads (encoding outside the timed part)
+        for name, Hkv, T, Hq, L in (("llama8b_8k", 8, 8192, 32, 1), ("qwen30b_32k", 4, 32768, 32, 48)):
+            ek = [encode.encode(inputs.kv_tokens(0, 0, h, 0, 0, T), P1[0, h]) for h in range(Hkv)]
+            ev = [encode.encode(inputs.kv_tokens(0, 0, h, 1, 0, T), P1[0, h]) for h in range(Hkv)]
+            q = inputs.queries(0, 0, 1, Hq)[0].astype(np.float64)
+            t0 = time.perf_counter()
+            attention.attention_rotated(q, np.stack([e["codes"] for e in ek]), np.stack([e["norm16"] for e in ek]),
+                                        np.stack([e["codes"] for e in ev]), np.stack([e["norm16"] for e in ev]),
+                                        P1[0, :Hkv])
+            us = (time.perf_counter() - t0) * 1e6
+            out["decode_us_per_layer"][f"{name} (one layer)"] = us
+            if L > 1:
+                out[f"decode_ms_per_step_{name}_extrapolated"] = us * L / 1e3
+    return out
+
+
+def oracle_parity_sample(stack, layer, head, seed=0):
+    """Parity of the timed step on one (layer, kv head): the oracle encodes the same fp16 tokens
+    the bench's cache was filled with (tokens 0..ctx-2, regenerated from their device generator)
+    plus the step's new token, its codes and norms are compared with the GPU's records
+    (iq_export_codes), and its attention for the group's query heads with the step's output."""
+    import torch
+
+    from oracle import attention, encode, rotation
+    from rotated_bit_kv_iq_b200 import inputs
+
+    assert stack.B == 1
+    Bd, dev = stack.Bd, stack.dev
+    T = int(stack.ctx[0])
+    G = stack.Hq // stack.Hkv
+    P = rotation.init_rotation(inputs.ROTATION_SEED, stack.L, stack.Hkv)[layer, head]
+    x = {}
+    for w, new in ((0, stack.knew), (1, stack.vnew)):
+        old = inputs.kv_tokens_device(seed, layer, stack.Hkv, w, T - 1, device=dev)[:, head].cpu().numpy()
+        x[w] = np.concatenate([old, new[layer, 0, 0, head:head + 1].cpu().numpy()])
+    enc = {w: encode.encode(x[w], P) for w in (0, 1)}
+    codes = torch.empty((stack.Hkv, T, 128), dtype=torch.uint8, device=dev)
+    norms = torch.empty((stack.Hkv, T), dtype=torch.int16, device=dev)
+    excluded = mismatched = 0
+    ulp = 0
+    for w in (0, 1):
+        Bd.iq_export_codes(stack.cache, layer, w, 0, 0, T, codes, norms)
+        torch.cuda.synchronize()
+        gc = codes[head].cpu().numpy()
+        gn = norms[head].cpu().numpy().view(np.uint16)
+        near = enc[w]["near"]
+        excluded += int(near.sum())
+        mismatched += int(((gc != enc[w]["codes"]) & ~near).sum())
+        ulp = max(ulp, int(np.abs(gn.astype(np.int64) - enc[w]["norm16"].astype(np.int64)).max()))
+    q = stack.q[layer, 0, head * G:(head + 1) * G].cpu().numpy().astype(np.float64)
+    ref = attention.attention_rotated(q, enc[0]["codes"][None], enc[0]["norm16"][None], enc[1]["codes"][None],
+                                      enc[1]["norm16"][None], P[None])
+    got = stack.out[layer, 0, head * G:(head + 1) * G].cpu().numpy().astype(np.float64)
+    den = np.maximum(np.abs(ref).max(axis=1), 1e-300)
+    err = float((np.abs(got - ref).max(axis=1) / den).max())
+    n_codes = 2 * T * 128
+    return {"sample": f"layer {layer}, kv head {head} ({G} q heads), {T} tokens of K and V, timed step's output",
+            "max_rel_err": err, "tolerance": 2e-3, "code_mismatches_outside_band": mismatched,
+            "excluded_codes": excluded, "codes_checked": n_codes, "exclusion_rate": excluded / n_codes,
+            "norm_ulp_max": ulp, "pass": bool(err < 2e-3 and mismatched == 0 and ulp <= 1)}
+
+
 def reference_arm(args):
     """--impl reference: the oracle on bounded samples of the headline workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -403,13 +531,16 @@ def reference_arm(args):
         if i >= args.warmup:
             per_step.append((gbs, el))
     gbs = float(np.mean([g for g, _ in per_step]))
-    sample = "fp64 oracle decode attention, 1 kv head x 8 q heads x 32768 tokens per slice, repeated ~2 s per step"
+    model, affinity = _cpu_info()
+    sample = ("fp64 oracle decode attention, 1 kv head x 8 q heads x 32768 tokens per slice; each 'step' is a "
+              "~2 s sampling window of repeated slices (ms_per_step is that window, not a decode step)")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([e for _, e in per_step]) * 1e3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": HEADLINE + " (oracle sample)"},
-        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "cpu_model": model, "affinity_cores": affinity},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -425,7 +556,10 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="headline workload only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed step's output")
     ap.add_argument("--layers", type=int, default=0, help="override the stack depth (profiling runs)")
+    ap.add_argument("--only", default="", choices=["", "serving", "encode"],
+                    help="run one secondary workload alone (profiling runs); no headline line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -455,6 +589,16 @@ def main():
 
     Bd.lib()
     stream = torch.cuda.Stream(device=dev)
+    if args.only:
+        if args.only == "serving":
+            res = bench_serving(args.steps, args.warmup, dev, stream, seed=rank, world=world, n_layers=args.layers)
+        else:
+            res = bench_encode(args.steps, args.warmup, dev, stream)
+        if rank == 0:
+            print(json.dumps({"only": args.only, **res}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     cfg = inputs.CONFIGS[HEADLINE]
     n_layers = args.layers or cfg["n_layers"]
     stack = DecodeStack(cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], n_layers, [cfg["ctx"]],
@@ -478,14 +622,16 @@ def main():
     layer_bytes = int(stack.ctx.sum()) * stack.Hkv * BYTES_PER_TOKEN_HEAD
     peak, peak_kind = _peaks()
     achieved = layer_bytes / (kern_ms * 1e-3) / 1e9
-    e2e_ms, h2d, d2h = time_e2e(stack, args.steps, args.warmup, stream)
+    e2e_ms, e2e_direct_ms, h2d, d2h = time_e2e(stack, args.steps, args.warmup, stream)
     e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_direct_ms = max_over_ranks(e2e_direct_ms, dev)
     del graph
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 tensor-core inputs, f32 accumulate, 3-bit codes", "data": "synthetic",
+        "dtype": "int8 hi/lo tensor-core products (s32 accumulate); fp32 softmax, scaling and accumulation "
+                 "across tiles; 3-bit codes, binary16 norms", "data": "synthetic",
         "config": {"workload": "qwen30b_32k: decode step (append + attend) B=1, 32 q / 4 kv heads, d=128, "
                                "48 layers, ctx 32768, packed 3-bit cache", "l2": "inputs larger than L2 (629 MB/step)",
                    "graph": f"{stack.L}-layer step replayed as one CUDA graph", "layers": stack.L,
@@ -495,10 +641,17 @@ def main():
                      "kernel": "decode_kernel (one launch per layer: append + split attention + merge), CUDA-graph step time / layers",
                      "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
         "e2e": {"value": job_gbs(world, stack.bytes_per_step, e2e_ms), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "calls": "48 iq_decode_step calls captured once as a CUDA graph, replayed each step",
+                "direct_calls": {"value": job_gbs(world, stack.bytes_per_step, e2e_direct_ms), "unit": "GB/s",
+                                 "ms_per_step": e2e_direct_ms,
+                                 "calls": "48 iq_decode_step calls through the C ABI every step"}},
         "gpu_launches": stack.L * DecodeStack.launches_per_layer * args.steps,
         "clocks": clk.summary(),
     }
+    if rank == 0 and not args.no_parity:
+        # the timed step's own output and records against the oracle, on one (layer, kv head)
+        result["parity"] = oracle_parity_sample(stack, stack.L - 1, 1 % stack.Hkv, seed=rank)
     del stack
     torch.cuda.empty_cache()
 
@@ -524,8 +677,10 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_cpu:
         gbs, n, el = oracle_decode_sample(args.cpu_seconds)
+        model, affinity = _cpu_info()
         result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                  "sample": f"{n} x (1 kv head, 8 q heads, 32768 tokens) decode slices in {el:.1f} s"}
+                                  "sample": f"{n} x (1 kv head, 8 q heads, 32768 tokens) decode slices in {el:.1f} s",
+                                  "cpu_model": model, "affinity_cores": affinity, **oracle_config_rates()}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:

@@ -114,13 +114,19 @@ iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size
                          size_t* pool_bytes_host);
 
 /* Rotation parameters from a seed (host-only; writes n_layers*n_kv_heads*256 floats to
- * params_host).  Each quaternion is drawn uniformly from the unit 3-sphere by Marsaglia's
+ * params_host).  Defined by: RotaryQuant abstract (arXiv 2608.08081), 256 parameters per head
+ * for the block-diagonal SO(4) stage; "RotaryQuant" (rebasdaily.com), section
+ * "妙处不只是压缩，而是不再展开", the WHT + SO(4) structure they parametrise.  Each quaternion is drawn uniformly from the unit 3-sphere by Marsaglia's
  * method from a splitmix64 counter stream keyed by (seed, layer, head, block, side); the
  * pages publish no parameter values, they fix only their number (256 per head).
  * Errors: IQ_ERR_INVALID_ARG for NULL params_host or non-positive sizes. */
 iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, float* params_host);
 
 /* Quantise-and-append: encode n_new new tokens of every sequence into layer `layer`.
+ * Defined by: "RotaryQuant" (rebasdaily.com), section "妙处不只是压缩，而是不再展开" (rotate,
+ * then scalar-quantise each coordinate to 3 bits and pack); "压缩与速度的博弈" (zhichai.net),
+ * sections "Beta 分布的魔力" (rotated unit-vector coordinates ~ N(0, 1/d)) and "Lloyd-Max 最优量化"
+ * (the quantiser).
  *   k_dev, v_dev : fp16 [batch][n_new][Hkv][128]; either may be NULL (that side skipped).
  *   start_pos_dev: int32 [batch], position of each sequence's first new token.
  *   params_dev   : float32 [L][Hkv][32][2][4].
@@ -143,6 +149,11 @@ iq_status iq_encode_append(const iq_cache* cache, int32_t layer, const void* k_d
 size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx);
 
 /* Decode attention over the packed cache of layer `layer`.
+ * Defined by: "RotaryQuant" (rebasdaily.com), section "妙处不只是压缩，而是不再展开" and its
+ * abstract (attention directly on the packed tensors: rotated query, scores, softmax, value sum,
+ * one inverse rotation); "RotorQuant" (sd114.wiki), section "3. V 缓存的逆旋转修复" (the value sum
+ * goes back through the inverse rotation); "压缩与速度的博弈" (zhichai.net), section
+ * "为什么压缩 KV 缓存这么难？" (softmax(Q K^T / sqrt(d)) V).
  *   q_dev        : [batch][n_q_heads][128], fp16 (IQ_F16) or fp32 (IQ_F32).
  *   ctx_len_dev  : int32 [batch], tokens 0..ctx_len-1 of each sequence are attended;
  *                  0 gives a zero output row; values outside [0, max_ctx] are clamped
@@ -168,6 +179,8 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
                               size_t workspace_bytes, iq_stream_t stream);
 
 /* Decode step: append one new token to every sequence and attend over it, in one kernel.
+ * Defined by: the two calls above; "RotorQuant" (sd114.wiki), section "2. 延迟量化策略" (a token
+ * generated during decoding is quantised when it is inserted into the cache).
  *   k_new_dev, v_new_dev: fp16 [batch][Hkv][128], the new token's K and V; it is encoded (as by
  *                  iq_encode_append) into position ctx_len[b]-1 of sequence b.
  *   Other arguments and the result as for iq_decode_attention over positions [0, ctx_len[b]);
@@ -200,13 +213,18 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
  * max_ctx) exceeds IQ_NOALLOC_SCRATCH_BYTES.  All calls on a device share the one array: calls
  * that overlap on the GPU (other streams, or a second call before the first has finished on a
  * stream that is not ordered after it) race on it.  Each call clears the array's arrival
- * counters (cudaMemsetAsync on its stream) before the kernel; nothing else has to start zeroed. */
+ * counters (cudaMemsetAsync on its stream) before the kernel; nothing else has to start zeroed.
+ * The looked-up address is kept for the life of the process: after cudaDeviceReset (or anything
+ * else that destroys the device's primary context) it is stale, and this entry point must not
+ * be called on that device again. */
 iq_status iq_decode_attention_noalloc(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype,
                                       int32_t batch, int32_t n_q_heads, const int32_t* ctx_len_dev,
                                       int32_t max_ctx, const float* params_dev, float* out_dev,
                                       iq_stream_t stream);
 
-/* Read back tokens [t0, t0+n) of sequence `seq` in layer `layer` as canonical codes:
+/* Read back tokens [t0, t0+n) of sequence `seq` in layer `layer` as canonical codes (a test
+ * and inspection utility: the pages define no such call; it undoes only this library's own
+ * bit layout):
  *   codes_dev: uint8 [Hkv][n][128] (coordinate order), norms_dev: uint16 [Hkv][n] or NULL.
  *   kv: 0 = K pool, 1 = V pool.  Host-checked against the sequence capacity. */
 iq_status iq_export_codes(const iq_cache* cache, int32_t layer, int32_t kv, int32_t seq, int32_t t0,

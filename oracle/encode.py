@@ -64,7 +64,9 @@ def encode(x16, params_head, bits=3):
     u = math.sqrt(D) * z
     _, b = codebook(bits)
     codes = quantise(u, bits)
-    near = np.any(np.abs(u[..., None] - b) < BOUNDARY_BAND, axis=-1)
+    near = np.zeros(u.shape, dtype=bool)
+    for bj in b:  # within the band of any boundary
+        near |= np.abs(u - bj) < BOUNDARY_BAND
     n16, sat = norm_to_fp16_bits(n)
     return {"codes": codes, "norm16": n16, "u": u, "near": near, "saturated": sat, "norm": n}
 

@@ -33,7 +33,10 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <algorithm>
+#include <map>
 #include <mutex>
+#include <tuple>
 
 #include "iq_device.cuh"
 
@@ -79,15 +82,33 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two fit; else
-// one, which leaves the other half of every SM free for the next kernel's CTAs to start their
-// loads early (programmatic dependent launch).
-int decode_ctas(int batch, int n_kv_heads, int max_ctx) {
+// CTAs of one launch that the SMs hold at once: the occupancy calculator's figure for this
+// kernel instantiation at the launch's dynamic shared memory (rounded up to 1 KB), cached per
+// device.  The final merge waits for other CTAs of the same grid, so a grid must never exceed it.
+static int resident_per_sm(const void* fn, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const size_t bucket = (smem + 1023) & ~(size_t)1023;
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, size_t>, int> memo;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev, fn, bucket);
+  const auto it = memo.find(key);
+  if (it != memo.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DEC_THREADS, bucket) != cudaSuccess) n = 0;
+  memo[key] = n;
+  return n;
+}
+
+// Two CTAs per SM when the problem is large (each warp gets >= 16 tiles) and two are resident;
+// else one, which leaves the other half of every SM free for the next kernel's CTAs to start
+// their loads early (programmatic dependent launch).  0 when not even one CTA fits.
+int decode_ctas(int batch, int n_kv_heads, int max_ctx, int resident) {
   const int n_sm = sm_count();
   const long long tiles = (long long)batch * n_kv_heads * ((max_ctx + TT - 1) / TT);
-  const bool fits2 = 2 * (DecSmem::bytes(batch) + 1024) <= 228 * 1024;
   const bool big = tiles >= (long long)n_sm * 2 * DEC_WARPS * 16;
-  return n_sm * ((fits2 && big) ? 2 : 1);
+  return n_sm * std::min(resident, big ? 2 : 1);
 }
 
 struct Workspace {
@@ -921,12 +942,11 @@ static int launch_decode_impl(const LayerView& v, const void* q, int q_f32, int 
     cudaFuncSetAttribute(decode_kernel<FUSED, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
     cudaFuncSetAttribute(decode_kernel<FUSED, true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
-  const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx);
-  if (a.g_real <= 4)
-    return (int)launch_pdl(decode_kernel<FUSED, true>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
-                           (cudaStream_t)stream, a);
-  return (int)launch_pdl(decode_kernel<FUSED, false>, dim3(ctas), dim3(DEC_THREADS), DecSmem::bytes(batch),
-                         (cudaStream_t)stream, a);
+  auto kern = a.g_real <= 4 ? decode_kernel<FUSED, true> : decode_kernel<FUSED, false>;
+  const size_t smem = DecSmem::bytes(batch);
+  const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx, resident_per_sm((const void*)kern, smem));
+  if (ctas == 0) return (int)cudaErrorInvalidConfiguration;
+  return (int)launch_pdl(kern, dim3(ctas), dim3(DEC_THREADS), smem, (cudaStream_t)stream, a);
 }
 
 int launch_decode(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads, const int32_t* ctx_len,

@@ -66,8 +66,9 @@ int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void*
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
                   uint16_t* norms, const KernelConsts& kc, void* stream);
 
-// Decode grid (host): CTAs of one decode launch on the current device.
-int decode_ctas(int batch, int n_kv_heads, int max_ctx);
+// Decode grid (host): CTAs of one decode launch on the current device, given how many CTAs of
+// the kernel an SM holds at once.
+int decode_ctas(int batch, int n_kv_heads, int max_ctx, int resident_per_sm);
 size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx);
 size_t decode_counter_bytes(int batch, int n_kv_heads);  // leading bytes that must be zero between calls
 constexpr int DECODE_MAX_BATCH = 2048;  // sequences per decode call (per-CTA plan in shared memory)

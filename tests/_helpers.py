@@ -1,9 +1,18 @@
-"""Shared test utilities: oracle-side encoding of seeded inputs and cache upload."""
+"""Shared test utilities: oracle-side encoding of seeded inputs, cache upload, guard bands and
+the record of parity margins."""
 
 import numpy as np
 
-from oracle import attention, encode, packing
+from oracle import attention, encode, packing, rotation
 from rotated_bit_kv_iq_b200 import inputs
+
+TILE = 32
+
+
+def oracle_params(seed, n_layers, n_kv_heads):
+    """Rotation parameters drawn by the oracle's own generator (the product's generator is
+    checked against it bit for bit in the host tests; the oracle never uses the product's)."""
+    return rotation.init_rotation(seed, n_layers, n_kv_heads)
 
 
 def oracle_encode_stream(params_head, layer, head, which, t0, n, n_outliers=4, heavy_frac=0.0, seed=inputs.DATA_SEED):
@@ -12,28 +21,55 @@ def oracle_encode_stream(params_head, layer, head, which, t0, n, n_outliers=4, h
     return x, encode.encode(x, params_head)
 
 
-def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n16):
-    """Write oracle-packed records of tokens 0..T-1 of one sequence/head into the device pool.
+def tile_records(k_codes, k_n16, v_codes, v_n16):
+    """Oracle-packed tile records of tokens 0..T-1 of one (sequence, kv head): (ceil(T/32), 3200)
+    uint8; slots past T are zero."""
+    T = k_codes.shape[0]
+    nt = (T + TILE - 1) // TILE
+    krec = np.zeros((nt * TILE, 48), np.uint8)
+    krec[:T] = packing.pack_k_fast(k_codes)
+    vrec = np.zeros((nt * 2, 768), np.uint8)
+    vb = packing.pack_v_fast(v_codes)
+    vrec[:vb.shape[0]] = vb
+    kn = np.zeros(nt * TILE, np.uint16)
+    vn = np.zeros(nt * TILE, np.uint16)
+    kn[:T] = k_n16
+    vn[:T] = v_n16
+    rec = np.concatenate([krec.reshape(nt, TILE * 48), vrec.reshape(nt, 2 * 768),
+                          kn.reshape(nt, TILE).view(np.uint8), vn.reshape(nt, TILE).view(np.uint8)], axis=1)
+    assert rec.shape[1] == 3200
+    return rec
 
-    seq_pages: physical page ids of the sequence, in order."""
+
+def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n16):
+    """Write oracle-packed records of tokens 0..T-1 of one sequence/head into the device pool
+    (one host-to-device copy).  seq_pages: physical page ids of the sequence, in order."""
     import torch
 
     ps = cache.page_size
     T = k_codes.shape[0]
-    krec = torch.from_numpy(packing.pack_k_fast(k_codes))
-    vrec = torch.from_numpy(packing.pack_v_fast(v_codes))
-    kn = torch.from_numpy(np.asarray(k_n16).view(np.int16).copy())
-    vn = torch.from_numpy(np.asarray(v_n16).view(np.int16).copy())
-    kv_k, kv_v = cache.k_code_view(), cache.v_code_view()
-    k_nv, v_nv = cache.k_norm_view(), cache.v_norm_view()
-    for t0 in range(0, T, 32):  # one tile record (32 slots of one page) at a time
-        page, slot = int(seq_pages[t0 // ps]), t0 % ps
-        tile, m = slot // 32, min(32, T - t0)
-        kv_k[layer, page, head, tile, :m] = krec[t0:t0 + m].to(kv_k.device)
+    if T == 0:
+        return
+    rec = torch.from_numpy(tile_records(k_codes, k_n16, v_codes, v_n16)).to(cache.pool.device)
+    nt = rec.shape[0]
+    t0 = np.arange(nt) * TILE
+    pages = torch.as_tensor(np.asarray(seq_pages)[t0 // ps].astype(np.int64), device=cache.pool.device)
+    tiles = torch.as_tensor((t0 % ps) // TILE, dtype=torch.int64, device=cache.pool.device)
+    tv = cache.tiles()
+    # a partial last tile keeps the pool's bytes of the slots past T
+    full = nt if T % TILE == 0 else nt - 1
+    if full:
+        tv[layer, pages[:full], head, tiles[:full]] = rec[:full]
+    if full < nt:
+        m = T - full * TILE
+        last = tv[layer, pages[full], head, tiles[full]].clone()
+        r = rec[full]
+        last[:48 * m] = r[:48 * m]
         nb = (m + 15) // 16
-        kv_v[layer, page, head, tile, :nb] = vrec[t0 // 16:t0 // 16 + nb].to(kv_v.device)
-        k_nv[layer, page, head, tile, :m] = kn[t0:t0 + m].to(k_nv.device)
-        v_nv[layer, page, head, tile, :m] = vn[t0:t0 + m].to(v_nv.device)
+        last[1536:1536 + 768 * nb] = r[1536:1536 + 768 * nb]
+        last[3072:3072 + 2 * m] = r[3072:3072 + 2 * m]
+        last[3136:3136 + 2 * m] = r[3136:3136 + 2 * m]
+        tv[layer, pages[full], head, tiles[full]] = last
 
 
 def max_rel_err(out, ref):
@@ -47,3 +83,38 @@ def max_rel_err(out, ref):
 
 def oracle_attention(q, k_codes, k_n16, v_codes, v_n16, params):
     return attention.attention_rotated(q, k_codes, k_n16, v_codes, v_n16, params)
+
+
+PARITY_RECORDS = []
+
+
+def record_parity(case, max_rel_err=None, excluded=None, codes=None, norm_ulp=None):
+    """Keep one case's parity margins for the terminal summary (tests/conftest.py)."""
+    PARITY_RECORDS.append({"case": case, "max_rel_err": max_rel_err, "excluded": excluded, "codes": codes,
+                                    "norm_ulp": norm_ulp})
+
+
+# ------------------------------------------------------------------ guard bands
+CANARY = 0x5A  # byte written before and after every output and workspace a GPU test hands to a kernel
+GUARD = 4096
+
+
+class Guarded:
+    """A device buffer with GUARD bytes of canary on each side; `.t` is the usable view."""
+
+    def __init__(self, shape, dtype, fill=None, device="cuda"):
+        import torch
+
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.raw = torch.full((GUARD + ((n + 255) // 256) * 256 + GUARD,), CANARY, dtype=torch.uint8, device=device)
+        self.n = n
+        body = self.raw[GUARD:GUARD + n]
+        self.t = body.view(dtype).view(*shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, label=""):
+        head = self.raw[:GUARD]
+        tail = self.raw[GUARD + self.n:]
+        assert bool((head == CANARY).all()), f"{label}: bytes written before the buffer"
+        assert bool((tail == CANARY).all()), f"{label}: bytes written after the buffer"

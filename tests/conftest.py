@@ -28,3 +28,22 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    # parity margins recorded by the GPU tests (tests/_helpers.record_parity), printed so that
+    # every run's log shows how much of each tolerance was used
+    from tests._helpers import PARITY_RECORDS
+
+    if not PARITY_RECORDS:
+        return
+    tr = terminalreporter
+    tr.section("parity margins (GPU vs fp64 oracle)")
+    tr.write_line(f"{'case':<58} {'max_rel_err':>11} {'of 2e-3':>7} {'excluded':>9} {'codes':>10} "
+                  f"{'norm_ulp':>8}")
+    for r in PARITY_RECORDS:
+        err = r.get("max_rel_err")
+        tr.write_line(
+            f"{r['case'][:58]:<58} {('%.3e' % err) if err is not None else '-':>11} "
+            f"{('%.0f%%' % (100 * err / 2e-3)) if err is not None else '-':>7} "
+            f"{r.get('excluded', '-')!s:>9} {r.get('codes', '-')!s:>10} {r.get('norm_ulp', '-')!s:>8}")

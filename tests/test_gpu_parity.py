@@ -13,7 +13,7 @@ import torch
 from oracle import attention, encode, packing
 from rotated_bit_kv_iq_b200 import binding as B
 from rotated_bit_kv_iq_b200 import inputs
-from tests._helpers import max_rel_err, upload_sequence
+from tests._helpers import Guarded, max_rel_err, oracle_params, record_parity, upload_sequence
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -41,7 +41,7 @@ def _export(cache, layer, kv, seq, t0, n):
     return codes.cpu().numpy(), norms.cpu().numpy().view(np.uint16)
 
 
-def _check_codes(gpu_codes, gpu_n16, ref, label, cap=True):
+def _check_codes(gpu_codes, gpu_n16, ref, label, cap=True, record=None):
     near = ref["near"]
     diff = gpu_codes != ref["codes"]
     bad = diff & ~near
@@ -53,12 +53,16 @@ def _check_codes(gpu_codes, gpu_n16, ref, label, cap=True):
     assert np.all(np.abs(gpu_codes.astype(int) - ref["codes"].astype(int))[diff] == 1)
     ulp = np.abs(gpu_n16.astype(np.int64) - ref["norm16"].astype(np.int64))
     assert ulp.max() <= 1, f"{label}: norm off by {ulp.max()} ulp"
+    if record is not None:
+        record["excluded"] = record.get("excluded", 0) + int(near.sum())
+        record["codes"] = record.get("codes", 0) + int(near.size)
+        record["norm_ulp"] = max(record.get("norm_ulp", 0), int(ulp.max()))
 
 
 # ------------------------------------------------------------------------- encode
 def test_encode_tiny_config_matches_oracle():
     """Single head, 512 tokens, 2 outlier channels (the tiny workload); records checked byte by byte."""
-    T, P = 512, B.iq_init_rotation(inputs.ROTATION_SEED, 1, 1)
+    T, P = 512, oracle_params(inputs.ROTATION_SEED, 1, 1)
     cache = B.PagedCache(1, 1, 512, 1)
     xs, refs = {}, {}
     for which in (0, 1):
@@ -69,9 +73,10 @@ def test_encode_tiny_config_matches_oracle():
     start = torch.zeros(1, dtype=torch.int32, device=DEV)
     B.iq_encode_append(cache, 0, k, v, start, _params_dev(P))
     torch.cuda.synchronize()
+    rec = {}
     for which in (0, 1):
         codes, n16 = _export(cache, 0, which, 0, 0, T)
-        _check_codes(codes[0], n16[0], refs[which], f"kv={which}")
+        _check_codes(codes[0], n16[0], refs[which], f"kv={which}", record=rec)
         # byte-level format check: oracle packer on the GPU's codes where they were excluded
         expect = np.where(refs[which]["near"], codes[0], refs[which]["codes"])
         if which == 0:
@@ -81,12 +86,13 @@ def test_encode_tiny_config_matches_oracle():
             got = cache.v_code_view()[0, 0, 0].reshape(-1, 768)[: T // 16].cpu().numpy()
             np.testing.assert_array_equal(got, packing.pack_v_fast(expect))
     assert cache.status.item() == 0
+    record_parity("encode tiny (512 tok, 1 head)", **rec)
 
 
 def test_encode_ragged_paged_multi_sequence():
     """3 sequences, 2 kv heads, 64-token pages in a shuffled pool, odd start positions."""
     Hkv, ps, n_pages, L = 2, 64, 24, 2
-    P = B.iq_init_rotation(7, L, Hkv)
+    P = oracle_params(7, L, Hkv)
     perm = inputs.page_permutation(3, n_pages)
     table = torch.from_numpy(perm.reshape(3, 8)).to(DEV)
     cache = B.PagedCache(L, Hkv, ps, n_pages, block_table=table)
@@ -104,19 +110,21 @@ def test_encode_ragged_paged_multi_sequence():
                        torch.from_numpy(starts).to(DEV), _params_dev(P))
     torch.cuda.synchronize()
     assert cache.status.item() == 0
+    rec = {}
     for b in range(3):
         for which in (0, 1):
             codes, n16 = _export(cache, layer, which, b, int(starts[b]), n_new)
             for h in range(Hkv):
                 ref = encode.encode(X[which][b, :, h], P[layer, h])
-                _check_codes(codes[h], n16[h], ref, f"b={b} h={h} kv={which}")
+                _check_codes(codes[h], n16[h], ref, f"b={b} h={h} kv={which}", record=rec)
+    record_parity("encode ragged paged (3 seq, 77 tok, 5% t3)", **rec)
 
 
 def test_encode_single_token_appends_keep_block_neighbours():
     """Decode-style appends of one token at a time: every V write changes only its own bits of
     a 16-token V block (the other tokens' codes must survive)."""
     Hkv, L = 2, 1
-    P = B.iq_init_rotation(5, L, Hkv)
+    P = oracle_params(5, L, Hkv)
     cache = B.PagedCache(L, Hkv, 64, 2)
     T = 9
     X = {w: np.stack([inputs.kv_tokens(21, 0, h, w, 0, T) for h in range(Hkv)], axis=1) for w in (0, 1)}
@@ -137,7 +145,7 @@ def test_encode_edge_values():
     """Zero vector, saturating norm, fp16 subnormals, a single hot coordinate.  Constant vectors
     rotate to exact zeros (= the middle boundary), so the exclusion-rate cap does not apply;
     excluded codes must still be one of the two adjacent cells."""
-    P = B.iq_init_rotation(1, 1, 1)
+    P = oracle_params(1, 1, 1)
     x = np.zeros((6, 128), dtype=np.float16)
     x[1] = 60000.0
     x[2] = np.float16(6e-8)
@@ -161,7 +169,7 @@ def test_encode_ingest_layer_sampled(heavy):
     """Ingest shape (32768 tokens x 8 kv heads, one layer, 1% Student-t tokens) in the bench's
     launch configuration; sampled token ranges of every head checked against the oracle."""
     Hkv, T, L = 8, 32768, 1
-    P = B.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)
+    P = oracle_params(inputs.ROTATION_SEED, L, Hkv)
     cache = B.PagedCache(L, Hkv, T, 1)
     X = {w: np.stack([inputs.kv_tokens(0, 0, h, w, 0, T, heavy_frac=heavy) for h in range(Hkv)], axis=1)[None]
          for w in (0, 1)}
@@ -169,12 +177,14 @@ def test_encode_ingest_layer_sampled(heavy):
                        torch.zeros(1, dtype=torch.int32, device=DEV), _params_dev(P))
     torch.cuda.synchronize()
     rng = np.random.default_rng(1)
+    rec = {}
     for which in (0, 1):
         for h in range(Hkv):
             t0 = int(rng.integers(0, T - 1024))
             codes, n16 = _export(cache, 0, which, 0, t0, 1024)
             ref = encode.encode(X[which][0, t0:t0 + 1024, h], P[0, h])
-            _check_codes(codes[h], n16[h], ref, f"h={h} kv={which}")
+            _check_codes(codes[h], n16[h], ref, f"h={h} kv={which}", record=rec)
+    record_parity(f"encode ingest layer sampled (heavy {heavy})", **rec)
 
 
 # ------------------------------------------------------------------------- decode
@@ -189,31 +199,36 @@ def _oracle_cache(P_layer, layer, Hkv, T, seed=0, n_outliers=4):
 
 
 def _decode(cache, layer, q, ctx, max_ctx, P):
+    """iq_decode_attention with guard bands around the output and the workspace."""
     Bn, Hq = q.shape[0], q.shape[1]
-    out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
-    ws = torch.zeros(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx), dtype=torch.uint8, device=DEV)
+    out = Guarded((Bn, Hq, 128), torch.float32, fill=float("nan"))
+    ws = Guarded((B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx),), torch.uint8, fill=0)
     B.iq_decode_attention(cache, layer, q, torch.from_numpy(np.asarray(ctx, np.int32)).to(DEV), max_ctx,
-                          _params_dev(P), out, ws)
+                          _params_dev(P), out.t, ws.t)
     torch.cuda.synchronize()
-    return out.cpu().numpy()
+    out.check("out")
+    ws.check("workspace")
+    return out.t.cpu().numpy()
 
 
 def test_decode_tiny_config():
     """Single head, fp32 query, context 512 (group size 1)."""
-    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, 1)
+    P = oracle_params(inputs.ROTATION_SEED, 1, 1)
     kc, kn, vc, vn = _oracle_cache(P[0], 0, 1, 512, n_outliers=2)
     cache = B.PagedCache(1, 1, 512, 1)
     upload_sequence(cache, 0, [0], 0, kc[0], kn[0], vc[0], vn[0])
     q = inputs.queries(0, 0, 1, 1, dtype="f32")
     out = _decode(cache, 0, torch.from_numpy(q).to(DEV), [512], 512, P)
     ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[0])
-    assert max_rel_err(out[0], ref) < TOL
+    err = max_rel_err(out[0], ref)
+    record_parity("decode tiny (G=1, fp32 q, ctx 512)", max_rel_err=err)
+    assert err < TOL
 
 
 def test_decode_gqa4_llama_8k_full():
     """Llama-3.1-8B-shaped layer: 32 q heads / 8 kv heads, context 8192, fp16 q; all heads."""
     Hq, Hkv, T = 32, 8, 8192
-    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, Hkv)
+    P = oracle_params(inputs.ROTATION_SEED, 1, Hkv)
     kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, T)
     cache = B.PagedCache(1, Hkv, T, 1)
     for h in range(Hkv):
@@ -222,13 +237,14 @@ def test_decode_gqa4_llama_8k_full():
     out = _decode(cache, 0, torch.from_numpy(q).to(DEV), [T], T, P)
     ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[0])
     err = max_rel_err(out[0], ref)
+    record_parity("decode llama8b 8K layer, all heads (G=4)", max_rel_err=err)
     assert err < TOL, err
 
 
 def test_decode_gqa8_qwen_32k_layer_full():
     """Qwen3-30B-A3B-shaped layer: 32 q heads / 4 kv heads, context 32768 (a later layer index)."""
     Hq, Hkv, T, L, layer = 32, 4, 32768, 3, 2
-    P = B.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)
+    P = oracle_params(inputs.ROTATION_SEED, L, Hkv)
     kc, kn, vc, vn = _oracle_cache(P[layer], layer, Hkv, T)
     cache = B.PagedCache(L, Hkv, T, 1)
     for h in range(Hkv):
@@ -237,6 +253,7 @@ def test_decode_gqa8_qwen_32k_layer_full():
     out = _decode(cache, layer, torch.from_numpy(q).to(DEV), [T], T, P)
     ref = attention.attention_rotated(q[0].astype(np.float64), kc, kn, vc, vn, P[layer])
     err = max_rel_err(out[0], ref)
+    record_parity("decode qwen30b 32K layer, all heads (G=8)", max_rel_err=err)
     assert err < TOL, err
 
 
@@ -249,7 +266,7 @@ def test_decode_ragged_paged_batch(G):
     ctx = [0, 1, 15, 17, 300, 1000]
     ps, maxp = 64, 16
     n_pages = len(ctx) * maxp
-    P = B.iq_init_rotation(3, 1, Hkv)
+    P = oracle_params(3, 1, Hkv)
     perm = inputs.page_permutation(9, n_pages)
     table_np = perm.reshape(len(ctx), maxp)
     cache = B.PagedCache(1, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
@@ -265,6 +282,8 @@ def test_decode_ragged_paged_batch(G):
         refs.append(attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[0]))
     out = _decode(cache, 0, torch.from_numpy(q).to(DEV), ctx, 1024, P)
     assert np.all(out[0] == 0)
+    err = max(max_rel_err(out[b], refs[b]) for b in range(1, len(ctx)))
+    record_parity(f"decode ragged paged batch (G={G})", max_rel_err=err)
     for b in range(1, len(ctx)):
         assert max_rel_err(out[b], refs[b]) < TOL, (b, max_rel_err(out[b], refs[b]))
     assert cache.status.item() == 0
@@ -282,7 +301,7 @@ def test_decode_serving_batch_sampled():
     n_pages = Bn * maxp
     perm = inputs.page_permutation(inputs.DATA_SEED, n_pages)
     table_np = perm.reshape(Bn, maxp)
-    P = B.iq_init_rotation(inputs.ROTATION_SEED, 1, Hkv)
+    P = oracle_params(inputs.ROTATION_SEED, 1, Hkv)
     cache = B.PagedCache(1, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
     g = torch.Generator(device=DEV).manual_seed(0)
     cache.k_codes.copy_(torch.randint(0, 256, cache.k_codes.shape, generator=g, device=DEV, dtype=torch.uint8))
@@ -300,6 +319,8 @@ def test_decode_serving_batch_sampled():
         refs[b] = attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[0])
     out = _decode(cache, 0, torch.from_numpy(q).to(DEV), ctx, int(ctx.max()), P)
     assert np.isfinite(out).all()
+    record_parity("decode serving shape, 3 of 16 seq (G=4)", max_rel_err=max(max_rel_err(out[b], refs[b])
+                                                                            for b in sampled))
     for b in sampled:
         assert max_rel_err(out[b], refs[b]) < TOL, (b, max_rel_err(out[b], refs[b]))
 
@@ -307,7 +328,7 @@ def test_decode_serving_batch_sampled():
 def test_encode_then_decode_end_to_end():
     """GPU encode followed by GPU decode vs the oracle's encode + attention of the same inputs."""
     Hq, Hkv, T = 16, 2, 3000
-    P = B.iq_init_rotation(2, 1, Hkv)
+    P = oracle_params(2, 1, Hkv)
     cache = B.PagedCache(1, Hkv, 3008, 1)
     X = {w: np.stack([inputs.kv_tokens(31, 0, h, w, 0, T) for h in range(Hkv)], axis=1)[None] for w in (0, 1)}
     B.iq_encode_append(cache, 0, torch.from_numpy(X[0]).to(DEV), torch.from_numpy(X[1]).to(DEV),
@@ -319,14 +340,16 @@ def test_encode_then_decode_end_to_end():
         q[0].astype(np.float64),
         np.stack([e["codes"] for e in enc[0]]), np.stack([e["norm16"] for e in enc[0]]),
         np.stack([e["codes"] for e in enc[1]]), np.stack([e["norm16"] for e in enc[1]]), P[0])
-    assert max_rel_err(out[0], ref) < TOL
+    err = max_rel_err(out[0], ref)
+    record_parity("GPU encode -> GPU decode vs oracle (3000 tok)", max_rel_err=err)
+    assert err < TOL
 
 
 def test_decode_flags_bad_context_and_pages():
     """ctx above max_ctx is clamped and flagged; a block-table entry outside the pool is skipped
     and flagged; the output stays finite."""
     Hkv, Hq = 1, 4
-    P = B.iq_init_rotation(1, 1, Hkv)
+    P = oracle_params(1, 1, Hkv)
     table = torch.tensor([[0, 1], [2, 999]], dtype=torch.int32, device=DEV)
     cache = B.PagedCache(1, Hkv, 64, 3, block_table=table)
     cache.pool.zero_()
@@ -345,7 +368,7 @@ def _step_case(G, ctx, ps, maxp, layer=0, L=1, seed=0, graph_layers=None):
     Hq = G * Hkv
     Bn = len(ctx)
     n_pages = Bn * maxp
-    P = B.iq_init_rotation(seed + 3, L, Hkv)
+    P = oracle_params(seed + 3, L, Hkv)
     perm = inputs.page_permutation(seed + 9, n_pages)
     table_np = perm.reshape(Bn, maxp)
     cache = B.PagedCache(L, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
@@ -368,28 +391,188 @@ def _step_case(G, ctx, ps, maxp, layer=0, L=1, seed=0, graph_layers=None):
     return cache, P, cases
 
 
+def _run_step(cache, layer, q, knew, vnew, ctx, max_ctx, P):
+    """iq_decode_step with guard bands around the output and the workspace; returns the output."""
+    Bn, Hq = q.shape[0], q.shape[1]
+    out = Guarded((Bn, Hq, 128), torch.float32, fill=float("nan"))
+    ws = Guarded((B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, max_ctx),), torch.uint8, fill=0)
+    B.iq_decode_step(cache, layer, torch.as_tensor(q).to(DEV), torch.as_tensor(knew).to(DEV),
+                     torch.as_tensor(vnew).to(DEV), torch.as_tensor(np.asarray(ctx, np.int32)).to(DEV), max_ctx,
+                     _params_dev(P), out.t, ws.t)
+    torch.cuda.synchronize()
+    out.check("out")
+    ws.check("workspace")
+    return out.t.cpu().numpy()
+
+
+def _check_appended(cache, layer, b, pos, knew_b, vnew_b, P_layer, rec):
+    """The records the step wrote at position pos of sequence b equal the oracle's encoding."""
+    for kv, x in ((0, knew_b), (1, vnew_b)):
+        codes, n16 = _export(cache, layer, kv, b, pos, 1)
+        for h in range(cache.n_kv_heads):
+            e = encode.encode(np.array([x[h]]), P_layer[h])
+            _check_codes(codes[h], n16[h], e, f"b={b} kv={kv} h={h}", cap=False, record=rec)
+
+
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_step_matches_oracle(G):
     """Fused append + attention: new tokens at odd and even positions, page boundaries, ctx = 1."""
     ctx = [1, 2, 64, 65, 129, 700]
     cache, P, cases = _step_case(G, ctx, ps=64, maxp=11)
     q, knew, vnew, refs = cases[0]
-    Bn, Hq = q.shape[0], q.shape[1]
-    out = torch.empty((Bn, Hq, 128), dtype=torch.float32, device=DEV)
-    ws = torch.zeros(B.iq_decode_workspace_size(Bn, Hq, cache.n_kv_heads, 704), dtype=torch.uint8, device=DEV)
-    B.iq_decode_step(cache, 0, torch.from_numpy(q).to(DEV), torch.from_numpy(knew).to(DEV), torch.from_numpy(vnew).to(DEV),
-                     torch.tensor(ctx, dtype=torch.int32, device=DEV), 704, _params_dev(P), out, ws)
-    torch.cuda.synchronize()
-    o = out.cpu().numpy()
+    o = _run_step(cache, 0, q, knew, vnew, ctx, 704, P)
+    rec = {"max_rel_err": 0.0}
     for b, T in enumerate(ctx):
-        ref, kc, kn, vc, vn = refs[b]
-        assert max_rel_err(o[b], ref) < TOL, (b, max_rel_err(o[b], ref))
-        for kv, (rc, rn) in enumerate([(kc, kn), (vc, vn)]):
-            codes, n16 = _export(cache, 0, kv, b, T - 1, 1)
-            for h in range(cache.n_kv_heads):
-                e = encode.encode(np.array([knew[b, h] if kv == 0 else vnew[b, h]]), P[0, h])
-                _check_codes(codes[h], n16[h], e, f"b={b} kv={kv}", cap=False)
+        ref = refs[b][0]
+        err = max_rel_err(o[b], ref)
+        rec["max_rel_err"] = max(rec["max_rel_err"], err)
+        assert err < TOL, (b, err)
+        _check_appended(cache, 0, b, T - 1, knew[b], vnew[b], P[0], rec)
     assert cache.status.item() == 0
+    record_parity(f"decode step, ragged paged (G={G})", **rec)
+
+
+def _oracle_fill_contiguous(cache, layer, P_layer, T_cached, seed, heads):
+    """Oracle encodings of tokens 0..T_cached-1 of each kv head uploaded to page 0 (a contiguous
+    cache); returns the codes and norms per head, for the oracle's attention."""
+    out = []
+    for h in heads:
+        ek = encode.encode(inputs.kv_tokens(seed, layer, h, 0, 0, T_cached), P_layer[h])
+        ev = encode.encode(inputs.kv_tokens(seed, layer, h, 1, 0, T_cached), P_layer[h])
+        upload_sequence(cache, layer, [0], h, ek["codes"], ek["norm16"], ev["codes"], ev["norm16"])
+        out.append((ek, ev))
+    return out
+
+
+def test_decode_step_headline_layer_full():
+    """The kernel the headline bench times, at the size and in the launch configuration it is
+    timed at: one layer of the Qwen3-30B-A3B-shaped step (batch 1, 32 q / 4 kv heads, group 8,
+    contiguous 32768-token cache, max_ctx 32768).  Tokens 0..32766 hold the oracle's encoding;
+    the step appends token 32767 from its fp16 inputs and attends over all 32768.  Every output
+    row and the appended records are compared with the oracle."""
+    Hq, Hkv, T, L, layer, seed = 32, 4, 32768, 2, 1, 0
+    P = oracle_params(inputs.ROTATION_SEED, L, Hkv)
+    cache = B.PagedCache(L, Hkv, T, 1)
+    enc = _oracle_fill_contiguous(cache, layer, P[layer], T - 1, seed, range(Hkv))
+    knew = np.stack([inputs.kv_tokens(seed, layer, h, 0, T - 1, 1)[0] for h in range(Hkv)])[None]
+    vnew = np.stack([inputs.kv_tokens(seed, layer, h, 1, T - 1, 1)[0] for h in range(Hkv)])[None]
+    q = inputs.queries(seed, layer, 1, Hq)
+    o = _run_step(cache, layer, q, knew, vnew, [T], T, P)
+    kc, kn, vc, vn = [], [], [], []
+    for h in range(Hkv):
+        ek_new = encode.encode(knew[0, h:h + 1], P[layer, h])
+        ev_new = encode.encode(vnew[0, h:h + 1], P[layer, h])
+        kc.append(np.concatenate([enc[h][0]["codes"], ek_new["codes"]]))
+        kn.append(np.concatenate([enc[h][0]["norm16"], ek_new["norm16"]]))
+        vc.append(np.concatenate([enc[h][1]["codes"], ev_new["codes"]]))
+        vn.append(np.concatenate([enc[h][1]["norm16"], ev_new["norm16"]]))
+    ref = attention.attention_rotated(q[0].astype(np.float64), np.stack(kc), np.stack(kn), np.stack(vc),
+                                      np.stack(vn), P[layer])
+    err = max_rel_err(o[0], ref)
+    rec = {"max_rel_err": err}
+    _check_appended(cache, layer, 0, T - 1, knew[0], vnew[0], P[layer], rec)
+    record_parity("decode step, headline 32K layer (G=8), bench launch", **rec)
+    assert err < TOL, err
+    assert cache.status.item() == 0
+
+
+def test_decode_step_serving_layer_sampled():
+    """The kernel the serving bench times, at its size and launch configuration: 16 sequences with
+    the seeded contexts in [2048, 32768], 64-token pages of a shuffled pool, 32 q / 8 kv heads
+    (group 4), max_ctx = the longest context.  Three sequences hold the oracle's encoding of tokens
+    0..ctx-2 (the others random records); the step appends every sequence's token ctx-1 and the
+    three sampled sequences are compared with the oracle in full."""
+    Bn, Hq, Hkv, ps = 16, 32, 8, 64
+    cfg = inputs.CONFIGS["serve_b16"]
+    ctx = inputs.context_lengths(inputs.DATA_SEED, Bn, cfg["ctx_lo"], cfg["ctx_hi"])
+    maxp = (int(ctx.max()) + ps - 1) // ps
+    n_pages = Bn * maxp
+    table_np = inputs.page_permutation(inputs.DATA_SEED, n_pages).reshape(Bn, maxp)
+    P = oracle_params(inputs.ROTATION_SEED, 1, Hkv)
+    cache = B.PagedCache(1, Hkv, ps, n_pages, block_table=torch.from_numpy(table_np).to(DEV))
+    g = torch.Generator(device=DEV).manual_seed(1)
+    cache.k_codes.copy_(torch.randint(0, 256, cache.k_codes.shape, generator=g, device=DEV, dtype=torch.uint8))
+    cache.v_codes.copy_(torch.randint(0, 256, cache.v_codes.shape, generator=g, device=DEV, dtype=torch.uint8))
+    norms = (torch.rand(cache.k_norms.shape, generator=g, device=DEV) * 40 + 1).half().view(torch.int16)
+    cache.k_norms.copy_(norms)
+    cache.v_norms.copy_(norms.flip(0))
+    sampled = [0, 7, 15]
+    knew = np.stack([np.stack([inputs.kv_tokens(60 + b, 0, h, 0, int(ctx[b]) - 1, 1)[0] for h in range(Hkv)])
+                     for b in range(Bn)])
+    vnew = np.stack([np.stack([inputs.kv_tokens(60 + b, 0, h, 1, int(ctx[b]) - 1, 1)[0] for h in range(Hkv)])
+                     for b in range(Bn)])
+    q = inputs.queries(inputs.DATA_SEED, 0, Bn, Hq)
+    refs = {}
+    for b in sampled:
+        T = int(ctx[b])
+        kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, T, seed=60 + b)  # token T-1 = the appended one
+        for h in range(Hkv):
+            upload_sequence(cache, 0, table_np[b], h, kc[h, :T - 1], kn[h, :T - 1], vc[h, :T - 1], vn[h, :T - 1])
+        refs[b] = attention.attention_rotated(q[b].astype(np.float64), kc, kn, vc, vn, P[0])
+    o = _run_step(cache, 0, q, knew, vnew, ctx, int(ctx.max()), P)
+    assert np.isfinite(o).all()
+    rec = {"max_rel_err": max(max_rel_err(o[b], refs[b]) for b in sampled)}
+    for b in sampled:
+        _check_appended(cache, 0, b, int(ctx[b]) - 1, knew[b], vnew[b], P[0], rec)
+    record_parity("decode step, serving 16 seq (G=4), 3 sampled, bench launch", **rec)
+    for b in sampled:
+        assert max_rel_err(o[b], refs[b]) < TOL, (b, max_rel_err(o[b], refs[b]))
+    assert cache.status.item() == 0
+
+
+# ------------------------------------------------------------------------- device error paths
+def _small_case():
+    Hkv, Hq, T = 1, 8, 200
+    P = oracle_params(1, 1, Hkv)
+    cache = B.PagedCache(1, Hkv, 256, 1)
+    kc, kn, vc, vn = _oracle_cache(P[0], 0, Hkv, T, seed=3)
+    upload_sequence(cache, 0, [0], 0, kc[0], kn[0], vc[0], vn[0])
+    q = torch.from_numpy(inputs.queries(3, 0, 1, Hq)).to(DEV)
+    return cache, P, q, T, (kc, kn, vc, vn)
+
+
+def test_decode_flags_workspace_counters_left_set():
+    """A workspace whose arrival counters were not zeroed: the merging CTAs see more arrivals than
+    partials and flag IQ_DEVERR_WORKSPACE (no wait is involved); a zeroed workspace then gives
+    the oracle's result again."""
+    cache, P, q, T, (kc, kn, vc, vn) = _small_case()
+    n = B.iq_decode_workspace_size(1, 8, 1, T)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
+    ws[:4].view(torch.int32).fill_(1000)  # group 0's arrival counter
+    out = torch.empty((1, 8, 128), dtype=torch.float32, device=DEV)
+    ctx = torch.tensor([T], dtype=torch.int32, device=DEV)
+    B.iq_decode_attention(cache, 0, q, ctx, T, _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    assert cache.status.item() & B.IQ_DEVERR_WORKSPACE
+    cache.status.zero_()
+    ws.zero_()
+    B.iq_decode_attention(cache, 0, q, ctx, T, _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    assert cache.status.item() == 0
+    ref = attention.attention_rotated(q.cpu().numpy()[0].astype(np.float64), kc, kn, vc, vn, P[0])
+    assert max_rel_err(out.cpu().numpy()[0], ref) < TOL
+
+
+def test_decode_bounded_wait_times_out_and_reports():
+    """The merge wait is bounded: counters preset so that the arrivals can never reach the number
+    of partials (a count nothing completes) make the merging CTAs give up after about a second,
+    flag IQ_DEVERR_TIMEOUT and finish; the context stays usable and the next call is correct."""
+    cache, P, q, T, (kc, kn, vc, vn) = _small_case()
+    n = B.iq_decode_workspace_size(1, 8, 1, T)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
+    ws[:4].view(torch.int32).fill_(-1000)  # arrivals start far below zero
+    out = torch.empty((1, 8, 128), dtype=torch.float32, device=DEV)
+    ctx = torch.tensor([T], dtype=torch.int32, device=DEV)
+    B.iq_decode_attention(cache, 0, q, ctx, T, _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    assert cache.status.item() & B.IQ_DEVERR_TIMEOUT
+    cache.status.zero_()
+    ws.zero_()
+    B.iq_decode_attention(cache, 0, q, ctx, T, _params_dev(P), out, ws)
+    torch.cuda.synchronize()
+    assert cache.status.item() == 0
+    ref = attention.attention_rotated(q.cpu().numpy()[0].astype(np.float64), kc, kn, vc, vn, P[0])
+    assert max_rel_err(out.cpu().numpy()[0], ref) < TOL
 
 
 def test_decode_step_chain_in_cuda_graph():
