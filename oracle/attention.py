@@ -18,6 +18,8 @@ They must agree to ~1e-10.
 
 GQA (q heads sharing a kv head): q head h reads kv head h // G, G = Hq / Hkv.
 An empty context (ctx = 0) yields a zero output vector (the pages are silent).
+K and V may use different codebook widths ([TQ-RQ] section "K 和 V 的非对称需求": keys need
+more bits than values) and any rotation variant of oracle.rotation.
 """
 
 import math
@@ -31,19 +33,21 @@ from .rotation import rotate, rotate_inverse
 D = 128
 
 
-def dequantise(codes, norm16, params_head, bits=3):
+def dequantise(codes, norm16, params_head, bits=3, variant="iso"):
     """Explicit fp64 vectors n * R^T c~[codes] for one kv head: (T, 128)."""
     ct, _ = codebook_for_dim(D, bits)
     n = fp16_bits_to_float(norm16)
-    return n[:, None] * rotate_inverse(ct[np.asarray(codes, dtype=np.int64)], params_head)
+    return n[:, None] * rotate_inverse(ct[np.asarray(codes, dtype=np.int64)], params_head, variant)
 
 
-def attention_dequant(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3):
+def attention_dequant(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3, v_bits=None, variant="iso"):
     """Plain softmax attention on the explicitly dequantised cache.
 
     q: (Hq, 128); k_codes/v_codes: (Hkv, T, 128); k_norm16/v_norm16: (Hkv, T);
-    params: (Hkv, 32, 2, 4).  Returns (Hq, 128) fp64.
+    params: (Hkv, ...) per-head rotation parameters.  bits: K codebook width; v_bits: V width
+    (default: bits).  Returns (Hq, 128) fp64.
     """
+    v_bits = bits if v_bits is None else v_bits
     q = np.asarray(q, dtype=np.float64)
     Hq = q.shape[0]
     Hkv, T = np.asarray(k_codes).shape[:2]
@@ -52,8 +56,8 @@ def attention_dequant(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3):
     if T == 0:
         return out
     for kv in range(Hkv):
-        Kh = dequantise(k_codes[kv], k_norm16[kv], params[kv], bits)
-        Vh = dequantise(v_codes[kv], v_norm16[kv], params[kv], bits)
+        Kh = dequantise(k_codes[kv], k_norm16[kv], params[kv], bits, variant)
+        Vh = dequantise(v_codes[kv], v_norm16[kv], params[kv], v_bits, variant)
         for h in range(kv * G, (kv + 1) * G):
             s = Kh @ q[h] / math.sqrt(D)
             p = np.exp(s - s.max())
@@ -61,25 +65,27 @@ def attention_dequant(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3):
     return out
 
 
-def attention_rotated(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3):
+def attention_rotated(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3, v_bits=None, variant="iso"):
     """The packed pipeline's order: same inputs and output as `attention_dequant`."""
+    v_bits = bits if v_bits is None else v_bits
     q = np.asarray(q, dtype=np.float64)
     Hq = q.shape[0]
     Hkv, T = np.asarray(k_codes).shape[:2]
     G = Hq // Hkv
-    ct, _ = codebook_for_dim(D, bits)
+    ct_k, _ = codebook_for_dim(D, bits)
+    ct_v, _ = codebook_for_dim(D, v_bits)
     out = np.zeros((Hq, D))
     if T == 0:
         return out
     for kv in range(Hkv):
         nk = fp16_bits_to_float(k_norm16[kv])
         nv = fp16_bits_to_float(v_norm16[kv])
-        Ck = ct[np.asarray(k_codes[kv], dtype=np.int64)]  # (T, 128) rotated-basis keys (unit scale)
-        Cv = ct[np.asarray(v_codes[kv], dtype=np.int64)]
+        Ck = ct_k[np.asarray(k_codes[kv], dtype=np.int64)]  # (T, 128) rotated-basis keys (unit scale)
+        Cv = ct_v[np.asarray(v_codes[kv], dtype=np.int64)]
         for h in range(kv * G, (kv + 1) * G):
-            q_r = rotate(q[h], params[kv])  # rotate the query once
+            q_r = rotate(q[h], params[kv], variant)  # rotate the query once
             s = nk * (Ck @ q_r) / math.sqrt(D)  # scores straight from codes and norms
             p = np.exp(s - s.max())
             acc = (p * nv) @ Cv  # accumulate values in the rotated basis
-            out[h] = rotate_inverse(acc / p.sum(), params[kv])  # one inverse rotation per output
+            out[h] = rotate_inverse(acc / p.sum(), params[kv], variant)  # one inverse rotation per output
     return out

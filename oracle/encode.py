@@ -43,11 +43,12 @@ def fp16_bits_to_float(bits):
     return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
 
 
-def encode(x16, params_head, bits=3):
+def encode(x16, params_head, bits=3, variant="iso"):
     """Encode fp16 vectors of one (layer, kv head).
 
     x16: (N, 128) float16 (or anything exactly representable in it).
-    params_head: (32, 2, 4) rotation parameters of that head.
+    params_head: rotation parameters of that head ((32, 2, 4) for "iso"; see oracle.rotation).
+    bits: 2, 3 or 4 (the 2**bits-level Lloyd–Max codebook).
     Returns dict with
       codes  (N, 128) uint8   -- ascending centroid index per rotated coordinate
       norm16 (N,) uint16      -- binary16 bits of ||x||
@@ -60,7 +61,7 @@ def encode(x16, params_head, bits=3):
     n = np.sqrt(np.sum(x * x, axis=-1))
     safe = np.where(n > 0.0, n, 1.0)
     x_hat = np.where((n > 0.0)[..., None], x / safe[..., None], 0.0)
-    z = rotate(x_hat, params_head)
+    z = rotate(x_hat, params_head, variant)
     u = math.sqrt(D) * z
     _, b = codebook(bits)
     codes = quantise(u, bits)

@@ -8,13 +8,18 @@ is 7 x 128 = 896 add/sub for the seven WHT butterfly stages plus 32 x 16 = 512 f
 the 4x4 block products (each block's 4x4 matrix formed once per head from its
 quaternion pair; the 1/sqrt(d) scale folded into it).
 
+The variants without the WHT ([TQ-RQ] section "三种变体"; "RotorQuant" sd114.wiki section
+"1. 绕过蝴蝶网络") are printed at 512 FMAs and 128 parameters (quaternion blocks of 4) and
+256 FMAs and 128 parameters (Givens blocks of 2); they are counted the same way, each block's
+matrix built from its parameters and applied with counted multiply / fused multiply-add.
+
 The counts are obtained by running the transforms on a counting scalar type, not by
 formula, so a dropped or duplicated stage changes them.
 """
 
 import numpy as np
 
-from .rotation import block_matrices
+from .rotation import D, block_matrices, rotate
 
 
 class Counter:
@@ -81,6 +86,28 @@ def count_blocks(params, y):
     return c, out
 
 
+def variant_blocks(params, variant):
+    """(first coordinate, matrix) of each block of a variant without the WHT; each matrix is
+    the block's action read off column by column on unit vectors."""
+    size = 4 if variant == "quat" else 2
+    R = rotate(np.eye(D), params, variant).T  # column c = image of unit vector c
+    return [(k, R[k:k + size, k:k + size]) for k in range(0, D, size)]
+
+
+def count_variant_blocks(params, variant, y):
+    c = Counter()
+    out = []
+    for k, m in variant_blocks(params, variant):
+        n = m.shape[0]
+        yb = [CNum(y[k + i], c) for i in range(n)]
+        for r in range(n):
+            acc = mul(m[r, 0], yb[0], c)
+            for col in range(1, n):
+                acc = fma(m[r, col], yb[col], acc, c)
+            out.append(acc.v)
+    return c, out
+
+
 def count_dense(d=128):
     """A dense d x d rotation applied to one vector, counted the same way."""
     c = Counter()
@@ -94,8 +121,13 @@ def count_dense(d=128):
     return c
 
 
-def rotation_op_counts(params, d=128):
-    """{'wht': add/sub count, 'so4': multiply-class count, 'total', 'dense', 'params'}."""
+def rotation_op_counts(params, d=128, variant="iso"):
+    """{'wht': add/sub count, 'so4': multiply-class count, 'total', 'dense', 'params'}
+    ('blocks' instead of 'so4' and no WHT for the quat / planar variants)."""
+    if variant != "iso":
+        cb, _ = count_variant_blocks(params, variant, [float(i) for i in range(d)])
+        n = cb.mul + cb.fma
+        return {"wht": 0, "blocks": n, "total": n, "params": int(np.asarray(params).size)}
     cw, y = count_wht(d)
     cb, _ = count_blocks(params, y)
     cd = count_dense(d)

@@ -23,6 +23,21 @@ Readings where the pages are silent (each listed in the design notes):
     (seed, layer, head, block, side) feeding Marsaglia's (1972) method for a
     uniform point on the 3-sphere; computed in fp64 and rounded to fp32.
     (Parity unpinned: the pages publish no parameter values.)
+
+Two block rotations without the WHT are the variants of the same idea ("压缩与速度的
+博弈" [TQ-RQ] section "三种变体": quaternion SO(4) blocks of 4 at 512 FMAs and 128
+parameters, Givens 2D blocks of 2 at 256 FMAs and 128 parameters; [RQ-wiki] section
+"1. 绕过蝴蝶网络": an independent 2D Givens or 4D quaternion rotation per pair or group of
+coordinates, no butterfly network, 128 rotation parameters):
+  * "quat":   block k maps y[4k..4k+3] to q_k * y_blk (left multiplication by one unit
+              quaternion, a left-isoclinic rotation); parameters [32][4] per head.
+  * "planar": pair i maps (y[2i], y[2i+1]) to (c y0 - s y1, s y0 + c y1), the Givens
+              rotation by the angle with cosine c and sine s; parameters [64][2] = (c, s)
+              per head, rescaled to unit length at use.
+The original structure is "iso" (WHT then quaternion pairs, [32][2][4] per head).
+Their parameters come from the same counter streams with the variant's index in the
+stream identifier; a Givens pair is a uniform point on the unit circle obtained by
+normalising a point drawn uniformly from the unit disc (rejection sampling).
 """
 
 import math
@@ -112,14 +127,65 @@ def so4_apply_inverse(z, params):
     return y.reshape(z.shape)
 
 
-def rotate(x, params):
-    """Forward rotation R x = S (H_hat x) along the last axis."""
-    return so4_apply(wht(x), params)
+VARIANTS = ("iso", "quat", "planar")
+PARAMS_PER_HEAD = {"iso": 256, "quat": 128, "planar": 128}
+PARAM_SHAPE = {"iso": (N_BLOCKS, 2, 4), "quat": (N_BLOCKS, 4), "planar": (D // 2, 2)}
 
 
-def rotate_inverse(z, params):
-    """Inverse rotation R^T z = H_hat (S^T z); H_hat is its own inverse."""
-    return wht(so4_apply_inverse(z, params))
+def quat_left_apply(y, params):
+    """Block k maps y[4k:4k+4] to q_k * y_blk (params (32, 4), each row rescaled to unit)."""
+    q = unit_params(params)
+    yb = np.asarray(y, dtype=np.float64).reshape(y.shape[:-1] + (N_BLOCKS, 4))
+    return quat_mul(np.broadcast_to(q, yb.shape), yb).reshape(y.shape)
+
+
+def quat_left_apply_inverse(z, params):
+    """The inverse: conj(q_k) * z_blk."""
+    q = unit_params(params)
+    zb = np.asarray(z, dtype=np.float64).reshape(z.shape[:-1] + (N_BLOCKS, 4))
+    return quat_mul(np.broadcast_to(quat_conj(q), zb.shape), zb).reshape(z.shape)
+
+
+def givens_apply(y, params):
+    """Pair i maps (y[2i], y[2i+1]) to (c y0 - s y1, s y0 + c y1) (params (64, 2) = (c, s))."""
+    p = unit_params(params)
+    yp = np.asarray(y, dtype=np.float64).reshape(y.shape[:-1] + (D // 2, 2))
+    c, s = p[:, 0], p[:, 1]
+    out = np.stack([c * yp[..., 0] - s * yp[..., 1], s * yp[..., 0] + c * yp[..., 1]], axis=-1)
+    return out.reshape(y.shape)
+
+
+def givens_apply_inverse(z, params):
+    """The transpose: (c z0 + s z1, -s z0 + c z1)."""
+    p = unit_params(params)
+    zp = np.asarray(z, dtype=np.float64).reshape(z.shape[:-1] + (D // 2, 2))
+    c, s = p[:, 0], p[:, 1]
+    out = np.stack([c * zp[..., 0] + s * zp[..., 1], -s * zp[..., 0] + c * zp[..., 1]], axis=-1)
+    return out.reshape(z.shape)
+
+
+def rotate(x, params, variant="iso"):
+    """Forward rotation along the last axis: iso R x = S (H_hat x); quat / planar: the block
+    rotation alone (no WHT)."""
+    if variant == "iso":
+        return so4_apply(wht(x), params)
+    if variant == "quat":
+        return quat_left_apply(np.asarray(x, dtype=np.float64), params)
+    if variant == "planar":
+        return givens_apply(np.asarray(x, dtype=np.float64), params)
+    raise ValueError(variant)
+
+
+def rotate_inverse(z, params, variant="iso"):
+    """Inverse rotation: iso R^T z = H_hat (S^T z) (H_hat is its own inverse); quat / planar:
+    the inverse block rotation."""
+    if variant == "iso":
+        return wht(so4_apply_inverse(z, params))
+    if variant == "quat":
+        return quat_left_apply_inverse(np.asarray(z, dtype=np.float64), params)
+    if variant == "planar":
+        return givens_apply_inverse(np.asarray(z, dtype=np.float64), params)
+    raise ValueError(variant)
 
 
 def block_matrices(params):
@@ -134,12 +200,15 @@ def block_matrices(params):
     return mats
 
 
-def rotation_matrix(params, d=D):
-    """Explicit d x d matrix R = S H_hat (for brute-force checks on tiny inputs)."""
-    S = np.zeros((d, d))
-    for k, m in enumerate(block_matrices(params)):
-        S[4 * k : 4 * k + 4, 4 * k : 4 * k + 4] = m
-    return S @ (hadamard_matrix(d) / math.sqrt(d))
+def rotation_matrix(params, d=D, variant="iso"):
+    """Explicit d x d matrix of the forward rotation, built column by column by applying it to
+    the unit vectors (for "iso" also assembled as S H_hat from the block matrices)."""
+    if variant == "iso":
+        S = np.zeros((d, d))
+        for k, m in enumerate(block_matrices(params)):
+            S[4 * k : 4 * k + 4, 4 * k : 4 * k + 4] = m
+        return S @ (hadamard_matrix(d) / math.sqrt(d))
+    return rotate(np.eye(d), params, variant).T
 
 
 # ------------------------------------------------------------------- seed -> params
@@ -151,9 +220,11 @@ def _mix64(z):
     return z ^ (z >> 31)
 
 
-def stream_id(layer, head, block, side):
-    """64-bit identifier of the parameter stream of one quaternion."""
-    return ((((layer * 65536) + head) * 64 + block) * 2 + side) & MASK64
+def stream_id(layer, head, block, side, variant=0):
+    """64-bit identifier of the parameter stream of one quaternion (or Givens pair); variant 0
+    ("iso") uses block 0..31 and side 0 (qL) / 1 (qR), 1 ("quat") block 0..31, 2 ("planar")
+    pair 0..63 as the block, both with side 0."""
+    return (((((variant * 65536 + layer) * 65536) + head) * 64 + block) * 2 + side) & MASK64
 
 
 class _Stream:
@@ -194,13 +265,38 @@ def random_unit_quaternion(seed, sid):
     return (x1, x2, x3 * t, x4 * t)
 
 
-def init_rotation(seed, n_layers, n_kv_heads):
-    """Rotation parameters [L][Hkv][32][2][4], fp32 (fp64 values rounded to nearest)."""
-    out = np.zeros((n_layers, n_kv_heads, N_BLOCKS, 2, 4), dtype=np.float32)
+def random_unit_circle(seed, sid):
+    """A uniform point (c, s) on the unit circle, in fp64: (x, y) uniform in the open unit disc
+    without the origin (rejection: 0 < r2 = x^2 + y^2 < 1), then (x / r, y / r), r = sqrt(r2)."""
+    st = _Stream(seed, sid)
+    while True:
+        x = 2.0 * st.uniform() - 1.0
+        y = 2.0 * st.uniform() - 1.0
+        r2 = x * x + y * y
+        if 0.0 < r2 < 1.0:
+            break
+    r = math.sqrt(r2)
+    return (x / r, y / r)
+
+
+def init_rotation(seed, n_layers, n_kv_heads, variant="iso"):
+    """Rotation parameters [L][Hkv][*PARAM_SHAPE[variant]], fp32 (fp64 values rounded to
+    nearest): iso [32][2][4] (qL, qR per block), quat [32][4], planar [64][2] (c, s)."""
+    out = np.zeros((n_layers, n_kv_heads) + PARAM_SHAPE[variant], dtype=np.float32)
+    vi = VARIANTS.index(variant)
     for l in range(n_layers):
         for h in range(n_kv_heads):
-            for k in range(N_BLOCKS):
-                for side in range(2):
-                    q = random_unit_quaternion(seed, stream_id(l, h, k, side))
-                    out[l, h, k, side, :] = np.array(q, dtype=np.float64).astype(np.float32)
+            if variant == "iso":
+                for k in range(N_BLOCKS):
+                    for side in range(2):
+                        q = random_unit_quaternion(seed, stream_id(l, h, k, side))
+                        out[l, h, k, side, :] = np.array(q, dtype=np.float64).astype(np.float32)
+            elif variant == "quat":
+                for k in range(N_BLOCKS):
+                    q = random_unit_quaternion(seed, stream_id(l, h, k, 0, vi))
+                    out[l, h, k, :] = np.array(q, dtype=np.float64).astype(np.float32)
+            else:
+                for i in range(D // 2):
+                    out[l, h, i, :] = np.array(random_unit_circle(seed, stream_id(l, h, i, 0, vi)),
+                                               dtype=np.float64).astype(np.float32)
     return out

@@ -372,3 +372,222 @@ def test_planted_mistakes_are_caught():
     Pbad[..., 0, :], Pbad[..., 1, :] = P[..., 1, :], P[..., 0, :]
     x = np.random.default_rng(6).standard_normal(128)
     assert np.abs(rotation.rotate(x, Pbad[0]) - rotation.rotate(x, P[0])).max() > 1e-3
+
+
+# ------------------------------------------------------------------ other bit widths
+@pytest.mark.parametrize("bits,tag", [(2, "n4"), (4, "n16")])
+def test_lloyd_max_2_and_4_bit_match_textbook_table(bits, tag):
+    g = _golden("lloyd_max_gaussian_2bit_4bit.txt")
+    c, b = codebook.codebook(bits)
+    n = 1 << bits
+
+    def slack(v):
+        return 0.6 * 10.0 ** -(len(v.split(".")[1]) if "." in v else 0)
+
+    for got, printed in [(c[n // 2:], g[f"{tag}_output_levels"]), (-c[:n // 2][::-1], g[f"{tag}_output_levels"]),
+                         (b[n // 2 - 1:], g[f"{tag}_decision_levels"])]:
+        assert len(got) == len(printed)
+        for x, v in zip(got, printed):
+            assert abs(x - float(v)) <= slack(v) + 1e-12, (x, v)
+    mse = codebook.gaussian_mse(c, b)
+    tol = 1e-5 if bits == 4 else slack(g[f"{tag}_mse"][0])
+    assert abs(mse - float(g[f"{tag}_mse"][0])) <= tol, mse
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_lloyd_max_2_and_4_bit_are_minima_of_mse(bits):
+    """An independent optimiser (Nelder-Mead on the MSE functional) finds the same levels, and
+    a Monte Carlo estimate of the error agrees with the closed form."""
+    c, b = codebook.codebook(bits)
+    n = 1 << bits
+
+    def mse(pos):
+        levels = np.sort(np.concatenate([-pos[::-1], pos]))
+        return codebook.gaussian_mse(levels, 0.5 * (levels[1:] + levels[:-1]))
+
+    x0 = np.linspace(0.2, 2.5, n // 2)
+    res = scipy.optimize.minimize(mse, x0=x0, method="Nelder-Mead",
+                                  options={"xatol": 1e-11, "fatol": 1e-15, "maxiter": 200000, "maxfev": 200000})
+    np.testing.assert_allclose(np.sort(res.x), c[n // 2:], atol=2e-5)
+    x = np.random.default_rng(8).standard_normal(2_000_000)
+    q = c[np.searchsorted(b, x, side="left")]
+    assert abs(np.mean((x - q) ** 2) - codebook.gaussian_mse(c, b)) < 3e-4
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_chunk_golden_fixtures_other_widths(bits):
+    g = _golden("packing_chunks.txt")
+    if bits == 4:
+        y = [s % 16 for s in range(32)]
+        assert packing.pack_chunk(y, 4).hex() == g["chunk4_mod16"][0]
+        assert packing.unpack_chunk(bytes.fromhex(g["chunk4_mod16"][0]), 4) == y
+    else:
+        y = [s % 4 for s in range(32)]
+        assert packing.pack_chunk(y, 2).hex() == g["chunk2_mod4"][0]
+        assert packing.unpack_chunk(bytes.fromhex(g["chunk2_mod4"][0]), 2) == y
+        y = [3 if 8 <= s < 16 else 0 for s in range(32)]
+        assert packing.pack_chunk(y, 2).hex() == g["chunk2_slots8to15_are_3"][0]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pack_round_trip_and_ownership_all_widths(bits):
+    rng = np.random.default_rng(13)
+    top = (1 << bits) - 1
+    codes = rng.integers(0, top + 1, (37, 128)).astype(np.uint8)
+    np.testing.assert_array_equal(packing.unpack_k(packing.pack_k(codes, bits), bits), codes)
+    np.testing.assert_array_equal(packing.unpack_v(packing.pack_v(codes, bits), 37, bits), codes)
+    np.testing.assert_array_equal(packing.pack_k_fast(codes, bits), packing.pack_k(codes, bits))
+    np.testing.assert_array_equal(packing.pack_v_fast(codes, bits), packing.pack_v(codes, bits))
+    np.testing.assert_array_equal(packing.unpack_v_fast(packing.pack_v(codes, bits), 37, bits), codes)
+    np.testing.assert_array_equal(packing.unpack_k_fast(packing.pack_k(codes, bits), bits), codes)
+    own = packing.v_bit_owner(bits)
+    assert np.all(np.bincount(own, minlength=16) == 128 * bits)
+    base = rng.integers(0, top + 1, (16, 128)).astype(np.uint8)
+    bits0 = np.unpackbits(packing.pack_v(base, bits)[0], bitorder="little")
+    cbits = 32 * bits  # bits per chunk
+    for u in (0, 6, 9, 15):
+        alt = base.copy()
+        alt[u] = top - alt[u]  # flips every code bit of token u
+        bits1 = np.unpackbits(packing.pack_v(alt, bits)[0], bitorder="little")
+        np.testing.assert_array_equal(np.nonzero(bits0 != bits1)[0], np.nonzero(own == u)[0])
+        # in every width token u owns nibbles j and j+4 of every word of its 16 chunks
+        j, tq = 2 * (u // 8) + (u % 2), (u % 8) // 2
+        pos = np.nonzero(own == u)[0]
+        assert set(((pos // cbits) // 2 % 4).tolist()) == {tq}
+        assert set(((pos % 32) // 4).tolist()) == {j, j + 4}
+
+
+# ------------------------------------------------------------------ rotation variants
+def test_variant_params_shapes_units_and_streams():
+    for v in ("quat", "planar"):
+        P = rotation.init_rotation(1, 2, 3, v)
+        assert P.shape == (2, 3) + rotation.PARAM_SHAPE[v] and P.dtype == np.float32
+        assert P[0, 0].size == rotation.PARAMS_PER_HEAD[v] == 128
+        n = np.linalg.norm(P.astype(np.float64), axis=-1)
+        assert np.abs(n - 1).max() < 3e-7
+        np.testing.assert_array_equal(P, rotation.init_rotation(1, 2, 3, v))
+    # Givens angles are uniform on the circle: mean of (c, s) ~ 0, E[c^2] = 1/2
+    G = rotation.init_rotation(5, 8, 8, "planar").reshape(-1, 2).astype(np.float64)
+    assert np.abs(G.mean(0)).max() < 0.03 and abs((G[:, 0] ** 2).mean() - 0.5) < 0.02
+    # the variants' streams differ from the iso streams
+    Q = rotation.init_rotation(1, 1, 1, "quat")[0, 0]
+    I = rotation.init_rotation(1, 1, 1, "iso")[0, 0]
+    assert not np.array_equal(Q, I[:, 0])
+
+
+def test_planar_blocks_are_givens_rotations():
+    """Each 2x2 block equals the matrix exponential of the skew generator of its angle
+    (scipy.linalg.expm), an independent construction of the Givens rotation."""
+    P = rotation.init_rotation(3, 1, 1, "planar")[0, 0].astype(np.float64)
+    R = rotation.rotation_matrix(P, variant="planar")
+    for i in range(64):
+        c, s = P[i] / np.linalg.norm(P[i])
+        th = math.atan2(s, c)
+        ref = scipy.linalg.expm(np.array([[0.0, -th], [th, 0.0]]))
+        np.testing.assert_allclose(R[2 * i:2 * i + 2, 2 * i:2 * i + 2], ref, atol=1e-14)
+    off = R.copy()
+    for i in range(64):
+        off[2 * i:2 * i + 2, 2 * i:2 * i + 2] = 0
+    assert np.all(off == 0)
+
+
+def test_quat_blocks_are_left_isoclinic():
+    """Each 4x4 block is left multiplication by its unit quaternion (the explicit matrix of
+    Hamilton's product), lies in SO(4), and commutes with every right multiplication."""
+    P = rotation.init_rotation(4, 1, 1, "quat")[0, 0].astype(np.float64)
+    R = rotation.rotation_matrix(P, variant="quat")
+
+    def Lmat(q):
+        w, x, y, z = q
+        return np.array([[w, -x, -y, -z], [x, w, -z, y], [y, z, w, -x], [z, -y, x, w]])
+
+    def Rmat(q):
+        w, x, y, z = q
+        return np.array([[w, -x, -y, -z], [x, w, z, -y], [y, -z, w, x], [z, y, -x, w]])
+
+    rng = np.random.default_rng(9)
+    for k in range(32):
+        q = P[k] / np.linalg.norm(P[k])
+        m = R[4 * k:4 * k + 4, 4 * k:4 * k + 4]
+        np.testing.assert_allclose(m, Lmat(q), atol=1e-14)
+        assert abs(np.linalg.det(m) - 1) < 1e-13
+        p = rng.standard_normal(4)
+        np.testing.assert_allclose(m @ Rmat(p), Rmat(p) @ m, atol=1e-13)
+
+
+@pytest.mark.parametrize("variant", ["quat", "planar"])
+def test_variant_round_trip_orthogonal(variant):
+    P = rotation.init_rotation(2, 1, 1, variant)[0, 0]
+    R = rotation.rotation_matrix(P, variant=variant)
+    np.testing.assert_allclose(R @ R.T, np.eye(128), atol=1e-13)
+    assert abs(np.linalg.det(R) - 1) < 1e-10
+    x = np.random.default_rng(5).standard_normal((7, 128))
+    assert np.abs(rotation.rotate_inverse(rotation.rotate(x, P, variant), P, variant) - x).max() <= 1e-12
+    np.testing.assert_allclose(rotation.rotate_inverse(x, P, variant), x @ R, atol=1e-13)
+
+
+def test_variant_op_counts_match_the_printed_figures():
+    g = _golden("rotation_op_counts.txt")
+    q = opcount.rotation_op_counts(rotation.init_rotation(1, 1, 1, "quat")[0, 0], variant="quat")
+    p = opcount.rotation_op_counts(rotation.init_rotation(1, 1, 1, "planar")[0, 0], variant="planar")
+    assert q["total"] == int(g["quat_fma"][0]) and q["wht"] == 0
+    assert p["total"] == int(g["planar_fma"][0]) and p["wht"] == 0
+    assert q["params"] == p["params"] == int(g["variant_params"][0])
+
+
+@pytest.mark.parametrize("variant,bits", [("iso", 2), ("iso", 4), ("quat", 3), ("planar", 3), ("planar", 4)])
+def test_encode_constructed_centroid_vectors_all_forms(variant, bits):
+    """x = n R^T c~[k*] (rounded to fp16) encodes to k* for every width and rotation (k* drawn
+    with the cell probabilities so that the unit-length rescaling keeps each level in its cell)."""
+    P = rotation.init_rotation(1, 1, 1, variant)[0, 0]
+    c, b = codebook.codebook(bits)
+    ct, _ = codebook.codebook_for_dim(128, bits)
+    e_ = np.concatenate([[-np.inf], b, [np.inf]])
+    mass = scipy.stats.norm.cdf(e_[1:]) - scipy.stats.norm.cdf(e_[:-1])
+    rng = np.random.default_rng(17)
+    done = 0
+    while done < 10:
+        kstar = rng.choice(1 << bits, size=128, p=mass / mass.sum())
+        u = math.sqrt(128) / np.linalg.norm(c[kstar]) * c[kstar]
+        if np.any(encode.quantise(u, bits) != kstar):  # rescaling crossed a boundary: draw again
+            continue
+        n = rng.uniform(0.5, 300.0)
+        x = (n * rotation.rotate_inverse(ct[kstar], P, variant)).astype(np.float16)
+        e = encode.encode(x[None], P, bits, variant)
+        ok = e["codes"][0] == kstar
+        assert np.all(ok | e["near"][0]), np.nonzero(~ok)
+        done += 1
+
+
+@pytest.mark.parametrize("variant,kb,vb", [("iso", 4, 2), ("iso", 4, 3), ("quat", 3, 3), ("planar", 3, 2)])
+def test_rotated_equals_dequantised_attention_all_forms(variant, kb, vb):
+    rng = np.random.default_rng(21)
+    Hkv, T = 2, 29
+    P = rotation.init_rotation(1, 1, Hkv, variant)[0]
+    kc = rng.integers(0, 1 << kb, (Hkv, T, 128)).astype(np.uint8)
+    vc = rng.integers(0, 1 << vb, (Hkv, T, 128)).astype(np.uint8)
+    kn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 60, (Hkv, T)))
+    vn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 10, (Hkv, T)))
+    q = rng.standard_normal((6, 128))
+    a = attention.attention_rotated(q, kc, kn, vc, vn, P, kb, vb, variant)
+    b = attention.attention_dequant(q, kc, kn, vc, vn, P, kb, vb, variant)
+    assert np.abs(a - b).max() / np.abs(b).max() < 1e-10
+    for kv in range(Hkv):  # and the dequantised form is plain softmax attention (torch SDPA, fp64)
+        K = torch.from_numpy(attention.dequantise(kc[kv], kn[kv], P[kv], kb, variant))
+        V = torch.from_numpy(attention.dequantise(vc[kv], vn[kv], P[kv], vb, variant))
+        Q = torch.from_numpy(q[3 * kv:3 * kv + 3])
+        ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None])[0]
+        np.testing.assert_allclose(b[3 * kv:3 * kv + 3], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_planted_variant_mistakes_are_caught():
+    """A Givens pair applied with the sign of its sine flipped, or a quaternion applied on the
+    right instead of the left, is a different rotation: the explicit-matrix pins would fail."""
+    x = np.random.default_rng(6).standard_normal(128)
+    Pp = rotation.init_rotation(1, 1, 1, "planar")[0, 0].astype(np.float64)
+    flipped = Pp * np.array([1.0, -1.0])
+    assert np.abs(rotation.rotate(x, flipped, "planar") - rotation.rotate(x, Pp, "planar")).max() > 1e-3
+    Pq = rotation.init_rotation(1, 1, 1, "quat")[0, 0].astype(np.float64)
+    q = rotation.unit_params(Pq)
+    right = rotation.quat_mul(x.reshape(32, 4), q).reshape(128)
+    assert np.abs(right - rotation.rotate(x, Pq, "quat")).max() > 1e-3
