@@ -1,5 +1,5 @@
 /*
- * iq.h -- C ABI of the IsoQuant packed-3-bit KV cache library (libiq.so, sm_100a).
+ * iq.h -- C ABI of the IsoQuant packed KV cache library (libiq.so, sm_100a).
  *
  * What the library computes (sources are web pages, cited by title and section):
  *   - "RotaryQuant" write-up, rebasdaily.com 2026-08-14, section
@@ -13,7 +13,10 @@
  *     "Beta 分布的魔力" (rotated unit-vector coordinates ~ N(0, 1/d)) and
  *     "Lloyd-Max 最优量化" (the optimal scalar quantiser, applied by lookup).
  *   - "RotorQuant：LLM KV 缓存压缩的“几何革命”" (sd114.wiki), section
- *     "3. V 缓存的逆旋转修复": values must be rotated back with the inverse rotation.
+ *     "3. V 缓存的逆旋转修复": values must be rotated back with the inverse rotation;
+ *     section "1. 绕过蝴蝶网络" and "压缩与速度的博弈" section "三种变体": the block rotations
+ *     without the WHT (one quaternion per group of 4, or a Givens rotation per pair);
+ *     "压缩与速度的博弈" section "K 和 V 的非对称需求": more bits for K than for V.
  *
  * Conventions for every entry point:
  *   - Pointers named *_dev / all tensors are DEVICE memory owned by the caller; the
@@ -30,34 +33,46 @@
  *   - No C++ exception crosses this interface.
  *   - head_dim is 128; every device pointer must be 16-byte aligned (workspace 256).
  *
- * Cache layout: one pool, [L][n_pages][Hkv][page_size/32] tile records of 3200 bytes; the
- *   tile record of 32 consecutive slots s0..s0+31 (s0 a multiple of 32) holds
- *       bytes [0, 1536)     the 32 K records, slot order (48 bytes each)
- *       bytes [1536, 3072)  the two V blocks of slots s0..s0+15 and s0+16..s0+31
- *       bytes [3072, 3136)  the 32 K norms (binary16), bytes [3136, 3200) the 32 V norms
- *   (100 bytes per token and kv head; one tile record is one bulk copy for the decoder).
+ * Code widths: K codes of kb bits and V codes of vb bits per coordinate, (kb, vb) one of
+ *   (2,2), (3,2), (3,3), (4,2), (4,3), (4,4) (K never narrower than V); 3 bits by default.
+ * Cache layout: one pool, [L][n_pages][Hkv][page_size/32] tile records of
+ *   TB = 512 kb + 512 vb + 128 bytes (3200 for 3/3); the tile record of 32 consecutive slots
+ *   s0..s0+31 (s0 a multiple of 32) holds
+ *       bytes [0, 512 kb)                 the 32 K records, slot order (16 kb bytes each)
+ *       bytes [512 kb, 512 (kb + vb))     the two V blocks of slots s0..s0+15 and s0+16..s0+31
+ *       next 64 bytes                     the 32 K norms (binary16), then the 32 V norms
+ *   (16 (kb + vb) + 4 bytes per token and kv head; 100 for 3/3; one tile record is one bulk copy
+ *   for the decoder).
  *   Token t of sequence b lives on page
  *       block_table_dev[b * max_pages_per_seq + t / page_size]   (paged), or
  *       b                                                         (block_table_dev == NULL)
  *   at slot t % page_size.  page_size is a positive multiple of 32.
  *
  * Record formats (this library's own; the pages fix none):
- *   code k in 0..7 = index of the ascending Lloyd-Max centroid of N(0,1):
- *       k = #{ j : u > b_j },  u = sqrt(128) * (R x / ||x||),  R = S * H/sqrt(128)
- *   32-code chunk = 12 bytes = little-endian uint32 W0,W1,W2; for j in 0..7:
- *       bits [4j,4j+3) of Ww = code of slot 8w+j; bit 4j+3 of Ww = bit w of slot 24+j
+ *   code k in 0..2^bits-1 = index of the ascending Lloyd-Max centroid of N(0,1):
+ *       k = #{ j : u > b_j },  u = sqrt(128) * (R x / ||x||)
+ *   32-code chunk = 4*bits bytes = little-endian uint32 words W0..W(bits-1); for j in 0..7:
+ *       3 bits: bits [4j,4j+3) of Ww = code of slot 8w+j; bit 4j+3 of Ww = bit w of slot 24+j
+ *       4 bits: bits [4j,4j+4) of Ww = code of slot 8w+j
+ *       2 bits: bits [4j,4j+2) of Ww = code of slot 16w+j; bits [4j+2,4j+4) = slot 16w+8+j
  *   K record (per token): chunk c = 0..3, slot s -> coordinate 32c+s.
  *   V block (positions 16b..16b+15 of one sequence and kv head): 64 chunks, chunk
- *       (g, tq, h) (g 0..7, tq 0..3, h 0..1) at byte 12*(2*(4g+tq)+h); its slot
+ *       (g, tq, h) (g 0..7, tq 0..3, h 0..1) at byte 4*bits*(2*(4g+tq)+h); its slot
  *       8*(m/2) + 4*(m%2) + j (m 0..7, j 0..3) holds token 8*(j/2) + 2*tq + (j%2) of the block
- *       at coordinate 16m + g + 8h.  Token u owns nibbles j, j+4 (spare bit included) of the
- *       words of the 16 chunks with tq = (u%8)/2, j = 2*(u/8) + u%2, and nothing else.
+ *       at coordinate 16m + g + 8h.  Token u owns nibbles j, j+4 of the words of the 16 chunks
+ *       with tq = (u%8)/2, j = 2*(u/8) + u%2, and nothing else (in every width).
  *   Norm: ||x||_2 of the fp16 input, rounded to binary16 (nearest even), saturating
  *       at 65504.
  *
- * Rotation parameters: float32 [L][Hkv][32][2][4] = per 4-coordinate block k the unit
- *   quaternions (qL, qR), each (w,x,y,z); block k maps y[4k..4k+3] (read as a
- *   quaternion) to qL * y * conj(qR).  R x = S(H x / sqrt(128)), H Sylvester-ordered.
+ * Rotation R (iq_cache.rotation), parameters float32 [L][Hkv][P] (P per head):
+ *   IQ_ROT_ISO (P = 256): [32][2][4] = per 4-coordinate block k the unit quaternions (qL, qR),
+ *       each (w,x,y,z); R x = S(H x / sqrt(128)), H Sylvester-ordered, block k of S maps
+ *       y[4k..4k+3] (read as a quaternion) to qL * y * conj(qR).
+ *   IQ_ROT_QUAT (P = 128): [32][4] = one unit quaternion q per block; block k maps
+ *       x[4k..4k+3] to q * x (no WHT).
+ *   IQ_ROT_PLANAR (P = 128): [64][2] = (c, s) per coordinate pair i; (x[2i], x[2i+1]) ->
+ *       (c x0 - s x1, s x0 + c x1) (no WHT).
+ *   Every stored quaternion and (c, s) pair is rescaled to unit length at use.
  */
 #ifndef IQ_H
 #define IQ_H
@@ -74,7 +89,8 @@ typedef struct CUstream_st* iq_stream_t; /* same type as cudaStream_t */
 typedef enum {
   IQ_OK = 0,
   IQ_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, inconsistent shapes */
-  IQ_ERR_UNSUPPORTED = 2, /* head_dim != 128, GQA group size not 1, 2, 4 or 8, bad dtype */
+  IQ_ERR_UNSUPPORTED = 2, /* head_dim != 128, GQA group size not 1, 2, 4 or 8, bad dtype, code widths
+                             or rotation variant not supported */
   IQ_ERR_CAPACITY = 3,    /* a host-known size exceeds the cache's capacity */
   IQ_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than iq_decode_workspace_size */
   IQ_ERR_ALIGNMENT = 5,   /* a device pointer is not 16-byte aligned (workspace: 256) */
@@ -82,6 +98,8 @@ typedef enum {
 } iq_status;
 
 typedef enum { IQ_F16 = 0, IQ_F32 = 1 } iq_dtype;
+
+typedef enum { IQ_ROT_ISO = 0, IQ_ROT_QUAT = 1, IQ_ROT_PLANAR = 2 } iq_rotation;
 
 /* Bits OR-ed into *status_dev by kernels that meet bad data (see conventions). */
 #define IQ_DEVERR_POSITION 1u /* token position outside its sequence's pages */
@@ -100,6 +118,9 @@ typedef struct {
   const int32_t* block_table_dev;  /* [batch][max_pages_per_seq] or NULL */
   int32_t max_pages_per_seq;       /* ignored when block_table_dev is NULL */
   uint32_t* status_dev;            /* device word for IQ_DEVERR_* bits, or NULL */
+  int32_t k_bits;                  /* K code width: 2, 3 or 4 (0 = 3) */
+  int32_t v_bits;                  /* V code width: 2, 3 or 4 (0 = 3); (k_bits, v_bits) as listed above */
+  int32_t rotation;                /* iq_rotation */
 } iq_cache;
 
 /* Library version string (static storage). */
@@ -108,10 +129,11 @@ const char* iq_version(void);
 /* Human-readable text of a status code (static storage; never NULL). */
 const char* iq_status_string(iq_status s);
 
-/* Bytes of the cache pool for the given geometry (100 per token slot and kv head).
- * Host-only; returns IQ_ERR_INVALID_ARG on bad sizes (page_size not a positive multiple of 32). */
-iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
-                         size_t* pool_bytes_host);
+/* Bytes of the cache pool for the given geometry and code widths (0 = 3 bits; 100 bytes per
+ * token slot and kv head for 3/3).  Host-only; returns IQ_ERR_INVALID_ARG on bad sizes (page_size
+ * not a positive multiple of 32), IQ_ERR_UNSUPPORTED for a width pair not listed above. */
+iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages, int32_t k_bits,
+                         int32_t v_bits, size_t* pool_bytes_host);
 
 /* Rotation parameters from a seed (host-only; writes n_layers*n_kv_heads*256 floats to
  * params_host).  Defined by: RotaryQuant abstract (arXiv 2608.08081), 256 parameters per head
@@ -122,6 +144,20 @@ iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size
  * Errors: IQ_ERR_INVALID_ARG for NULL params_host or non-positive sizes. */
 iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, float* params_host);
 
+/* Parameters per head of a rotation variant (256, 128, 128), 0 for an unknown value. */
+int32_t iq_rotation_params_per_head(int32_t rotation);
+
+/* Rotation parameters of any variant (host-only; writes n_layers*n_kv_heads*P floats).
+ * IQ_ROT_ISO gives the same values as iq_init_rotation; IQ_ROT_QUAT draws one quaternion per
+ * block from the unit 3-sphere, IQ_ROT_PLANAR one (c, s) pair per coordinate pair from the unit
+ * circle (a disc point by rejection, normalised), each from its own splitmix64 stream.
+ * Defined by: "压缩与速度的博弈" (zhichai.net), section "三种变体" (128 parameters for the
+ * quaternion and the Givens variants); "RotorQuant" (sd114.wiki), section "1. 绕过蝴蝶网络".
+ * Errors: IQ_ERR_INVALID_ARG for NULL params_host or non-positive sizes, IQ_ERR_UNSUPPORTED for
+ * an unknown variant. */
+iq_status iq_init_rotation_variant(uint64_t seed, int32_t rotation, int32_t n_layers, int32_t n_kv_heads,
+                                   float* params_host);
+
 /* Quantise-and-append: encode n_new new tokens of every sequence into layer `layer`.
  * Defined by: "RotaryQuant" (rebasdaily.com), section "妙处不只是压缩，而是不再展开" (rotate,
  * then scalar-quantise each coordinate to 3 bits and pack); "压缩与速度的博弈" (zhichai.net),
@@ -129,9 +165,10 @@ iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, 
  * (the quantiser).
  *   k_dev, v_dev : fp16 [batch][n_new][Hkv][128]; either may be NULL (that side skipped).
  *   start_pos_dev: int32 [batch], position of each sequence's first new token.
- *   params_dev   : float32 [L][Hkv][32][2][4].
- * Per vector: norm (fp32 accumulate) -> WHT -> SO(4) blocks -> threshold search against
- * the 7 Lloyd-Max boundaries -> packed record + binary16 norm written at its slot.
+ *   params_dev   : float32 [L][Hkv][P] of the cache's rotation variant.
+ * Per vector: norm (fp32 accumulate) -> rotation (WHT + SO(4) blocks, or the variant's blocks)
+ * -> threshold search against the 2^bits - 1 Lloyd-Max boundaries -> packed record + binary16
+ * norm written at its slot.
  * Writes only the bits of the tokens it encodes (the other tokens of a V block keep theirs;
  * tokens of one block may come from different calls, but calls that overlap on the GPU must
  * not append to the same block).  Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA; IQ_DEVERR_POSITION /
@@ -160,7 +197,7 @@ size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
  *                  into range and flagged with IQ_DEVERR_CTX.
  *   max_ctx      : host upper bound on ctx_len (sizes the split-K grid); must not exceed
  *                  the per-sequence capacity (page_size, or page_size*max_pages_per_seq).
- *   params_dev   : float32 [L][Hkv][32][2][4], the parameters used when encoding.
+ *   params_dev   : float32 [L][Hkv][P], the parameters used when encoding.
  *   out_dev      : float32 [batch][n_q_heads][128].
  *   workspace_dev: at least iq_decode_workspace_size(...) bytes, 256-byte aligned,
  *                  zero-filled before its first use (see iq_decode_workspace_size); calls

@@ -27,13 +27,33 @@ IQ_DEVERR_PAGE = 2
 IQ_DEVERR_CTX = 4
 IQ_DEVERR_TIMEOUT = 8
 IQ_DEVERR_WORKSPACE = 16
+IQ_ROT_ISO = 0
+IQ_ROT_QUAT = 1
+IQ_ROT_PLANAR = 2
+ROTATIONS = {"iso": IQ_ROT_ISO, "quat": IQ_ROT_QUAT, "planar": IQ_ROT_PLANAR}
+WIDTHS = ((2, 2), (3, 2), (3, 3), (4, 2), (4, 3), (4, 4))  # supported (K bits, V bits)
 
 HEAD_DIM = 128
-K_RECORD_BYTES = 48
 V_BLOCK_TOKENS = 16
-V_BLOCK_BYTES = 768
 TILE_TOKENS = 32
-TILE_BYTES = 3200  # 32 K records | 2 V blocks | 32 K norms | 32 V norms
+
+
+def k_record_bytes(bits=3):
+    return 16 * bits
+
+
+def v_block_bytes(bits=3):
+    return 256 * bits
+
+
+def tile_bytes(k_bits=3, v_bits=3):
+    """32 K records | 2 V blocks | 32 K norms | 32 V norms (3200 bytes for 3/3)."""
+    return 32 * k_record_bytes(k_bits) + 2 * v_block_bytes(v_bits) + 128
+
+
+K_RECORD_BYTES = k_record_bytes(3)
+V_BLOCK_BYTES = v_block_bytes(3)
+TILE_BYTES = tile_bytes(3, 3)
 
 
 class IqError(RuntimeError):
@@ -53,6 +73,9 @@ class iq_cache(ctypes.Structure):
         ("block_table_dev", ctypes.c_void_p),
         ("max_pages_per_seq", ctypes.c_int32),
         ("status_dev", ctypes.c_void_p),
+        ("k_bits", ctypes.c_int32),
+        ("v_bits", ctypes.c_int32),
+        ("rotation", ctypes.c_int32),
     ]
 
 
@@ -73,9 +96,13 @@ def lib():
         L.iq_status_string.restype = ctypes.c_char_p
         L.iq_status_string.argtypes = [ctypes.c_int]
         L.iq_cache_bytes.restype = ctypes.c_int
-        L.iq_cache_bytes.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz)]
+        L.iq_cache_bytes.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]
         L.iq_init_rotation.restype = ctypes.c_int
         L.iq_init_rotation.argtypes = [ctypes.c_uint64, i32, i32, vp]
+        L.iq_init_rotation_variant.restype = ctypes.c_int
+        L.iq_init_rotation_variant.argtypes = [ctypes.c_uint64, i32, i32, i32, vp]
+        L.iq_rotation_params_per_head.restype = i32
+        L.iq_rotation_params_per_head.argtypes = [i32]
         L.iq_encode_append.restype = ctypes.c_int
         L.iq_encode_append.argtypes = [P, i32, vp, vp, i32, i32, vp, vp, vp]
         L.iq_decode_workspace_size.restype = sz
@@ -120,9 +147,10 @@ def iq_status_string(status):
     return lib().iq_status_string(int(status)).decode()
 
 
-def iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages):
+def iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, k_bits=3, v_bits=3):
     a = ctypes.c_size_t(0)
-    _check("iq_cache_bytes", lib().iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, ctypes.byref(a)))
+    _check("iq_cache_bytes", lib().iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, k_bits, v_bits,
+                                                  ctypes.byref(a)))
     return a.value
 
 
@@ -131,6 +159,22 @@ def iq_init_rotation(seed, n_layers, n_kv_heads):
     out = np.zeros((n_layers, n_kv_heads, 32, 2, 4), dtype=np.float32)
     _check("iq_init_rotation", lib().iq_init_rotation(ctypes.c_uint64(seed), n_layers, n_kv_heads,
                                                       out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def iq_rotation_params_per_head(rotation):
+    return int(lib().iq_rotation_params_per_head(int(rotation)))
+
+
+PARAM_SHAPE = {IQ_ROT_ISO: (32, 2, 4), IQ_ROT_QUAT: (32, 4), IQ_ROT_PLANAR: (64, 2)}
+
+
+def iq_init_rotation_variant(seed, rotation, n_layers, n_kv_heads):
+    """Seeded parameters of any rotation variant: host float32 [L][Hkv][...] (see include/iq.h)."""
+    rot = ROTATIONS.get(rotation, rotation)
+    out = np.zeros((n_layers, n_kv_heads) + PARAM_SHAPE[rot], dtype=np.float32)
+    _check("iq_init_rotation_variant", lib().iq_init_rotation_variant(ctypes.c_uint64(seed), rot, n_layers,
+                                                                      n_kv_heads, out.ctypes.data_as(ctypes.c_void_p)))
     return out
 
 
@@ -194,41 +238,49 @@ class PagedCache:
     struct over it.
 
     page_size tokens per page (a multiple of 32); with block_table None, sequence b owns page b
-    (a contiguous cache of capacity page_size tokens per sequence).  The k_codes, v_codes,
-    k_norms and v_norms attributes are strided views of the pool's tile records."""
+    (a contiguous cache of capacity page_size tokens per sequence).  k_bits / v_bits are the
+    code widths, rotation the variant ("iso", "quat", "planar" or its IQ_ROT_* value).  The
+    k_codes, v_codes, k_norms and v_norms attributes are strided views of the pool's tile records."""
 
-    def __init__(self, n_layers, n_kv_heads, page_size, n_pages, block_table=None, device="cuda"):
+    def __init__(self, n_layers, n_kv_heads, page_size, n_pages, block_table=None, device="cuda", k_bits=3, v_bits=3,
+                 rotation=IQ_ROT_ISO):
         import torch
 
-        self.pool = torch.empty(iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages), dtype=torch.uint8,
-                                device=device)
+        self.k_bits, self.v_bits = k_bits, v_bits
+        self.rotation = ROTATIONS.get(rotation, rotation)
+        self.tile_bytes = tile_bytes(k_bits, v_bits)
+        self.pool = torch.empty(iq_cache_bytes(n_layers, n_kv_heads, page_size, n_pages, k_bits, v_bits),
+                                dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.block_table = block_table
         self.n_layers, self.n_kv_heads, self.page_size, self.n_pages = n_layers, n_kv_heads, page_size, n_pages
         self.max_pages_per_seq = int(block_table.shape[1]) if block_table is not None else 1
         t = self.tiles()
-        self.k_codes = t[..., 0:1536]
-        self.v_codes = t[..., 1536:3072]
-        self.k_norms = t[..., 3072:3136].view(torch.int16)
-        self.v_norms = t[..., 3136:3200].view(torch.int16)
+        kv0 = 32 * k_record_bytes(k_bits)
+        kn0 = kv0 + 2 * v_block_bytes(v_bits)
+        self.k_codes = t[..., 0:kv0]
+        self.v_codes = t[..., kv0:kn0]
+        self.k_norms = t[..., kn0:kn0 + 64].view(torch.int16)
+        self.v_norms = t[..., kn0 + 64:kn0 + 128].view(torch.int16)
         self.c = iq_cache(
             self.pool.data_ptr(), n_layers, n_kv_heads, HEAD_DIM, page_size, n_pages,
             block_table.data_ptr() if block_table is not None else None,
-            self.max_pages_per_seq, self.status.data_ptr(),
+            self.max_pages_per_seq, self.status.data_ptr(), k_bits, v_bits, self.rotation,
         )
 
     def tiles(self):
-        """[L][n_pages][Hkv][page_size/32][3200] tile records."""
-        return self.pool.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // TILE_TOKENS, TILE_BYTES)
+        """[L][n_pages][Hkv][page_size/32][tile_bytes] tile records."""
+        return self.pool.view(self.n_layers, self.n_pages, self.n_kv_heads, self.page_size // TILE_TOKENS,
+                              self.tile_bytes)
 
     # Views with the records' logical shapes (for writing oracle-made records in tests).
     def k_code_view(self):
-        """[L][n_pages][Hkv][page_size/32][32][48]"""
-        return self.k_codes.view(*self.k_codes.shape[:-1], TILE_TOKENS, K_RECORD_BYTES)
+        """[L][n_pages][Hkv][page_size/32][32][16 k_bits]"""
+        return self.k_codes.view(*self.k_codes.shape[:-1], TILE_TOKENS, k_record_bytes(self.k_bits))
 
     def v_code_view(self):
-        """[L][n_pages][Hkv][page_size/32][2][768]"""
-        return self.v_codes.view(*self.v_codes.shape[:-1], 2, V_BLOCK_BYTES)
+        """[L][n_pages][Hkv][page_size/32][2][256 v_bits]"""
+        return self.v_codes.view(*self.v_codes.shape[:-1], 2, v_block_bytes(self.v_bits))
 
     def k_norm_view(self):
         """[L][n_pages][Hkv][page_size/32][32] int16"""

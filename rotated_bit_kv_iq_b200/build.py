@@ -3,11 +3,15 @@
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libiq.so")
-CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu", "iq_noalloc.cu"]
+CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu", "iq_noalloc.cu",
+                # decode kernels, one unit per (K bits, V bits) pair
+                "iq_decode_k2v2.cu", "iq_decode_k3v2.cu", "iq_decode_k3v3.cu", "iq_decode_k4v2.cu",
+                "iq_decode_k4v3.cu", "iq_decode_k4v4.cu"]
 HOST_SOURCES = ["iq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -31,24 +35,26 @@ def build(verbose=False, force=False):
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_source_mtime():
         return LIB
     nvcc = _nvcc()
-    objs = []
     bdir = os.path.join(HERE, "_build")
     os.makedirs(bdir, exist_ok=True)
     common = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", CSRC, "-I", os.path.join(HERE, "..", "include")]
+    jobs = []
     for src in CUDA_SOURCES:
         obj = os.path.join(bdir, src + ".o")
         cmd = [nvcc, *ARCH, "-lineinfo", *common, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        jobs.append((cmd, obj))
     for src in HOST_SOURCES:
         obj = os.path.join(bdir, src + ".o")
         # host PRNG: IEEE double arithmetic without contraction (bit-reproducible parameters)
         cmd = [nvcc, *common, "-Wno-deprecated-gpu-targets", "-Xcompiler", "-ffp-contract=off", "-x", "c++", "-c",
                os.path.join(CSRC, src), "-o", obj]
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        jobs.append((cmd, obj))
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        for f in [ex.submit(subprocess.run, cmd, check=True) for cmd, _ in jobs]:
+            f.result()
+    objs = [obj for _, obj in jobs]
     tmp = LIB + ".tmp"
     subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart"], check=True)
     os.replace(tmp, LIB)

@@ -12,11 +12,12 @@ namespace iq {
 
 // Centroids reach the tensor cores as int8 pairs: alpha8 * c_k ~ hi_k + lo_k / 254 with
 // hi_k, lo_k integers in [-127, 127].  alpha8 is the scale (searched on a 1e-5 grid below the
-// largest admissible value) that minimises the worst relative error over the four centroid
-// magnitudes; for the 3-bit N(0,1) codebook it is under 3e-6, far below the fp32 rounding of
-// the products that follow.
-static void int8_levels(const Codebook& cb, double& alpha8, int hi[8], int lo[8]) {
-  const double cmax = cb.level[7];
+// largest admissible value) that minimises the worst relative error over the codebook's
+// positive levels; for the 2-, 3- and 4-bit N(0,1) codebooks it is far below the fp32 rounding
+// of the products that follow (3 bits: under 3e-6).
+static void int8_levels(const Codebook& cb, double& alpha8, int hi[16], int lo[16]) {
+  const int n = 1 << cb.bits;
+  const double cmax = cb.level[n - 1];
   double best = 1e30;
   alpha8 = 0.0;
   for (long i = 0;; ++i) {
@@ -24,50 +25,56 @@ static void int8_levels(const Codebook& cb, double& alpha8, int hi[8], int lo[8]
     if (a < 0.5 * 127.49 / cmax) break;
     double err = 0.0;
     bool ok = true;
-    for (int k = 4; k < 8; ++k) {
+    for (int k = n / 2; k < n; ++k) {
       const double v = a * cb.level[k];
       const double h = std::nearbyint(v);
       const double l = std::nearbyint((v - h) * 254.0);
       if (std::fabs(h) > 127.0 || std::fabs(l) > 127.0) { ok = false; break; }
       err = std::fmax(err, std::fabs((h + l / 254.0) / a - cb.level[k]) / cb.level[k]);
+      if (err >= best) { ok = false; break; }
     }
     if (ok && err < best) { best = err; alpha8 = a; }
   }
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < n; ++k) {
     const double v = alpha8 * cb.level[k];
     hi[k] = (int)std::nearbyint(v);
     lo[k] = (int)std::nearbyint((v - hi[k]) * 254.0);
   }
 }
 
-static KernelConsts make_consts() {
-  const Codebook cb = compute_codebook();
-  KernelConsts kc;
-  for (int j = 0; j < 3; ++j) kc.bound_pos[j] = (float)cb.bound[4 + j];
+static SideConsts make_side(int bits) {
+  const Codebook cb = compute_codebook(bits);
+  const int n = 1 << bits;
+  SideConsts sc = {};
+  sc.bits = bits;
+  for (int j = 0; j < n / 2 - 1; ++j) sc.bound_pos[j] = (float)cb.bound[n / 2 + j];
   double alpha8;
-  int hi[8], lo[8];
+  int hi[16], lo[16];
   int8_levels(cb, alpha8, hi, lo);
-  uint32_t h4[2] = {0, 0}, l4[2] = {0, 0};
-  for (int k = 0; k < 8; ++k) {
-    h4[k >> 2] |= (uint32_t)(uint8_t)(int8_t)hi[k] << (8 * (k & 3));
-    l4[k >> 2] |= (uint32_t)(uint8_t)(int8_t)lo[k] << (8 * (k & 3));
+  for (int k = 0; k < n; ++k) {
+    sc.lut_hi[k >> 2] |= (uint32_t)(uint8_t)(int8_t)hi[k] << (8 * (k & 3));
+    sc.lut_lo[k >> 2] |= (uint32_t)(uint8_t)(int8_t)lo[k] << (8 * (k & 3));
   }
-  kc.lut_hi[0] = h4[0];
-  kc.lut_hi[1] = h4[1];
-  kc.lut_lo[0] = l4[0];
-  kc.lut_lo[1] = l4[1];
-  kc.alpha8 = (float)alpha8;
-  return kc;
+  sc.alpha8 = (float)alpha8;
+  return sc;
 }
 
-const KernelConsts& kernel_consts() {
+const KernelConsts& kernel_consts(int kb, int vb) {
   static std::once_flag once;
-  static KernelConsts kc;
-  std::call_once(once, [] { kc = make_consts(); });
-  return kc;
+  static SideConsts side[5];
+  static KernelConsts table[5][5];
+  std::call_once(once, [] {
+    for (int b = 2; b <= 4; ++b) side[b] = make_side(b);
+    for (int k = 2; k <= 4; ++k)
+      for (int v = 2; v <= 4; ++v) table[k][v] = KernelConsts{side[k], side[v]};
+  });
+  return table[kb][vb];
 }
 
 static bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static int k_bits(const iq_cache* c) { return c->k_bits ? c->k_bits : 3; }
+static int v_bits(const iq_cache* c) { return c->v_bits ? c->v_bits : 3; }
 
 static iq_status check_cache(const iq_cache* c, int32_t layer) {
   if (!c) return IQ_ERR_INVALID_ARG;
@@ -78,21 +85,33 @@ static iq_status check_cache(const iq_cache* c, int32_t layer) {
   if (layer < 0 || layer >= c->n_layers) return IQ_ERR_INVALID_ARG;
   if (!c->pool) return IQ_ERR_INVALID_ARG;
   if (c->block_table_dev && c->max_pages_per_seq < 1) return IQ_ERR_INVALID_ARG;
+  if (!supported_widths(k_bits(c), v_bits(c))) return IQ_ERR_UNSUPPORTED;
+  if (c->rotation != IQ_ROT_ISO && c->rotation != IQ_ROT_QUAT && c->rotation != IQ_ROT_PLANAR) return IQ_ERR_UNSUPPORTED;
   if (!aligned(c->pool, 16)) return IQ_ERR_ALIGNMENT;
   return IQ_OK;
 }
 
+static size_t layer_pool_bytes(const iq_cache* c) {
+  return (size_t)c->n_pages * c->n_kv_heads * (c->page_size / TILE_TOKENS) * tile_bytes(k_bits(c), v_bits(c));
+}
+
 static LayerView view(const iq_cache* c, int32_t layer) {
   LayerView v;
-  const size_t per_layer_tiles = (size_t)c->n_pages * c->n_kv_heads * (c->page_size / TILE_TOKENS);
-  v.pool = (uint8_t*)c->pool + per_layer_tiles * TILE_BYTES * layer;
+  v.pool = (uint8_t*)c->pool + layer_pool_bytes(c) * layer;
   v.block_table = c->block_table_dev;
   v.max_pages = c->block_table_dev ? c->max_pages_per_seq : 1;
   v.page_size = c->page_size;
   v.n_pages = c->n_pages;
   v.n_kv_heads = c->n_kv_heads;
   v.status = c->status_dev;
+  v.kb = k_bits(c);
+  v.vb = v_bits(c);
+  v.rot = c->rotation;
   return v;
+}
+
+static const float* layer_params(const iq_cache* c, const float* params_dev, int32_t layer) {
+  return params_dev + (size_t)layer * c->n_kv_heads * params_per_head(c->rotation);
 }
 
 static int64_t seq_capacity(const iq_cache* c) {
@@ -105,7 +124,7 @@ using namespace iq;
 
 extern "C" {
 
-const char* iq_version(void) { return "libiq 0.1 (sm_100a; packed 3-bit IsoQuant KV)"; }
+const char* iq_version(void) { return "libiq 0.2 (sm_100a; packed 2/3/4-bit IsoQuant KV)"; }
 
 const char* iq_status_string(iq_status s) {
   switch (s) {
@@ -120,18 +139,31 @@ const char* iq_status_string(iq_status s) {
   return "unknown status";
 }
 
-iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages,
-                         size_t* pool_bytes_host) {
+iq_status iq_cache_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t page_size, int32_t n_pages, int32_t k_bits,
+                         int32_t v_bits, size_t* pool_bytes_host) {
   if (n_layers < 1 || n_kv_heads < 1 || page_size < TILE_TOKENS || page_size % TILE_TOKENS != 0 || n_pages < 1)
     return IQ_ERR_INVALID_ARG;
+  const int kb = k_bits ? k_bits : 3, vb = v_bits ? v_bits : 3;
+  if (!supported_widths(kb, vb)) return IQ_ERR_UNSUPPORTED;
   if (pool_bytes_host)
-    *pool_bytes_host = (size_t)n_layers * n_pages * n_kv_heads * (page_size / TILE_TOKENS) * TILE_BYTES;
+    *pool_bytes_host = (size_t)n_layers * n_pages * n_kv_heads * (page_size / TILE_TOKENS) * tile_bytes(kb, vb);
   return IQ_OK;
 }
 
 iq_status iq_init_rotation(uint64_t seed, int32_t n_layers, int32_t n_kv_heads, float* params_host) {
+  return iq_init_rotation_variant(seed, IQ_ROT_ISO, n_layers, n_kv_heads, params_host);
+}
+
+int32_t iq_rotation_params_per_head(int32_t rotation) {
+  return (rotation == IQ_ROT_ISO || rotation == IQ_ROT_QUAT || rotation == IQ_ROT_PLANAR) ? params_per_head(rotation)
+                                                                                         : 0;
+}
+
+iq_status iq_init_rotation_variant(uint64_t seed, int32_t rotation, int32_t n_layers, int32_t n_kv_heads,
+                                   float* params_host) {
   if (!params_host || n_layers < 1 || n_kv_heads < 1) return IQ_ERR_INVALID_ARG;
-  init_rotation_params(seed, n_layers, n_kv_heads, params_host);
+  if (iq_rotation_params_per_head(rotation) == 0) return IQ_ERR_UNSUPPORTED;
+  init_rotation_params(seed, rotation, n_layers, n_kv_heads, params_host);
   return IQ_OK;
 }
 
@@ -148,8 +180,8 @@ iq_status iq_encode_append(const iq_cache* cache, int32_t layer, const void* k_d
       !aligned(start_pos_dev, 4))
     return IQ_ERR_ALIGNMENT;
   const LayerView v = view(cache, layer);
-  const float* pl = params_dev + (size_t)layer * cache->n_kv_heads * NBLK * 8;
-  const int e = launch_encode(v, k_dev, v_dev, batch, n_new, start_pos_dev, pl, kernel_consts(), stream);
+  const int e = launch_encode(v, k_dev, v_dev, batch, n_new, start_pos_dev, layer_params(cache, params_dev, layer),
+                              kernel_consts(v.kb, v.vb), stream);
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 
@@ -179,9 +211,9 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
   if (!workspace_dev || workspace_bytes < need) return IQ_ERR_WORKSPACE;
   if (!aligned(workspace_dev, 256)) return IQ_ERR_ALIGNMENT;
   const LayerView v = view(cache, layer);
-  const float* pl = params_dev + (size_t)layer * cache->n_kv_heads * NBLK * 8;
-  const int e = launch_decode(v, q_dev, q_dtype == IQ_F32, batch, n_q_heads, ctx_len_dev, max_ctx, pl, out_dev,
-                              workspace_dev, kernel_consts(), stream);
+  const int e = launch_decode(v, q_dev, q_dtype == IQ_F32, batch, n_q_heads, ctx_len_dev, max_ctx,
+                              layer_params(cache, params_dev, layer), out_dev, workspace_dev,
+                              kernel_consts(v.kb, v.vb), stream);
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 
@@ -208,9 +240,9 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
   if (!workspace_dev || workspace_bytes < need) return IQ_ERR_WORKSPACE;
   if (!aligned(workspace_dev, 256)) return IQ_ERR_ALIGNMENT;
   const LayerView v = view(cache, layer);
-  const float* pl = params_dev + (size_t)layer * cache->n_kv_heads * NBLK * 8;
   const int e = launch_decode_step(v, q_dev, q_dtype == IQ_F32, k_new_dev, v_new_dev, batch, n_q_heads, ctx_len_dev,
-                                   max_ctx, pl, out_dev, workspace_dev, kernel_consts(), stream);
+                                   max_ctx, layer_params(cache, params_dev, layer), out_dev, workspace_dev,
+                                   kernel_consts(v.kb, v.vb), stream);
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 
@@ -222,7 +254,7 @@ iq_status iq_export_codes(const iq_cache* cache, int32_t layer, int32_t kv, int3
   if (!cache->block_table_dev && seq >= cache->n_pages) return IQ_ERR_CAPACITY;
   if ((int64_t)t0 + n > seq_capacity(cache)) return IQ_ERR_CAPACITY;
   const LayerView v = view(cache, layer);
-  const int e = launch_export(v, kv, seq, t0, n, codes_dev, norms_dev, kernel_consts(), stream);
+  const int e = launch_export(v, kv, seq, t0, n, codes_dev, norms_dev, stream);
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 

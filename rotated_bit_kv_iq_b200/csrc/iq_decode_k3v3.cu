@@ -1,0 +1,7 @@
+// Decode kernels for K codes of 3 bits and V codes of 3 bits (explicit instantiation).
+#include "iq_decode_impl.cuh"
+
+namespace iq {
+template int launch_decode_kv<3, 3>(const LayerView&, const void*, int, int, int, const int32_t*, int, const float*,
+                                   float*, void*, const KernelConsts&, void*, const void*, const void*);
+}  // namespace iq

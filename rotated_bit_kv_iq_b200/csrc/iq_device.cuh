@@ -79,6 +79,38 @@ __device__ __forceinline__ void fused_block_matrix(const float* q, float Mp[4][4
   }
 }
 
+// The 4x4 matrix that the rotation variant `rot` applies to coordinates 4k..4k+3 after the WHT
+// stages on bits 2..6 (ROT_ISO only), from the block's parameters p:
+//   ROT_ISO    (qL, qR) at p[0..7]: the fused matrix above;
+//   ROT_QUAT   q at p[0..3]: left multiplication y -> q * y (Hamilton product), q rescaled to unit;
+//   ROT_PLANAR (c0, s0, c1, s1) at p[0..3]: Givens rotations of the pairs (4k, 4k+1) and
+//              (4k+2, 4k+3), (y0, y1) -> (c y0 - s y1, s y0 + c y1), each (c, s) rescaled to unit.
+__device__ __forceinline__ void variant_block_matrix(int rot, const float* p, float Mp[4][4]) {
+  if (rot == ROT_ISO) {
+    fused_block_matrix(p, Mp);
+  } else if (rot == ROT_QUAT) {
+    float a0 = p[0], a1 = p[1], a2 = p[2], a3 = p[3];
+    const float na = 1.f / sqrtf(fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3))));
+    a0 *= na; a1 *= na; a2 *= na; a3 *= na;
+    Mp[0][0] = a0; Mp[0][1] = -a1; Mp[0][2] = -a2; Mp[0][3] = -a3;
+    Mp[1][0] = a1; Mp[1][1] = a0;  Mp[1][2] = -a3; Mp[1][3] = a2;
+    Mp[2][0] = a2; Mp[2][1] = a3;  Mp[2][2] = a0;  Mp[2][3] = -a1;
+    Mp[3][0] = a3; Mp[3][1] = -a2; Mp[3][2] = a1;  Mp[3][3] = a0;
+  } else {
+    const float n0 = 1.f / sqrtf(fmaf(p[0], p[0], p[1] * p[1])), n1 = 1.f / sqrtf(fmaf(p[2], p[2], p[3] * p[3]));
+    const float c0 = p[0] * n0, s0 = p[1] * n0, c1 = p[2] * n1, s1 = p[3] * n1;
+    Mp[0][0] = c0; Mp[0][1] = -s0; Mp[0][2] = 0.f; Mp[0][3] = 0.f;
+    Mp[1][0] = s0; Mp[1][1] = c0;  Mp[1][2] = 0.f; Mp[1][3] = 0.f;
+    Mp[2][0] = 0.f; Mp[2][1] = 0.f; Mp[2][2] = c1; Mp[2][3] = -s1;
+    Mp[3][0] = 0.f; Mp[3][1] = 0.f; Mp[3][2] = s1; Mp[3][3] = c1;
+  }
+}
+
+// Parameters of block k of kv head `head` in a layer's parameter array.
+__device__ __forceinline__ const float* block_params(const float* params_layer, int rot, int head, int k) {
+  return params_layer + (size_t)head * params_per_head(rot) + k * params_per_block(rot);
+}
+
 // ------------------------------------------------------------------ warp rotation
 // One warp rotates one 128-vector: lane l holds coordinates 4l..4l+3.  Forward: WHT
 // stages on coordinate bits 2..6 (lane bits 0..4) by shuffles, then M'_l.  Inverse:
@@ -96,8 +128,8 @@ __device__ __forceinline__ void warp_wht_bits2to6(float v[4]) {
   }
 }
 
-__device__ __forceinline__ void warp_rotate_forward(float v[4], const float Mp[4][4]) {
-  warp_wht_bits2to6(v);
+__device__ __forceinline__ void warp_rotate_forward(float v[4], const float Mp[4][4], bool wht) {
+  if (wht) warp_wht_bits2to6(v);
   float z[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) z[r] = Mp[r][0] * v[0] + Mp[r][1] * v[1] + Mp[r][2] * v[2] + Mp[r][3] * v[3];
@@ -105,30 +137,72 @@ __device__ __forceinline__ void warp_rotate_forward(float v[4], const float Mp[4
   for (int r = 0; r < 4; ++r) v[r] = z[r];
 }
 
-__device__ __forceinline__ void warp_rotate_inverse(float v[4], const float Mp[4][4]) {
+__device__ __forceinline__ void warp_rotate_inverse(float v[4], const float Mp[4][4], bool wht) {
   float z[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) z[c] = Mp[0][c] * v[0] + Mp[1][c] * v[1] + Mp[2][c] * v[2] + Mp[3][c] * v[3];
 #pragma unroll
   for (int c = 0; c < 4; ++c) v[c] = z[c];
-  warp_wht_bits2to6(v);
+  if (wht) warp_wht_bits2to6(v);
 }
 
 // ------------------------------------------------------------------ packed codes
-// 32-code chunk: W_w bits [4j,4j+3) = slot 8w+j, bit 4j+3 = bit w of slot 24+j.
-// Selector words for byte-permute lookups: sel[w] (w<3) holds slots 8w..8w+7 as clean
-// nibbles, sel[3] holds slots 24..31.
-__device__ __forceinline__ void chunk_selectors(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t sel[4]) {
-  sel[0] = w0 & 0x77777777u;
-  sel[1] = w1 & 0x77777777u;
-  sel[2] = w2 & 0x77777777u;
-  sel[3] = ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
+// A chunk holds 32 codes (slots 0..31) in BITS little-endian words; its four selector words
+// sel[w] (w = 0..3) hold slot 8w + j as nibble j, bits above the code clear:
+//   BITS 3: W_w bits [4j,4j+3) = slot 8w+j, bit 4j+3 = bit w of slot 24+j (w < 3);
+//   BITS 4: W_w = sel[w];
+//   BITS 2: W_w bits [4j,4j+2) = slot 16w+j, bits [4j+2,4j+4) = slot 16w+8+j (w < 2).
+template <int BITS>
+__device__ __forceinline__ void chunk_selectors(const uint32_t* w, uint32_t sel[4]) {
+  if constexpr (BITS == 3) {
+    sel[0] = w[0] & 0x77777777u;
+    sel[1] = w[1] & 0x77777777u;
+    sel[2] = w[2] & 0x77777777u;
+    sel[3] = ((w[0] >> 3) & 0x11111111u) | ((w[1] >> 2) & 0x22222222u) | ((w[2] >> 1) & 0x44444444u);
+  } else if constexpr (BITS == 4) {
+    sel[0] = w[0];
+    sel[1] = w[1];
+    sel[2] = w[2];
+    sel[3] = w[3];
+  } else {
+    sel[0] = w[0] & 0x33333333u;
+    sel[1] = (w[0] >> 2) & 0x33333333u;
+    sel[2] = w[1] & 0x33333333u;
+    sel[3] = (w[1] >> 2) & 0x33333333u;
+  }
+}
+
+// Storage word k (k < BITS) of a chunk from its four selector words (the inverse of the
+// above).  Every token's codes sit in whole nibbles of the selector words, and this map keeps
+// nibble positions: a nibble of the selector words lands in the same nibble of storage words.
+template <int BITS>
+__device__ __forceinline__ uint32_t pack_word(int k, uint32_t s0, uint32_t s1, uint32_t s2, uint32_t s3) {
+  if constexpr (BITS == 4) return k == 0 ? s0 : k == 1 ? s1 : k == 2 ? s2 : s3;
+  if constexpr (BITS == 3) {
+    const uint32_t s = k == 0 ? s0 : k == 1 ? s1 : s2;
+    return s | (((s3 >> k) & 0x11111111u) << 3);
+  }
+  return k == 0 ? (s0 | (s1 << 2)) : (s2 | (s3 << 2));
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
+}
+
+// Table lookup of four codes (nibbles 0..3 of s, bits above the code clear) into their int8
+// centroid terms: byte i of the result = entry (nibble i) of the 2^BITS-entry table t (byte k of
+// the little-endian words t[0..] = entry k).  2 and 3 bits: one byte permute; 4 bits: a permute
+// in each half of the table and a byte select on the code's top bit.
+template <int BITS>
+__device__ __forceinline__ uint32_t lut4(const uint32_t* t, uint32_t s) {
+  if constexpr (BITS == 2) return prmt(t[0], t[0], s);
+  if constexpr (BITS == 3) return prmt(t[0], t[1], s);
+  const uint32_t s7 = s & 0x7777u;
+  const uint32_t m = prmt(0x0000FF00u, 0u, (s >> 3) & 0x1111u);  // byte i = 0xFF when code i >= 8
+  const uint32_t a = prmt(t[0], t[1], s7), b = prmt(t[2], t[3], s7);
+  return (a & ~m) | (b & m);
 }
 
 // Packed fp32 pairs (add/sub/mul/fma .f32x2: two IEEE fp32 operations per instruction, each
@@ -192,16 +266,18 @@ __device__ __forceinline__ float half_bits_to_float(uint16_t h) { return __half2
 
 // Tile record holding `slot` of (page, kv head), and the pieces of one slot inside it.
 __device__ __forceinline__ uint8_t* tile_record(const LayerView& v, int page, int head, int slot) {
-  return v.pool + (((size_t)page * v.n_kv_heads + head) * (v.page_size / TILE_TOKENS) + slot / TILE_TOKENS) * TILE_BYTES;
+  return v.pool + (((size_t)page * v.n_kv_heads + head) * (v.page_size / TILE_TOKENS) + slot / TILE_TOKENS) *
+                      (size_t)tile_bytes(v.kb, v.vb);
 }
 __device__ __forceinline__ uint8_t* k_record(const LayerView& v, int page, int head, int slot) {
-  return tile_record(v, page, head, slot) + TR_K + (slot % TILE_TOKENS) * K_REC;
+  return tile_record(v, page, head, slot) + (slot % TILE_TOKENS) * k_rec_bytes(v.kb);
 }
 __device__ __forceinline__ uint8_t* v_block(const LayerView& v, int page, int head, int slot) {
-  return tile_record(v, page, head, slot) + TR_V + ((slot % TILE_TOKENS) / V_BLK_TOKENS) * V_BLK;
+  return tile_record(v, page, head, slot) + tr_v(v.kb) + ((slot % TILE_TOKENS) / V_BLK_TOKENS) * v_blk_bytes(v.vb);
 }
 __device__ __forceinline__ uint16_t* norm_slot(const LayerView& v, int page, int head, int slot, int side) {
-  return reinterpret_cast<uint16_t*>(tile_record(v, page, head, slot) + (side ? TR_VN : TR_KN)) + slot % TILE_TOKENS;
+  return reinterpret_cast<uint16_t*>(tile_record(v, page, head, slot) + (side ? tr_vn(v.kb, v.vb) : tr_kn(v.kb, v.vb))) +
+         slot % TILE_TOKENS;
 }
 
 // Resolve the page of token `pos` of sequence `b`; returns -1 (and flags) when invalid.
@@ -299,24 +375,37 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // ------------------------------------------------------------------ quantiser
-// code = #{ j : u > b_j } with u = sqrt(128) z / n, written with the three positive
-// thresholds t_j = b_j n / sqrt(128): magnitude class m = #{ |z| > t_j }, code = 4+m for
-// z > 0 and 3-m otherwise.  (Exact ties |z| = t_j are within rounding of a boundary.)
-__device__ __forceinline__ uint32_t quantise(float z, float t1, float t2, float t3) {
+// code = #{ j : u > b_j } with u = sqrt(128) z / n, written with the positive thresholds
+// t_j = b_j n / sqrt(128) (2^(BITS-1) - 1 of them; the middle boundary is 0): magnitude class
+// m = #{ |z| > t_j }, code = 2^(BITS-1) + m for z > 0 and 2^(BITS-1) - 1 - m otherwise.
+// (Exact ties |z| = t_j are within rounding of a boundary.)
+template <int BITS>
+__device__ __forceinline__ uint32_t quantise(float z, const float* t) {
   const float a = fabsf(z);
-  const uint32_t m = (uint32_t)(a > t1) + (uint32_t)(a > t2) + (uint32_t)(a > t3);
-  return z > 0.f ? 4u + m : 3u - m;
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < (1 << (BITS - 1)) - 1; ++j) m += (uint32_t)(a > t[j]);
+  constexpr uint32_t half = 1u << (BITS - 1);
+  return z > 0.f ? half + m : half - 1u - m;
+}
+
+// Thresholds of one side scaled to a vector of norm n: t_j = b_j n / sqrt(128).
+template <int BITS>
+__device__ __forceinline__ void scaled_thresholds(const SideConsts& sc, float n, float* t) {
+  const float s = n * 0.08838834764831845f;
+#pragma unroll
+  for (int j = 0; j < (1 << (BITS - 1)) - 1; ++j) t[j] = sc.bound_pos[j] * s;
 }
 
 // ------------------------------------------------------------------ one-warp vector encoder
-// One warp encodes one fp16 vector (128 values at `src`) into the K (side 0) or V (side 1)
-// record of kv head `head` at (page, slot); lane l owns coordinates 4l..4l+3 (one SO(4)
-// block).  WHT stages on coordinate bits 2..6 run as shuffles; the lane's fused block matrix
-// is passed in.  K words are assembled with two shuffles; a V block gets only this token's
-// bits (see below).
+// One warp encodes one fp16 vector (128 values at `src`) into the K (side 0, width KB) or V
+// (side 1, width VB) record of kv head `head` at (page, slot); lane l owns coordinates
+// 4l..4l+3 (one rotation block).  The WHT stages (ROT_ISO) run as shuffles; the lane's block
+// matrix is passed in.  A V block gets only this token's bits (see below).
+template <int BITS>
 __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __half* __restrict__ src, int head,
                                                    int side, int page, int slot, const float Mp[4][4],
-                                                   const KernelConsts& kc) {
+                                                   const SideConsts& sc) {
   const int lane = threadIdx.x & 31;
   const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
   const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
@@ -326,50 +415,62 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float n = sqrtf(ss);
-  warp_rotate_forward(x, Mp);
-  const float sc = n * 0.08838834764831845f;
-  const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
-  const uint32_t c0 = quantise(x[0], t1, t2, t3), c1 = quantise(x[1], t1, t2, t3);
-  const uint32_t c2 = quantise(x[2], t1, t2, t3), c3 = quantise(x[3], t1, t2, t3);
+  warp_rotate_forward(x, Mp, v.rot == ROT_ISO);
+  float t[7];
+  scaled_thresholds<BITS>(sc, n, t);
+  const uint32_t c0 = quantise<BITS>(x[0], t), c1 = quantise<BITS>(x[1], t);
+  const uint32_t c2 = quantise<BITS>(x[2], t), c3 = quantise<BITS>(x[3], t);
   if (side == 0) {
-    // K chunk c = lanes 8c..8c+7; word w = lanes 8c+2w (low half) and 8c+2w+1 (high half);
-    // spare slots 24..31 = lanes 8c+6, 8c+7.
+    // K chunk c = lanes 8c..8c+7; lane 8c + 2w + e holds nibbles 4e..4e+3 of selector word w.
     const uint32_t v16 = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
-    const uint32_t pair = v16 | (__shfl_xor_sync(0xffffffffu, v16, 1) << 16);
-    const uint32_t spare = __shfl_sync(0xffffffffu, pair, (lane & ~7) | 6);
-    const int w = (lane & 7) >> 1;
-    if ((lane & 1) == 0 && w < 3) {
-      const uint32_t word = pair | (((spare >> w) & 0x11111111u) << 3);
-      uint32_t* rec = reinterpret_cast<uint32_t*>(k_record(v, page, head, slot));
-      rec[3 * (lane >> 3) + w] = word;
+    const uint32_t sw = v16 | (__shfl_xor_sync(0xffffffffu, v16, 1) << 16);  // selector word on even lanes
+    uint32_t* rec = reinterpret_cast<uint32_t*>(k_record(v, page, head, slot));
+    if constexpr (BITS == 3) {
+      // storage word w = selector word w (lane 8c + 2w) with the spare bits of selector word 3
+      const uint32_t spare = __shfl_sync(0xffffffffu, sw, (lane & ~7) | 6);
+      const int w = (lane & 7) >> 1;
+      if ((lane & 1) == 0 && w < 3) rec[3 * (lane >> 3) + w] = sw | (((spare >> w) & 0x11111111u) << 3);
+    } else {
+      const int base = lane & ~7;
+      const uint32_t s0 = __shfl_sync(0xffffffffu, sw, base), s1 = __shfl_sync(0xffffffffu, sw, base + 2);
+      const uint32_t s2 = __shfl_sync(0xffffffffu, sw, base + 4), s3 = __shfl_sync(0xffffffffu, sw, base + 6);
+      const int k = lane & 7;
+      if (k < BITS) rec[BITS * (lane >> 3) + k] = pack_word<BITS>(k, s0, s1, s2, s3);
     }
   } else {
-    // V block: this token (u = slot mod 16) owns nibbles j and j+4 of the three words of the
-    // chunks (g, tq, h) with tq = (u mod 8) / 2, j = 2 (u / 8) + (u mod 2).  Word w of chunk
-    // (g, tq, h) takes codes of coordinates 32w + g + 8h (nibble j) and 32w + 16 + g + 8h
-    // (nibble j+4), and bit w of the codes of coordinates 96 + g + 8h and 112 + g + 8h as
-    // the spare bits.  Lane l writes words k = l and l + 32 (k < 48) of the token's
-    // (g, h, w) list; the other tokens' bits are kept (atomic and/or: tokens of one block may
-    // be appended by several warps of one launch).
+    // V block: this token (u = slot mod 16) owns nibbles j and j+4 of the selector words of
+    // the 16 chunks (g, tq, h), tq = (u mod 8) / 2, j = 2 (u / 8) + (u mod 2): nibble j of
+    // selector word w holds coordinate 32w + g + 8h and nibble j+4 coordinate 32w + 16 + g + 8h.
+    // Lane l writes the token's storage words r = l, l + 32 (r < 16 BITS) of its (g, h, word)
+    // list; the other tokens' bits are kept (atomic and/or: tokens of one block may be
+    // appended by several warps of one launch).
     const uint32_t mine = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
     const int u = slot & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
     uint8_t* blk = v_block(v, page, head, slot);
+    auto code_at = [&](int x) { return (__shfl_sync(0xffffffffu, mine, x >> 2) >> (8 * (x & 3))) & 0xFu; };
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int k = lane + 32 * r;
-      const int kk = k < 48 ? k : 0;
-      const int gh = kk / 3, w = kk % 3;
-      const int g = gh >> 1, h = gh & 1;
-      const int x0 = 32 * w + g + 8 * h, x1 = x0 + 16, x2 = 96 + g + 8 * h, x3 = x2 + 16;
-      const uint32_t y0 = (__shfl_sync(0xffffffffu, mine, x0 >> 2) >> (8 * (x0 & 3))) & 7u;
-      const uint32_t y1 = (__shfl_sync(0xffffffffu, mine, x1 >> 2) >> (8 * (x1 & 3))) & 7u;
-      const uint32_t y2 = (__shfl_sync(0xffffffffu, mine, x2 >> 2) >> (8 * (x2 & 3))) & 7u;
-      const uint32_t y3 = (__shfl_sync(0xffffffffu, mine, x3 >> 2) >> (8 * (x3 & 3))) & 7u;
-      if (k < 48) {
-        const uint32_t n0 = y0 | (((y2 >> w) & 1u) << 3), n1 = y1 | (((y3 >> w) & 1u) << 3);
-        const uint32_t bits = (n0 << (4 * j)) | (n1 << (16 + 4 * j));
-        const uint32_t mask = (0xFu << (4 * j)) | (0xFu << (16 + 4 * j));
-        unsigned int* word = reinterpret_cast<unsigned int*>(blk + 12 * (2 * (4 * g + tq) + h) + 4 * w);
+      const int kk = lane + 32 * r;
+      const int k = kk < 16 * BITS ? kk : 0;
+      const int gh = k / BITS, w = k % BITS;
+      const int x = (gh >> 1) + 8 * (gh & 1);  // g + 8h
+      // the token's nibbles j (n0) and j+4 (n1) of storage word w, from the codes they hold
+      uint32_t n0, n1;
+      if constexpr (BITS == 4) {
+        n0 = code_at(32 * w + x);
+        n1 = code_at(32 * w + 16 + x);
+      } else if constexpr (BITS == 3) {
+        n0 = code_at(32 * w + x) | (((code_at(96 + x) >> w) & 1u) << 3);
+        n1 = code_at(32 * w + 16 + x) | (((code_at(112 + x) >> w) & 1u) << 3);
+      } else {
+        n0 = code_at(64 * w + x) | (code_at(64 * w + 32 + x) << 2);
+        n1 = code_at(64 * w + 16 + x) | (code_at(64 * w + 48 + x) << 2);
+      }
+      if (kk < 16 * BITS) {
+        const uint32_t bits = (n0 << (4 * j)) | (n1 << (4 * (j + 4)));
+        const uint32_t mask = (0xFu << (4 * j)) | (0xFu << (4 * (j + 4)));
+        unsigned int* word =
+            reinterpret_cast<unsigned int*>(blk + chunk_bytes(BITS) * (2 * (4 * (gh >> 1) + tq) + (gh & 1)) + 4 * w);
         atomicAnd(word, ~mask);
         atomicOr(word, bits);
       }

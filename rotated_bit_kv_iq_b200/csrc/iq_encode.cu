@@ -7,10 +7,12 @@
 //
 // Mapping: one thread encodes one 128-vector entirely in registers (all seven butterfly
 // stages are register-local, no shuffles).  A CTA covers 128 consecutive positions of one
-// (sequence, kv head, K|V); the head's 32 fused block matrices live in shared memory and
-// every lane of a warp reads the same one at the same time (broadcast).  Instead of
-// normalising the vector, the rotated coordinates z = R x are compared with the
-// boundaries scaled by ||x||/sqrt(128).
+// (sequence, kv head, K|V); the head's 32 block matrices live in shared memory and every
+// lane of a warp reads the same one at the same time (broadcast).  Instead of normalising
+// the vector, the rotated coordinates z = R x are compared with the boundaries scaled by
+// ||x||/sqrt(128).  The code width (2, 3 or 4 bits, "压缩与速度的博弈" section "K 和 V 的非对称需求")
+// is a template parameter; the rotation variant (WHT + quaternion pairs, one quaternion per
+// block, Givens pairs: section "三种变体") is read from the layer view.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -20,23 +22,30 @@ namespace iq {
 
 constexpr int ENC_THREADS = 128;
 
+// Encodes the vectors of the sides side0 .. side0 + n_sides - 1 (0 = K, 1 = V), all of width BITS
+// (so one set of codebook constants, sc, serves every side of the launch);
+// WHT: the layer's rotation is ROT_ISO (WHT stages, then the fused quaternion-pair blocks); else
+// the variant's blocks alone.  (A compile-time choice: a run-time branch around the unrolled
+// stages cost the kernel a quarter more registers.)
+template <int BITS, bool WHT>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int n_new,
-              const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
-  // fused block matrices M'_k as column pairs: smat[k][c][0] = (M'[0][c], M'[1][c]),
+              const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, SideConsts sc,
+              int side0, int n_sides) {
+  // block matrices M'_k as column pairs: smat[k][c][0] = (M'[0][c], M'[1][c]),
   // smat[k][c][1] = (M'[2][c], M'[3][c])
   __shared__ uint64_t smat[NBLK][4][2];
   pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.z;
-  const int head = blockIdx.y >> 1;
-  const int side = blockIdx.y & 1;  // 0 = K, 1 = V
+  const int head = blockIdx.y / n_sides;
+  const int side = side0 + blockIdx.y % n_sides;  // 0 = K, 1 = V
   const __half* src = side ? v_src : k_src;
   if (src == nullptr) return;
 
   if (threadIdx.x < NBLK) {
     float Mp[4][4];
-    fused_block_matrix(params_layer + ((size_t)head * NBLK + threadIdx.x) * 8, Mp);
+    variant_block_matrix(v.rot, block_params(params_layer, v.rot, head, threadIdx.x), Mp);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       smat[threadIdx.x][c][0] = f2(Mp[0][c], Mp[1][c]);
@@ -81,21 +90,23 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   f2s(ss, ss0, ss1);
   const float n = sqrtf(ss0 + ss1);
 
-  // Butterfly stages on coordinate bits 2..6 (bits 0,1 are inside M'), two butterflies per
-  // packed instruction.
+  if (WHT) {
+    // Butterfly stages on coordinate bits 2..6 (bits 0,1 are inside M'), two butterflies per
+    // packed instruction.
 #pragma unroll
-  for (int bit = 2; bit < 7; ++bit) {
-    const int h = 1 << (bit - 1);  // in pairs
+    for (int bit = 2; bit < 7; ++bit) {
+      const int h = 1 << (bit - 1);  // in pairs
 #pragma unroll
-    for (int i = 0; i < D / 2; ++i) {
-      if ((i & h) == 0) {
-        const uint64_t a = y[i], c = y[i + h];
-        y[i] = add2(a, c);
-        y[i + h] = sub2(a, c);
+      for (int i = 0; i < D / 2; ++i) {
+        if ((i & h) == 0) {
+          const uint64_t a = y[i], c = y[i + h];
+          y[i] = add2(a, c);
+          y[i + h] = sub2(a, c);
+        }
       }
     }
   }
-  // Fused SO(4) blocks: rows (0,1) and (2,3) as pairs, z = M' v.
+  // Block matrices: rows (0,1) and (2,3) as pairs, z = M' v.
 #pragma unroll
   for (int k = 0; k < NBLK; ++k) {
     float v0, v1, v2, v3;
@@ -111,9 +122,9 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     y[2 * k + 1] = fma2(smat[k][0][1], b0, z23);
   }
 
-  const float sc = n * 0.08838834764831845f;  // n / sqrt(128)
-  const float t1 = kc.bound_pos[0] * sc, t2 = kc.bound_pos[1] * sc, t3 = kc.bound_pos[2] * sc;
-  // codes once: cw[r] holds coordinates 8r..8r+7 as nibbles (bit 3 clear)
+  float t[7];
+  scaled_thresholds<BITS>(sc, n, t);
+  // codes once: cw[r] holds coordinates 8r..8r+7 as nibbles (bits above the code clear)
   uint32_t cw[16];
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
@@ -122,33 +133,33 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     for (int e = 0; e < 4; ++e) {
       float za, zb;
       f2s(y[4 * r + e], za, zb);
-      w |= quantise(za, t1, t2, t3) << (8 * e);
-      w |= quantise(zb, t1, t2, t3) << (8 * e + 4);
+      w |= quantise<BITS>(za, t) << (8 * e);
+      w |= quantise<BITS>(zb, t) << (8 * e + 4);
     }
     cw[r] = w;
   }
 
   const int slot = pos % v.page_size;
   if (side == 0) {
-    // K record: chunk c = cw[4c..4c+3]; word w of the chunk = slots 8w..8w+7 plus bit w of
-    // slots 24..31 as the spare bits.
+    // K record: chunk c has selector words cw[4c..4c+3] (slot 8w + j = coordinate 32c + 8w + j).
     if (active) {
-      uint32_t rec[12];
+      uint32_t rec[4 * BITS];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int w = 0; w < 3; ++w) rec[3 * c + w] = cw[4 * c + w] | (((cw[4 * c + 3] >> w) & 0x11111111u) << 3);
+        for (int k = 0; k < BITS; ++k)
+          rec[BITS * c + k] = pack_word<BITS>(k, cw[4 * c], cw[4 * c + 1], cw[4 * c + 2], cw[4 * c + 3]);
       uint4* dst = reinterpret_cast<uint4*>(k_record(v, page, head, slot));
-      dst[0] = make_uint4(rec[0], rec[1], rec[2], rec[3]);
-      dst[1] = make_uint4(rec[4], rec[5], rec[6], rec[7]);
-      dst[2] = make_uint4(rec[8], rec[9], rec[10], rec[11]);
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) dst[i] = make_uint4(rec[4 * i], rec[4 * i + 1], rec[4 * i + 2], rec[4 * i + 3]);
     }
   } else {
     // V block (16 tokens = 16 consecutive lanes): token u = lane mod 16 owns nibbles j and
-    // j+4 of the words of chunks (g, tq, h), tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2); word w
-    // takes coordinates 32w + g + 8h, 32w + 16 + g + 8h and, as spare bits (bit w), 96 + g + 8h
-    // and 112 + g + 8h.  The four tokens of a quad (lanes u, u^1, u^8, u^9) OR their words
-    // together and member j stores the chunks of g = 2j, 2j+1 (24 contiguous bytes each).
+    // j+4 of the selector words of chunks (g, tq, h), tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2);
+    // nibble j of selector word w holds coordinate 32w + g + 8h and nibble j+4 coordinate
+    // 32w + 16 + g + 8h.  Packing keeps nibble positions, so the four tokens of a quad (lanes
+    // u, u^1, u^8, u^9) pack their own nibbles, OR the storage words together and member j
+    // stores the two chunks (h = 0, 1) of g = 2j, 2j+1 (2 BITS contiguous words each g).
     const unsigned lane = threadIdx.x & 31;
     const int u = lane & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
     uint32_t qmask = active ? ((0xFu << (4 * j)) | (0xFu << (16 + 4 * j))) : 0u;
@@ -161,33 +172,34 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     uint8_t* blk = v_block(v, qpage < 0 ? 0 : qpage, head, slot);
 #pragma unroll 1
     for (int g = 0; g < 8; ++g) {  // rolled: keeps the kernel's code small
-      uint32_t wd[6];
+      uint32_t wd[2 * BITS];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         // codes of coordinates 16m + g + 8h: nibble g of cw[2m + h]
-        uint32_t cm[8];
+        uint32_t sw[4];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) cm[m] = (cw[2 * m + h] >> (4 * g)) & 7u;
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t a = (cw[4 * w + h] >> (4 * g)) & 0xFu, c = (cw[4 * w + 2 + h] >> (4 * g)) & 0xFu;
+          sw[w] = active ? ((a << (4 * j)) | (c << (16 + 4 * j))) : 0u;
+        }
 #pragma unroll
-        for (int w = 0; w < 3; ++w) {
-          const uint32_t n0 = cm[2 * w] | (((cm[6] >> w) & 1u) << 3), n1 = cm[2 * w + 1] | (((cm[7] >> w) & 1u) << 3);
-          uint32_t part = active ? ((n0 << (4 * j)) | (n1 << (16 + 4 * j))) : 0u;
+        for (int k = 0; k < BITS; ++k) {
+          uint32_t part = pack_word<BITS>(k, sw[0], sw[1], sw[2], sw[3]);
           part |= __shfl_xor_sync(0xffffffffu, part, 1);
           part |= __shfl_xor_sync(0xffffffffu, part, 8);
-          wd[3 * h + w] = part;
+          wd[BITS * h + k] = part;
         }
       }
       if (j == (g >> 1) && qmask != 0u) {
-        uint32_t* dst = reinterpret_cast<uint32_t*>(blk + 24 * (4 * g + tq));
+        uint32_t* dst = reinterpret_cast<uint32_t*>(blk + 2 * chunk_bytes(BITS) * (4 * g + tq));
         if (qmask == 0xFFFFFFFFu) {
           uint2* d2 = reinterpret_cast<uint2*>(dst);
-          d2[0] = make_uint2(wd[0], wd[1]);
-          d2[1] = make_uint2(wd[2], wd[3]);
-          d2[2] = make_uint2(wd[4], wd[5]);
+#pragma unroll
+          for (int i = 0; i < BITS; ++i) d2[i] = make_uint2(wd[2 * i], wd[2 * i + 1]);
         } else {
           // tokens of this quad outside the launch keep their bits
 #pragma unroll
-          for (int i = 0; i < 6; ++i) {
+          for (int i = 0; i < 2 * BITS; ++i) {
             atomicAnd(reinterpret_cast<unsigned int*>(dst + i), ~qmask);
             atomicOr(reinterpret_cast<unsigned int*>(dst + i), wd[i]);
           }
@@ -201,6 +213,7 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
 
 // Small appends (decode steps): one warp per vector (see warp_encode_vector).
 constexpr int APP_WARPS = 4;
+template <int KB, int VB>
 __global__ void __launch_bounds__(APP_WARPS * 32)
 append_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __restrict__ v_src, int batch, int n_new,
               const int32_t* __restrict__ start_pos, const float* __restrict__ params_layer, KernelConsts kc) {
@@ -221,23 +234,53 @@ append_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
   const int page = resolve_page(v, b, pos);
   if (page < 0) return;
   float Mp[4][4];
-  fused_block_matrix(params_layer + ((size_t)head * NBLK + lane) * 8, Mp);
-  warp_encode_vector(v, src + (((size_t)b * n_new + i_new) * v.n_kv_heads + head) * D, head, side, page,
-                     pos % v.page_size, Mp, kc);
+  variant_block_matrix(v.rot, block_params(params_layer, v.rot, head, lane), Mp);
+  const __half* x = src + (((size_t)b * n_new + i_new) * v.n_kv_heads + head) * D;
+  if (side == 0)
+    warp_encode_vector<KB>(v, x, head, 0, page, pos % v.page_size, Mp, kc.k);
+  else
+    warp_encode_vector<VB>(v, x, head, 1, page, pos % v.page_size, Mp, kc.v);
+}
+
+template <int BITS>
+static int launch_bulk(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
+                       const int32_t* start_pos, const float* params_layer, const KernelConsts& kc, void* stream,
+                       int side0, int n_sides) {
+  dim3 grid((n_new + 15 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * n_sides, batch);
+  auto kern = v.rot == ROT_ISO ? encode_kernel<BITS, true> : encode_kernel<BITS, false>;
+  return (int)launch_pdl(kern, grid, dim3(ENC_THREADS), 0, (cudaStream_t)stream, v, (const __half*)k,
+                         (const __half*)vsrc, n_new, start_pos, params_layer, side0 == 0 ? kc.k : kc.v, side0, n_sides);
+}
+
+template <int KB, int VB>
+static int launch_encode_kv(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
+                            const int32_t* start_pos, const float* params_layer, const KernelConsts& kc, void* stream) {
+  const long vectors = (long)batch * n_new * v.n_kv_heads * 2;
+  if (n_new <= 8) {  // decode-style appends: latency matters, not throughput
+    const long blocks = (vectors + APP_WARPS - 1) / APP_WARPS;
+    return (int)launch_pdl(append_kernel<KB, VB>, dim3((unsigned)blocks), dim3(APP_WARPS * 32), 0,
+                           (cudaStream_t)stream, v, (const __half*)k, (const __half*)vsrc, batch, n_new, start_pos,
+                           params_layer, kc);
+  }
+  if (KB == VB) return launch_bulk<KB>(v, k, vsrc, batch, n_new, start_pos, params_layer, kc, stream, 0, 2);
+  int e = k ? launch_bulk<KB>(v, k, nullptr, batch, n_new, start_pos, params_layer, kc, stream, 0, 1) : 0;
+  if (e) return e;
+  return vsrc ? launch_bulk<VB>(v, nullptr, vsrc, batch, n_new, start_pos, params_layer, kc, stream, 1, 1) : 0;
 }
 
 int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
                   const int32_t* start_pos, const float* params_layer, const KernelConsts& kc, void* stream) {
   if (batch == 0 || n_new == 0) return 0;
-  const long vectors = (long)batch * n_new * v.n_kv_heads * 2;
-  if (n_new <= 8) {  // decode-style appends: latency matters, not throughput
-    const long blocks = (vectors + APP_WARPS - 1) / APP_WARPS;
-    return (int)launch_pdl(append_kernel, dim3((unsigned)blocks), dim3(APP_WARPS * 32), 0, (cudaStream_t)stream, v,
-                           (const __half*)k, (const __half*)vsrc, batch, n_new, start_pos, params_layer, kc);
-  }
-  dim3 grid((n_new + 15 + ENC_THREADS - 1) / ENC_THREADS, v.n_kv_heads * 2, batch);
-  return (int)launch_pdl(encode_kernel, grid, dim3(ENC_THREADS), 0, (cudaStream_t)stream, v, (const __half*)k,
-                         (const __half*)vsrc, n_new, start_pos, params_layer, kc);
+#define IQ_ENC(KB, VB) \
+  if (v.kb == KB && v.vb == VB) return launch_encode_kv<KB, VB>(v, k, vsrc, batch, n_new, start_pos, params_layer, kc, stream);
+  IQ_ENC(2, 2)
+  IQ_ENC(3, 2)
+  IQ_ENC(3, 3)
+  IQ_ENC(4, 2)
+  IQ_ENC(4, 3)
+  IQ_ENC(4, 4)
+#undef IQ_ENC
+  return (int)cudaErrorInvalidValue;
 }
 
 }  // namespace iq

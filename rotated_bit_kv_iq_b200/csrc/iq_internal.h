@@ -5,52 +5,83 @@
 
 #include "../../include/iq.h"
 
+#ifdef __CUDACC__
+#define IQ_HD __host__ __device__
+#else
+#define IQ_HD
+#endif
+
 namespace iq {
 
-constexpr int D = 128;          // head dimension
-constexpr int NBLK = 32;        // SO(4) blocks per head
-constexpr int K_REC = 48;       // bytes of a K record (one token)
+constexpr int D = 128;            // head dimension
+constexpr int NBLK = 32;          // 4-coordinate rotation blocks per head
 constexpr int V_BLK_TOKENS = 16;  // tokens per V block
-constexpr int V_BLK = 768;      // bytes of a V block (16 tokens x 128 codes x 3 bits)
-// Tile record: 32 consecutive slots of one (page, kv head), 3200 bytes:
-//   [0, 1536) 32 K records | [1536, 3072) 2 V blocks | [3072, 3136) 32 K norms | [3136, 3200) 32 V norms
-constexpr int TILE_TOKENS = 32;
-constexpr int TR_K = 0;
-constexpr int TR_V = TR_K + TILE_TOKENS * K_REC;
-constexpr int TR_KN = TR_V + 2 * V_BLK;
-constexpr int TR_VN = TR_KN + TILE_TOKENS * 2;
-constexpr int TILE_BYTES = TR_VN + TILE_TOKENS * 2;
-static_assert(TILE_BYTES == 3200, "tile record size");
+constexpr int TILE_TOKENS = 32;   // slots per tile record
 
-// Lloyd-Max quantiser of N(0,1): 8 ascending levels, 7 midpoint boundaries (double).
+// Record geometry for a code width of `bits` (2, 3 or 4) per coordinate.  A chunk holds 32
+// codes in `bits` 32-bit words; a K record is four chunks (one token); a V block is 64 chunks
+// (16 tokens).  Tile record of 32 consecutive slots of one (page, kv head) with K width kb and
+// V width vb:
+//   [0, tr_v)        32 K records
+//   [tr_v, tr_kn)    2 V blocks
+//   [tr_kn, tr_vn)   32 K norms (binary16)
+//   [tr_vn, +64)     32 V norms (binary16)
+IQ_HD constexpr int chunk_bytes(int bits) { return 4 * bits; }
+IQ_HD constexpr int k_rec_bytes(int bits) { return 16 * bits; }
+IQ_HD constexpr int v_blk_bytes(int bits) { return 256 * bits; }
+IQ_HD constexpr int tr_v(int kb) { return TILE_TOKENS * k_rec_bytes(kb); }
+IQ_HD constexpr int tr_kn(int kb, int vb) { return tr_v(kb) + 2 * v_blk_bytes(vb); }
+IQ_HD constexpr int tr_vn(int kb, int vb) { return tr_kn(kb, vb) + 2 * TILE_TOKENS; }
+IQ_HD constexpr int tile_bytes(int kb, int vb) { return tr_vn(kb, vb) + 2 * TILE_TOKENS; }
+static_assert(tile_bytes(3, 3) == 3200, "tile record size of the 3-bit format");
+
+// The (K, V) code widths the kernels are built for (K never narrower than V).
+IQ_HD constexpr bool supported_widths(int kb, int vb) {
+  return (kb == 2 && vb == 2) || (kb == 3 && (vb == 2 || vb == 3)) || (kb == 4 && vb >= 2 && vb <= 4);
+}
+
+// Rotation variants (iq_rotation): WHT + quaternion pairs, one quaternion per block, Givens pairs.
+constexpr int ROT_ISO = 0, ROT_QUAT = 1, ROT_PLANAR = 2;
+IQ_HD constexpr int params_per_head(int rot) { return rot == ROT_ISO ? 256 : 128; }
+IQ_HD constexpr int params_per_block(int rot) { return rot == ROT_ISO ? 8 : 4; }
+
+// Lloyd-Max quantiser of N(0,1) with 2^bits ascending levels and midpoint boundaries (double).
 struct Codebook {
-  double level[8];
-  double bound[7];
+  int bits;
+  double level[16];
+  double bound[15];
 };
-Codebook compute_codebook();
+Codebook compute_codebook(int bits);
 
-// Seeded rotation parameters, [L][Hkv][32][2][4] float32, written to `out` (host).
-void init_rotation_params(uint64_t seed, int n_layers, int n_kv_heads, float* out);
+// Seeded rotation parameters, [L][Hkv][params_per_head(rot)] float32, written to `out` (host).
+void init_rotation_params(uint64_t seed, int rot, int n_layers, int n_kv_heads, float* out);
 
-// Constants handed to kernels by value.  The eight centroids reach the tensor cores as
-// int8 pairs: alpha8 * c_k = hi_k + lo_k / 254 (hi_k, lo_k in [-127, 127]).
+// Constants of one side's (K or V) codebook handed to kernels by value.  The levels reach the
+// tensor cores as int8 pairs: alpha8 * c_k = hi_k + lo_k / 254 (hi_k, lo_k in [-127, 127]);
+// byte k of the little-endian words lut_hi / lut_lo is entry k (2^bits entries).
+struct SideConsts {
+  float bound_pos[7];  // positive N(0,1) boundaries, ascending (the middle boundary is 0)
+  uint32_t lut_hi[4];
+  uint32_t lut_lo[4];
+  float alpha8;
+  int bits;
+};
 struct KernelConsts {
-  float bound_pos[3];    // positive N(0,1) boundaries b4, b5, b6 (b3 = 0)
-  uint32_t lut_hi[2];    // bytes hi_k, k = 0..3 in the first word, 4..7 in the second
-  uint32_t lut_lo[2];    // bytes lo_k
-  float alpha8;          // the int8 scale
+  SideConsts k, v;
 };
-const KernelConsts& kernel_consts();
+const KernelConsts& kernel_consts(int kb, int vb);
 
 // Device geometry of one layer's pools, resolved on the host.
 struct LayerView {
-  uint8_t* pool;         // layer base of the tile-record pool
+  uint8_t* pool;               // layer base of the tile-record pool
   const int32_t* block_table;  // NULL -> sequence b uses page b
-  int32_t max_pages;     // pages per sequence in the block table (1 when table is NULL)
+  int32_t max_pages;           // pages per sequence in the block table (1 when table is NULL)
   int32_t page_size;
   int32_t n_pages;
   int32_t n_kv_heads;
   uint32_t* status;
+  int32_t kb, vb;              // K and V code widths
+  int32_t rot;                 // rotation variant
 };
 
 // Kernel launchers (defined in the .cu files); return the launch error.
@@ -64,7 +95,7 @@ int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void*
                        int n_q_heads, const int32_t* ctx_len, int max_ctx, const float* params_layer, float* out,
                        void* workspace, const KernelConsts& kc, void* stream);
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
-                  uint16_t* norms, const KernelConsts& kc, void* stream);
+                  uint16_t* norms, void* stream);
 
 // Decode grid (host): CTAs of one decode launch on the current device, given how many CTAs of
 // the kernel an SM holds at once.

@@ -9,10 +9,10 @@ from rotated_bit_kv_iq_b200 import inputs
 TILE = 32
 
 
-def oracle_params(seed, n_layers, n_kv_heads):
+def oracle_params(seed, n_layers, n_kv_heads, variant="iso"):
     """Rotation parameters drawn by the oracle's own generator (the product's generator is
     checked against it bit for bit in the host tests; the oracle never uses the product's)."""
-    return rotation.init_rotation(seed, n_layers, n_kv_heads)
+    return rotation.init_rotation(seed, n_layers, n_kv_heads, variant)
 
 
 def oracle_encode_stream(params_head, layer, head, which, t0, n, n_outliers=4, heavy_frac=0.0, seed=inputs.DATA_SEED):
@@ -21,36 +21,39 @@ def oracle_encode_stream(params_head, layer, head, which, t0, n, n_outliers=4, h
     return x, encode.encode(x, params_head)
 
 
-def tile_records(k_codes, k_n16, v_codes, v_n16):
-    """Oracle-packed tile records of tokens 0..T-1 of one (sequence, kv head): (ceil(T/32), 3200)
-    uint8; slots past T are zero."""
+def tile_records(k_codes, k_n16, v_codes, v_n16, k_bits=3, v_bits=3):
+    """Oracle-packed tile records of tokens 0..T-1 of one (sequence, kv head):
+    (ceil(T/32), tile bytes) uint8; slots past T are zero."""
     T = k_codes.shape[0]
     nt = (T + TILE - 1) // TILE
-    krec = np.zeros((nt * TILE, 48), np.uint8)
-    krec[:T] = packing.pack_k_fast(k_codes)
-    vrec = np.zeros((nt * 2, 768), np.uint8)
-    vb = packing.pack_v_fast(v_codes)
+    kr, vbk = packing.k_record_bytes(k_bits), packing.v_block_bytes(v_bits)
+    krec = np.zeros((nt * TILE, kr), np.uint8)
+    krec[:T] = packing.pack_k_fast(k_codes, k_bits)
+    vrec = np.zeros((nt * 2, vbk), np.uint8)
+    vb = packing.pack_v_fast(v_codes, v_bits)
     vrec[:vb.shape[0]] = vb
     kn = np.zeros(nt * TILE, np.uint16)
     vn = np.zeros(nt * TILE, np.uint16)
     kn[:T] = k_n16
     vn[:T] = v_n16
-    rec = np.concatenate([krec.reshape(nt, TILE * 48), vrec.reshape(nt, 2 * 768),
+    rec = np.concatenate([krec.reshape(nt, TILE * kr), vrec.reshape(nt, 2 * vbk),
                           kn.reshape(nt, TILE).view(np.uint8), vn.reshape(nt, TILE).view(np.uint8)], axis=1)
-    assert rec.shape[1] == 3200
+    assert rec.shape[1] == TILE * kr + 2 * vbk + 128
     return rec
 
 
 def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n16):
     """Write oracle-packed records of tokens 0..T-1 of one sequence/head into the device pool
-    (one host-to-device copy).  seq_pages: physical page ids of the sequence, in order."""
+    (one host-to-device copy) in the cache's code widths.  seq_pages: physical page ids of the
+    sequence, in order."""
     import torch
 
     ps = cache.page_size
     T = k_codes.shape[0]
     if T == 0:
         return
-    rec = torch.from_numpy(tile_records(k_codes, k_n16, v_codes, v_n16)).to(cache.pool.device)
+    kb, vb = cache.k_bits, cache.v_bits
+    rec = torch.from_numpy(tile_records(k_codes, k_n16, v_codes, v_n16, kb, vb)).to(cache.pool.device)
     nt = rec.shape[0]
     t0 = np.arange(nt) * TILE
     pages = torch.as_tensor(np.asarray(seq_pages)[t0 // ps].astype(np.int64), device=cache.pool.device)
@@ -64,11 +67,14 @@ def upload_sequence(cache, layer, seq_pages, head, k_codes, k_n16, v_codes, v_n1
         m = T - full * TILE
         last = tv[layer, pages[full], head, tiles[full]].clone()
         r = rec[full]
-        last[:48 * m] = r[:48 * m]
-        nb = (m + 15) // 16
-        last[1536:1536 + 768 * nb] = r[1536:1536 + 768 * nb]
-        last[3072:3072 + 2 * m] = r[3072:3072 + 2 * m]
-        last[3136:3136 + 2 * m] = r[3136:3136 + 2 * m]
+        kr, vbk = packing.k_record_bytes(kb), packing.v_block_bytes(vb)
+        kv0 = TILE * kr
+        kn0 = kv0 + 2 * vbk
+        last[:kr * m] = r[:kr * m]
+        nblk = (m + 15) // 16
+        last[kv0:kv0 + vbk * nblk] = r[kv0:kv0 + vbk * nblk]
+        last[kn0:kn0 + 2 * m] = r[kn0:kn0 + 2 * m]
+        last[kn0 + 64:kn0 + 64 + 2 * m] = r[kn0 + 64:kn0 + 64 + 2 * m]
         tv[layer, pages[full], head, tiles[full]] = last
 
 

@@ -27,7 +27,8 @@ def test_library_exports_every_declared_symbol(lib):
     hdr = open(os.path.join(ROOT, "include", "iq.h")).read()
     names = set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(iq_\w+)\s*\(", hdr, flags=re.M))
     assert {"iq_init_rotation", "iq_encode_append", "iq_decode_attention", "iq_decode_workspace_size",
-            "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version", "iq_decode_step"} <= names
+            "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version", "iq_decode_step",
+            "iq_init_rotation_variant", "iq_rotation_params_per_head"} <= names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -49,11 +50,28 @@ def test_init_rotation_is_bit_identical_to_oracle(lib):
     np.testing.assert_array_equal(got.view(np.uint32), rotation.init_rotation(0xDEADBEEFCAFEF00D, 2, 3).view(np.uint32))
 
 
+@pytest.mark.parametrize("variant", ["quat", "planar"])
+def test_variant_params_are_bit_identical_to_oracle(lib, variant):
+    got = B.iq_init_rotation_variant(3, variant, 2, 3)
+    want = rotation.init_rotation(3, 2, 3, variant)
+    assert got.shape == want.shape and got.dtype == np.float32
+    np.testing.assert_array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert B.iq_rotation_params_per_head(B.ROTATIONS[variant]) == 128
+    assert B.iq_rotation_params_per_head(0) == 256 and B.iq_rotation_params_per_head(3) == 0
+    iso = B.iq_init_rotation_variant(1, "iso", 1, 2)
+    np.testing.assert_array_equal(iso.view(np.uint32), B.iq_init_rotation(1, 1, 2).view(np.uint32))
+    assert B.lib().iq_init_rotation_variant(1, 7, 1, 1, got.ctypes.data_as(ctypes.c_void_p)) == B.IQ_ERR_UNSUPPORTED
+
+
 def test_cache_bytes_and_workspace(lib):
     pb = B.iq_cache_bytes(2, 4, 64, 10)
     assert pb == 2 * 4 * 64 * 10 * 100  # 48 + 48 code bytes and 2 + 2 norm bytes per slot and kv head
+    for kb, vb in B.WIDTHS:  # 16 (kb + vb) code bytes and 4 norm bytes per slot and kv head
+        assert B.iq_cache_bytes(1, 2, 64, 3, kb, vb) == 2 * 64 * 3 * (16 * (kb + vb) + 4)
     with pytest.raises(B.IqError):
         B.iq_cache_bytes(1, 1, 48, 1)  # page size not a multiple of 32
+    with pytest.raises(B.IqError):
+        B.iq_cache_bytes(1, 1, 64, 1, 2, 3)  # V wider than K: not built
     w1 = B.iq_decode_workspace_size(1, 32, 4, 32768)
     w2 = B.iq_decode_workspace_size(2, 32, 4, 32768)
     assert 0 < w1 <= w2
@@ -101,6 +119,13 @@ def test_encode_rejects_bad_arguments(lib):
     assert _enc(_fake_cache(), batch=5) == B.IQ_ERR_CAPACITY           # more sequences than pages
     assert _enc(_fake_cache(), n_new=-1) == B.IQ_ERR_INVALID_ARG
     assert _enc(_fake_cache(block_table_dev=0xB0000, max_pages_per_seq=0)) == B.IQ_ERR_INVALID_ARG
+
+
+@cpu_only
+def test_calls_reject_unsupported_formats(lib):
+    for kw in (dict(k_bits=5), dict(k_bits=2, v_bits=3), dict(v_bits=1), dict(rotation=3), dict(rotation=-1)):
+        assert _enc(_fake_cache(**kw)) == B.IQ_ERR_UNSUPPORTED, kw
+        assert _dec(_fake_cache(**kw)) == B.IQ_ERR_UNSUPPORTED, kw
 
 
 @cpu_only
