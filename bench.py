@@ -318,6 +318,70 @@ def bench_encode(steps, warmup, device, stream):
             "bytes_per_launch": T * Hkv * 2 * BYTES_PER_VECTOR_ENCODE}
 
 
+def bench_prefill(steps, warmup, device, stream, world=1):
+    """Chunked prefill of one Llama-3.1-8B-shaped layer (32 q / 8 kv heads): an 8192-token prompt
+    in 16 chunks of 512; each chunk appends its K/V (iq_encode_append) and attends causally over the
+    packed cache (iq_prefill_attention).  The 48 launches of a step are replayed as one CUDA graph."""
+    import torch
+
+    from rotated_bit_kv_iq_b200 import binding as Bd
+    from rotated_bit_kv_iq_b200 import inputs
+
+    Hq, Hkv, T, C = 32, 8, 8192, 512
+    cache = Bd.PagedCache(1, Hkv, T, 1, device=device)
+    params = torch.from_numpy(Bd.iq_init_rotation(inputs.ROTATION_SEED, 1, Hkv)).to(device)
+    K = inputs.kv_tokens_device(0, 0, Hkv, 0, T, device=device).view(1, T, Hkv, 128)
+    V = inputs.kv_tokens_device(0, 0, Hkv, 1, T, device=device).view(1, T, Hkv, 128)
+    g = inputs._torch_gen(device, 0, 8)
+    q = torch.randn((1, T, Hq, 128), generator=g, device=device).to(torch.float16)
+    out = torch.empty((1, T, Hq, 128), dtype=torch.float32, device=device)
+    ws = torch.empty(Bd.iq_prefill_workspace_size(1, C, Hkv, T), dtype=torch.uint8, device=device)
+    starts = [torch.full((1,), c, dtype=torch.int32, device=device) for c in range(0, T, C)]
+    chunks = [(K[:, c:c + C].contiguous(), V[:, c:c + C].contiguous(), q[:, c:c + C].contiguous()) for c in range(0, T, C)]
+    outs = [torch.empty((1, C, Hq, 128), dtype=torch.float32, device=device) for _ in chunks]
+
+    def step():
+        for (k, v, qq), st, o in zip(chunks, starts, outs):
+            Bd.iq_encode_append(cache, 0, k, v, st, params, stream)
+            Bd.iq_prefill_attention(cache, 0, qq, st, T, params, o, ws, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(warmup):
+            graph.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, device)
+    del graph
+    # algorithmic attention work: query token at position p reads p + 1 keys; 2 flops per
+    # multiply-add, 2 x 128 multiply-adds per (query head, key) for scores and values
+    flops = sum(p + 1 for p in range(T)) * Hq * 4 * 128
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        peak_kind = "measured bf16 x 2 (nominal int8 / bf16 ratio)"
+    except Exception:
+        bf16, peak_kind = 1590.0, "fallback bf16 x 2 (nominal int8 / bf16 ratio)"
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"workload": "llama8b_prefill_8k: one layer, 32 q / 8 kv heads, 8192-token prompt in 16 chunks of 512 "
+                        "(append + causal attention over the packed cache per chunk)",
+            "value": world * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": 2 * bf16, "unit": "TFLOP/s",
+                         "frac": ach / (2 * bf16), "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "whole prefill step (encode + prefill attention + merge), algorithmic flops"},
+            "launches": 48 * steps}
+
+
 def max_over_ranks(x, device=None):
     """Max of a float over the ranks of the default process group (x itself without one).
     Every timed quantity of a multi-rank run goes through this, so that the job's time is
@@ -558,7 +622,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed step's output")
     ap.add_argument("--layers", type=int, default=0, help="override the stack depth (profiling runs)")
-    ap.add_argument("--only", default="", choices=["", "serving", "encode"],
+    ap.add_argument("--only", default="", choices=["", "serving", "encode", "prefill"],
                     help="run one secondary workload alone (profiling runs); no headline line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -592,6 +656,8 @@ def main():
     if args.only:
         if args.only == "serving":
             res = bench_serving(args.steps, args.warmup, dev, stream, seed=rank, world=world, n_layers=args.layers)
+        elif args.only == "prefill":
+            res = bench_prefill(args.steps, args.warmup, dev, stream, world=world)
         else:
             res = bench_encode(args.steps, args.warmup, dev, stream)
         if rank == 0:
@@ -673,6 +739,10 @@ def main():
                          "traffic": None, "kernel": "encode (one layer, K and V)", "peak_kind": peak_kind},
         }
         result["gpu_launches"] += 32 * args.steps
+        torch.cuda.empty_cache()
+        pre = bench_prefill(args.steps, args.warmup, dev, stream, world=world)
+        result["prefill"] = pre
+        result["gpu_launches"] += pre["launches"]
         torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -235,6 +235,33 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
                          const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
                          void* workspace_dev, size_t workspace_bytes, iq_stream_t stream);
 
+/* Workspace bytes iq_prefill_attention needs for these sizes on the current device (per query
+ * block of 8 tokens, kv head and split of the context: the split partials).  Needs no zeroing. */
+size_t iq_prefill_workspace_size(int32_t batch, int32_t n_tokens, int32_t n_kv_heads, int32_t max_ctx);
+
+/* Chunked-prefill attention over the packed cache of layer `layer`: n_tokens query tokens per
+ * sequence, causal.  Defined by: "RotaryQuant" (rebasdaily.com), section
+ * "妙处不只是压缩，而是不再展开" (attention on the packed tensors), applied to a chunk of prompt
+ * tokens; "RotorQuant" (sd114.wiki), section "性能基准", and "压缩与速度的博弈" (zhichai.net),
+ * section "宣称的数字", report prefill speed over such caches.
+ *   q_dev        : [batch][n_tokens][n_q_heads][128], fp16 (IQ_F16) or fp32 (IQ_F32).
+ *   start_pos_dev: int32 [batch]; query token i of sequence b is at position start_pos[b] + i and
+ *                  attends to positions 0 .. start_pos[b] + i of the cache, which must hold them
+ *                  (append the chunk's K/V with iq_encode_append first).  Values outside
+ *                  [0, max_ctx - n_tokens] are clamped into range and flagged with IQ_DEVERR_CTX.
+ *   max_ctx      : host upper bound on start_pos + n_tokens (sizes the split of the work); must
+ *                  not exceed the per-sequence capacity.
+ *   out_dev      : float32 [batch][n_tokens][n_q_heads][128].
+ *   workspace_dev: at least iq_prefill_workspace_size(...) bytes, 256-byte aligned.
+ * Each block of 8 query tokens shares every tile of packed K/V it loads (one warp per query
+ * token, tensor-core tiles as in decode); the result equals iq_decode_attention of each query
+ * token over its own causal context.  Two kernels (attention splits, then their merge with the
+ * inverse rotation); they wait for the preceding kernel on the stream before reading anything. */
+iq_status iq_prefill_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype, int32_t batch,
+                               int32_t n_tokens, int32_t n_q_heads, const int32_t* start_pos_dev, int32_t max_ctx,
+                               const float* params_dev, float* out_dev, void* workspace_dev, size_t workspace_bytes,
+                               iq_stream_t stream);
+
 /* Size of the fixed device scratch used by iq_decode_attention_noalloc (per device). */
 #define IQ_NOALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -89,3 +89,18 @@ def attention_rotated(q, k_codes, k_norm16, v_codes, v_norm16, params, bits=3, v
             acc = (p * nv) @ Cv  # accumulate values in the rotated basis
             out[h] = rotate_inverse(acc / p.sum(), params[kv], variant)  # one inverse rotation per output
     return out
+
+
+def prefill_attention(q, k_codes, k_norm16, v_codes, v_norm16, params, start, bits=3, v_bits=None, variant="iso"):
+    """Chunked prefill on the packed cache: q (n_tok, Hq, 128) are the queries of tokens at
+    positions start .. start + n_tok - 1 of one sequence; query token i attends to cache
+    positions 0 .. start + i (causal).  k_codes etc. hold at least start + n_tok positions.
+    Each query token is one decode-attention problem over its own prefix.  Returns
+    (n_tok, Hq, 128) fp64."""
+    q = np.asarray(q, dtype=np.float64)
+    out = np.zeros(q.shape)
+    for i in range(q.shape[0]):
+        T = start + i + 1
+        out[i] = attention_rotated(q[i], k_codes[:, :T], k_norm16[:, :T], v_codes[:, :T], v_norm16[:, :T], params,
+                                   bits, v_bits, variant)
+    return out

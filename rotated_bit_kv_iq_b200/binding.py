@@ -113,6 +113,10 @@ def lib():
         L.iq_decode_step.argtypes = [P, i32, vp, ctypes.c_int, vp, vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_decode_attention_noalloc.restype = ctypes.c_int
         L.iq_decode_attention_noalloc.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp]
+        L.iq_prefill_workspace_size.restype = sz
+        L.iq_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.iq_prefill_attention.restype = ctypes.c_int
+        L.iq_prefill_attention.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_export_codes.restype = ctypes.c_int
         L.iq_export_codes.argtypes = [P, i32, i32, i32, i32, i32, vp, vp, vp]
         _lib = L
@@ -211,6 +215,22 @@ def iq_decode_step(cache, layer, q, k_new, v_new, ctx_len, max_ctx, params, out,
         ctypes.byref(cache.c), layer, _ptr(q), dtype, _ptr(k_new), _ptr(v_new), int(q.shape[0]), int(q.shape[1]),
         _ptr(ctx_len), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace),
         int(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def iq_prefill_workspace_size(batch, n_tokens, n_kv_heads, max_ctx):
+    return int(lib().iq_prefill_workspace_size(batch, n_tokens, n_kv_heads, max_ctx))
+
+
+def iq_prefill_attention(cache, layer, q, start_pos, max_ctx, params, out, workspace, stream=None):
+    """q: [batch][n_tokens][Hq][128] fp16|fp32; out: fp32 of the same shape; query token i of sequence b
+    at position start_pos[b] + i attends causally to the cache's positions 0 .. start_pos[b] + i."""
+    import torch
+
+    dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
+    ws_bytes = 0 if workspace is None else int(workspace.numel() * workspace.element_size())
+    _check("iq_prefill_attention", lib().iq_prefill_attention(
+        ctypes.byref(cache.c), layer, _ptr(q), dtype, int(q.shape[0]), int(q.shape[1]), int(q.shape[2]),
+        _ptr(start_pos), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 IQ_NOALLOC_SCRATCH_BYTES = 4 << 20

@@ -246,6 +246,39 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 
+size_t iq_prefill_workspace_size(int32_t batch, int32_t n_tokens, int32_t n_kv_heads, int32_t max_ctx) {
+  if (batch < 0 || n_tokens < 0 || n_kv_heads < 1 || max_ctx < 0) return 0;
+  return prefill_workspace_bytes(batch, n_tokens, n_kv_heads, max_ctx);
+}
+
+iq_status iq_prefill_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype, int32_t batch,
+                               int32_t n_tokens, int32_t n_q_heads, const int32_t* start_pos_dev, int32_t max_ctx,
+                               const float* params_dev, float* out_dev, void* workspace_dev, size_t workspace_bytes,
+                               iq_stream_t stream) {
+  iq_status st = check_cache(cache, layer);
+  if (st != IQ_OK) return st;
+  if (batch < 0 || n_tokens < 0 || n_q_heads < 1 || max_ctx < n_tokens || !q_dev || !start_pos_dev || !params_dev ||
+      !out_dev)
+    return IQ_ERR_INVALID_ARG;
+  if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
+  if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
+  const int G = n_q_heads / cache->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
+  if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
+  if ((int64_t)batch * cache->n_kv_heads * ((n_tokens + 7) / 8) > (int64_t)1 << 24) return IQ_ERR_UNSUPPORTED;
+  if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(start_pos_dev, 4))
+    return IQ_ERR_ALIGNMENT;
+  const size_t need = prefill_workspace_bytes(batch, n_tokens, cache->n_kv_heads, max_ctx);
+  if (batch > 0 && n_tokens > 0 && (!workspace_dev || workspace_bytes < need)) return IQ_ERR_WORKSPACE;
+  if (workspace_dev && !aligned(workspace_dev, 256)) return IQ_ERR_ALIGNMENT;
+  const LayerView v = view(cache, layer);
+  const int e = launch_prefill(v, q_dev, q_dtype == IQ_F32, batch, n_tokens, n_q_heads, start_pos_dev, max_ctx,
+                               layer_params(cache, params_dev, layer), out_dev, workspace_dev,
+                               kernel_consts(v.kb, v.vb), stream);
+  return e ? IQ_ERR_CUDA : IQ_OK;
+}
+
 iq_status iq_export_codes(const iq_cache* cache, int32_t layer, int32_t kv, int32_t seq, int32_t t0, int32_t n,
                           uint8_t* codes_dev, uint16_t* norms_dev, iq_stream_t stream) {
   iq_status st = check_cache(cache, layer);

@@ -8,7 +8,7 @@
 #include <mutex>
 #include <tuple>
 
-#include "iq_decode_impl.cuh"
+#include "iq_prefill_impl.cuh"
 
 namespace iq {
 
@@ -81,6 +81,11 @@ Workspace carve_workspace(void* ws, int batch, int n_kv_heads) {
                                                const void*, const void*);
 IQ_DECODE_WIDTHS(IQ_DECL)
 #undef IQ_DECL
+#define IQ_DECL(KB, VB)                                                                                         \
+  extern template int launch_prefill_kv<KB, VB>(const LayerView&, const void*, int, int, int, int, const int32_t*, \
+                                                int, const float*, float*, void*, const KernelConsts&, void*, int);
+IQ_DECODE_WIDTHS(IQ_DECL)
+#undef IQ_DECL
 
 static int dispatch(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads, const int32_t* ctx_len,
                     int max_ctx, const float* params_layer, float* out, void* workspace, const KernelConsts& kc,
@@ -106,6 +111,27 @@ int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void*
                        void* workspace, const KernelConsts& kc, void* stream) {
   return dispatch(v, q, q_f32, batch, n_q_heads, ctx_len, max_ctx, params_layer, out, workspace, kc, stream, k_new,
                   v_new);
+}
+
+// Prefill workspace: per (group, split, query token, head) one (m, l) pair and one 128-float O.
+size_t prefill_workspace_bytes(int batch, int n_tok, int n_kv_heads, int max_ctx) {
+  const int n_qblk = (n_tok + PF_QB - 1) / PF_QB;
+  const int groups = batch * n_kv_heads * n_qblk;
+  const int splits = prefill_splits(groups, (max_ctx + TT - 1) / TT, sm_count());
+  const size_t rows = (size_t)groups * splits * PF_QB * HMAX;
+  return align256(rows * sizeof(float2)) + align256(rows * D * sizeof(float));
+}
+
+int launch_prefill(const LayerView& v, const void* q, int q_f32, int batch, int n_tok, int n_q_heads,
+                   const int32_t* start, int max_ctx, const float* params_layer, float* out, void* workspace,
+                   const KernelConsts& kc, void* stream) {
+#define IQ_CASE(KB, VB)                                                                                        \
+  if (v.kb == KB && v.vb == VB)                                                                               \
+    return launch_prefill_kv<KB, VB>(v, q, q_f32, batch, n_tok, n_q_heads, start, max_ctx, params_layer, out, \
+                                     workspace, kc, stream, sm_count());
+  IQ_DECODE_WIDTHS(IQ_CASE)
+#undef IQ_CASE
+  return (int)cudaErrorInvalidValue;
 }
 
 }  // namespace iq

@@ -441,25 +441,24 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
 // P4: head h < 4 fills the fragment rows of lanes g = h (hi, with lo2 as row g + 8) and
 // g = h + 4 (lo, row g + 8 zero); see process_tile.
 template <bool P4>
-__device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, int h, const float* prm,
-                                             uint32_t* qfrag, float* kappa) {
+__device__ __forceinline__ void rotate_query_row(const void* q, int q_f32, size_t row0, bool live, int rot, float alpha_k,
+                                                 int h, const float* prm, uint32_t* qfrag, float* kappa) {
   const int lane = threadIdx.x & 31;
   float x[4] = {0.f, 0.f, 0.f, 0.f};
-  const bool live = h < a.g_real;
   if (live) {
-    const size_t row = ((size_t)b * a.n_q_heads + (size_t)kvh * a.g_real + h) * D + 4 * lane;
-    if (a.q_f32) {
-      const float4 f = *reinterpret_cast<const float4*>((const float*)a.q + row);
+    const size_t row = row0 + 4 * lane;
+    if (q_f32) {
+      const float4 f = *reinterpret_cast<const float4*>((const float*)q + row);
       x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
     } else {
-      const uint2 u = *reinterpret_cast<const uint2*>((const __half*)a.q + row);
+      const uint2 u = *reinterpret_cast<const uint2*>((const __half*)q + row);
       const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
       const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
       x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
     }
     float Mp[4][4];
-    variant_block_matrix(a.v.rot, prm + lane * params_per_block(a.v.rot), Mp);
-    warp_rotate_forward(x, Mp, a.v.rot == ROT_ISO);
+    variant_block_matrix(rot, prm + lane * params_per_block(rot), Mp);
+    warp_rotate_forward(x, Mp, rot == ROT_ISO);
   }
   float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
@@ -489,7 +488,14 @@ __device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, i
     row[4 * cc + 2 * e + 1] = pack4(lo[0], lo[1], lo[2], lo[3]);
     row[16 + 2 * cc + e] = pack4(lo2[0], lo2[1], lo2[2], lo2[3]);
   }
-  if (lane == 0) kappa[h] = live ? kLog2e / (128.f * gam * a.kc.k.alpha8) : 0.f;
+  if (lane == 0) kappa[h] = live ? kLog2e / (128.f * gam * alpha_k) : 0.f;
+}
+
+template <bool P4>
+__device__ __forceinline__ void rotate_query(const DecArgs& a, int b, int kvh, int h, const float* prm,
+                                             uint32_t* qfrag, float* kappa) {
+  rotate_query_row<P4>(a.q, a.q_f32, ((size_t)b * a.n_q_heads + (size_t)kvh * a.g_real + h) * D, h < a.g_real, a.v.rot,
+                       a.kc.k.alpha8, h, prm, qfrag, kappa);
 }
 
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {

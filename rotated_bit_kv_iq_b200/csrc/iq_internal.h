@@ -94,6 +94,10 @@ int launch_decode(const LayerView& v, const void* q, int q_f32, int batch, int n
 int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void* k_new, const void* v_new, int batch,
                        int n_q_heads, const int32_t* ctx_len, int max_ctx, const float* params_layer, float* out,
                        void* workspace, const KernelConsts& kc, void* stream);
+int launch_prefill(const LayerView& v, const void* q, int q_f32, int batch, int n_tok, int n_q_heads,
+                   const int32_t* start, int max_ctx, const float* params_layer, float* out, void* workspace,
+                   const KernelConsts& kc, void* stream);
+size_t prefill_workspace_bytes(int batch, int n_tok, int n_kv_heads, int max_ctx);
 int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* codes,
                   uint16_t* norms, void* stream);
 

@@ -28,7 +28,8 @@ def test_library_exports_every_declared_symbol(lib):
     names = set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(iq_\w+)\s*\(", hdr, flags=re.M))
     assert {"iq_init_rotation", "iq_encode_append", "iq_decode_attention", "iq_decode_workspace_size",
             "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version", "iq_decode_step",
-            "iq_init_rotation_variant", "iq_rotation_params_per_head"} <= names
+            "iq_init_rotation_variant", "iq_rotation_params_per_head", "iq_prefill_attention",
+            "iq_prefill_workspace_size"} <= names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -162,6 +163,28 @@ def test_decode_step_rejects_bad_arguments(lib):
     assert step(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED
     assert step(_fake_cache(), ws_bytes=8) == B.IQ_ERR_WORKSPACE
     assert step(_fake_cache(head_dim=64)) == B.IQ_ERR_UNSUPPORTED
+
+
+@cpu_only
+def test_prefill_rejects_bad_arguments(lib):
+    f = B.lib().iq_prefill_attention
+
+    def pre(c, q=0x50000, dtype=0, batch=1, n_tok=8, hq=8, start=0x70000, max_ctx=32, ws=0xA0000, ws_bytes=1 << 30):
+        return f(ctypes.byref(c), 0, q, dtype, batch, n_tok, hq, start, max_ctx, 0x80000, 0x90000, ws, ws_bytes, None)
+
+    assert pre(_fake_cache(), n_tok=40) == B.IQ_ERR_INVALID_ARG      # max_ctx below the chunk
+    assert pre(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
+    assert pre(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert pre(_fake_cache(), hq=5) == B.IQ_ERR_INVALID_ARG
+    assert pre(_fake_cache(), dtype=3) == B.IQ_ERR_UNSUPPORTED
+    assert pre(_fake_cache(), start=None) == B.IQ_ERR_INVALID_ARG
+    assert pre(_fake_cache(), q=0x50004) == B.IQ_ERR_ALIGNMENT
+    assert pre(_fake_cache(), ws=None) == B.IQ_ERR_WORKSPACE
+    assert pre(_fake_cache(), ws_bytes=64) == B.IQ_ERR_WORKSPACE
+    assert pre(_fake_cache(), ws=0xA0040) == B.IQ_ERR_ALIGNMENT
+    assert pre(_fake_cache(k_bits=5)) == B.IQ_ERR_UNSUPPORTED
+    assert pre(_fake_cache(), batch=5) == B.IQ_ERR_CAPACITY
+    assert B.iq_prefill_workspace_size(1, 512, 8, 8192) > 0
 
 
 @cpu_only

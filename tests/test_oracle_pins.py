@@ -591,3 +591,29 @@ def test_planted_variant_mistakes_are_caught():
     q = rotation.unit_params(Pq)
     right = rotation.quat_mul(x.reshape(32, 4), q).reshape(128)
     assert np.abs(right - rotation.rotate(x, Pq, "quat")).max() > 1e-3
+
+
+def test_prefill_attention_is_causal_sdpa():
+    """The oracle's chunked prefill equals torch SDPA (fp64) on the dequantised cache with an
+    explicit causal mask (query i of the chunk sees keys 0 .. start + i)."""
+    rng = np.random.default_rng(31)
+    Hkv, G, start, C = 2, 3, 11, 7
+    T = start + C
+    P = rotation.init_rotation(1, 1, Hkv)[0]
+    kc = rng.integers(0, 8, (Hkv, T, 128)).astype(np.uint8)
+    vc = rng.integers(0, 8, (Hkv, T, 128)).astype(np.uint8)
+    kn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 40, (Hkv, T)))
+    vn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 10, (Hkv, T)))
+    q = rng.standard_normal((C, Hkv * G, 128))
+    out = attention.prefill_attention(q, kc, kn, vc, vn, P, start)
+    mask = torch.from_numpy(np.arange(T)[None, :] <= start + np.arange(C)[:, None])
+    for kv in range(Hkv):
+        K = torch.from_numpy(attention.dequantise(kc[kv], kn[kv], P[kv]))
+        V = torch.from_numpy(attention.dequantise(vc[kv], vn[kv], P[kv]))
+        for g in range(G):
+            h = kv * G + g
+            Q = torch.from_numpy(q[:, h])
+            ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], attn_mask=mask[None])[0]
+            np.testing.assert_allclose(out[:, h], ref.numpy(), rtol=1e-12, atol=1e-12)
+    # the last query token sees the whole cache: plain decode attention
+    np.testing.assert_allclose(out[-1], attention.attention_rotated(q[-1], kc, kn, vc, vn, P), atol=1e-13)
