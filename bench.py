@@ -382,6 +382,75 @@ def bench_prefill(steps, warmup, device, stream, world=1):
             "launches": 48 * steps}
 
 
+def bench_deferred(steps, warmup, device, stream, world=1, n_layers=32):
+    """Deferred quantisation on a Llama-3.1-8B-shaped stack (32 layers, 32 q / 8 kv heads): the
+    8192-token prompt stays fp16, 512 generated tokens are packed; one decode step appends the
+    next token (quantised) and attends over fp16 prefix + packed tail in every layer
+    (iq_decode_step_deferred), replayed as one CUDA graph."""
+    import torch
+
+    from rotated_bit_kv_iq_b200 import binding as Bd
+    from rotated_bit_kv_iq_b200 import inputs
+
+    Hq, Hkv, Lp, T = 32, 8, 8192, 8704
+    L = n_layers
+    cache = Bd.PagedCache(L, Hkv, T, 1, device=device)
+    params = torch.from_numpy(Bd.iq_init_rotation(inputs.ROTATION_SEED, L, Hkv)).to(device)
+    k16, v16, qs, kn, vn = [], [], [], [], []
+    start = torch.full((1,), Lp, dtype=torch.int32, device=device)
+    for l in range(L):
+        K = inputs.kv_tokens_device(0, l, Hkv, 0, T, device=device)  # (T, Hkv, 128)
+        V = inputs.kv_tokens_device(0, l, Hkv, 1, T, device=device)
+        k16.append(K[:Lp].permute(1, 0, 2).contiguous()[None])
+        v16.append(V[:Lp].permute(1, 0, 2).contiguous()[None])
+        Bd.iq_encode_append(cache, l, K[Lp:T - 1][None].contiguous(), V[Lp:T - 1][None].contiguous(), start, params,
+                            stream)
+        kn.append(K[T - 1][None].contiguous())
+        vn.append(V[T - 1][None].contiguous())
+        qs.append(inputs.queries_device(0, l, 1, Hq, device=device))
+    torch.cuda.synchronize()
+    plen = torch.full((1,), Lp, dtype=torch.int32, device=device)
+    ctx = torch.full((1,), T, dtype=torch.int32, device=device)
+    out = torch.empty((L, 1, Hq, 128), dtype=torch.float32, device=device)
+    ws = torch.zeros(Bd.iq_decode_deferred_workspace_size(1, Hq, Hkv, T, Lp), dtype=torch.uint8, device=device)
+
+    def step():
+        for l in range(L):
+            Bd.iq_decode_step_deferred(cache, l, k16[l], v16[l], plen, qs[l], kn[l], vn[l], ctx, T, params, out[l], ws,
+                                       stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(warmup):
+            graph.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, device)
+    del graph
+    layer_bytes = Hkv * (Lp * 2 * 256 + (T - Lp) * BYTES_PER_TOKEN_HEAD)  # fp16 K+V prefix, packed tail
+    peak, peak_kind = _peaks()
+    kern_ms = ms / L
+    ach = layer_bytes / (kern_ms * 1e-3) / 1e9
+    return {"workload": f"llama8b_deferred: {L} layers, 32 q / 8 kv heads, 8192-token fp16 prompt + 512 packed "
+                        "tokens, decode step appending the next token (deferred quantisation)",
+            "value": world * layer_bytes * L / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "us_per_layer": kern_ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                         "traffic": None, "peak_kind": peak_kind, "bytes_per_launch": layer_bytes,
+                         "kernel": "prefix_kernel + decode_kernel per layer, CUDA-graph step time / layers"},
+            "launches": 2 * L * steps}
+
+
 def max_over_ranks(x, device=None):
     """Max of a float over the ranks of the default process group (x itself without one).
     Every timed quantity of a multi-rank run goes through this, so that the job's time is
@@ -622,7 +691,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed step's output")
     ap.add_argument("--layers", type=int, default=0, help="override the stack depth (profiling runs)")
-    ap.add_argument("--only", default="", choices=["", "serving", "encode", "prefill"],
+    ap.add_argument("--only", default="", choices=["", "serving", "encode", "prefill", "deferred"],
                     help="run one secondary workload alone (profiling runs); no headline line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -658,6 +727,8 @@ def main():
             res = bench_serving(args.steps, args.warmup, dev, stream, seed=rank, world=world, n_layers=args.layers)
         elif args.only == "prefill":
             res = bench_prefill(args.steps, args.warmup, dev, stream, world=world)
+        elif args.only == "deferred":
+            res = bench_deferred(args.steps, args.warmup, dev, stream, world=world, n_layers=args.layers or 32)
         else:
             res = bench_encode(args.steps, args.warmup, dev, stream)
         if rank == 0:
@@ -743,6 +814,10 @@ def main():
         pre = bench_prefill(args.steps, args.warmup, dev, stream, world=world)
         result["prefill"] = pre
         result["gpu_launches"] += pre["launches"]
+        torch.cuda.empty_cache()
+        dfr = bench_deferred(args.steps, args.warmup, dev, stream, world=world)
+        result["deferred"] = dfr
+        result["gpu_launches"] += dfr["launches"]
         torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu:

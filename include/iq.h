@@ -235,6 +235,38 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
                          const int32_t* ctx_len_dev, int32_t max_ctx, const float* params_dev, float* out_dev,
                          void* workspace_dev, size_t workspace_bytes, iq_stream_t stream);
 
+/* Deferred quantisation ("RotorQuant" (sd114.wiki), section "2. 延迟量化策略"; "压缩与速度的博弈"
+ * (zhichai.net), section "延迟量化（Deferred Quantization）"): the prompt's K/V stay fp16 as the model
+ * produced them (no rotation, no quantisation) and tokens generated during decoding are quantised
+ * when they are inserted.  An fp16 prefix of one layer: */
+typedef struct {
+  const void* k_dev;       /* device fp16 [batch][n_kv_heads][max_len][128], unrotated K of positions 0.. */
+  const void* v_dev;       /* device fp16 [batch][n_kv_heads][max_len][128], unrotated V */
+  const int32_t* len_dev;  /* device int32 [batch]: positions 0 .. len-1 of sequence b are here */
+  int32_t max_len;         /* capacity of the arrays per sequence and kv head (tokens) */
+} iq_fp16_prefix;
+
+/* Workspace bytes iq_decode_step_deferred needs (the decode workspace plus the fp16 prefix's
+ * split partials); zero-filled before its first use, like the decode workspace. */
+size_t iq_decode_deferred_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx,
+                                         int32_t max_len);
+
+/* Decode step over a cache whose first len[b] positions are the fp16 prefix: the new token (k_new,
+ * v_new, position ctx_len[b]-1) is quantised and appended to the packed cache like
+ * iq_decode_step, and every query head attends over positions 0 .. ctx_len[b]-1: the prefix's from
+ * the fp16 arrays (exact fp16 products, fp32 sums), positions len[b] .. ctx_len[b]-1 from the
+ * packed cache.  Requires 0 <= len[b] < ctx_len[b] and len[b] <= max_len (values outside are
+ * clamped and flagged with IQ_DEVERR_CTX); the packed cache is read from the tile holding
+ * position len[b] on (earlier positions of that tile are ignored).  Other arguments, results and
+ * errors as for iq_decode_step, with the workspace of iq_decode_deferred_workspace_size.  Two
+ * kernels: the prefix's attention (split partials, rotated forward into the packed basis), then
+ * the fused step, which merges both before its single inverse rotation. */
+iq_status iq_decode_step_deferred(const iq_cache* cache, int32_t layer, const iq_fp16_prefix* prefix, const void* q_dev,
+                                  iq_dtype q_dtype, const void* k_new_dev, const void* v_new_dev, int32_t batch,
+                                  int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
+                                  const float* params_dev, float* out_dev, void* workspace_dev, size_t workspace_bytes,
+                                  iq_stream_t stream);
+
 /* Workspace bytes iq_prefill_attention needs for these sizes on the current device (per query
  * block of 8 tokens, kv head and split of the context: the split partials).  Needs no zeroing. */
 size_t iq_prefill_workspace_size(int32_t batch, int32_t n_tokens, int32_t n_kv_heads, int32_t max_ctx);

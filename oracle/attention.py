@@ -104,3 +104,31 @@ def prefill_attention(q, k_codes, k_norm16, v_codes, v_norm16, params, start, bi
         out[i] = attention_rotated(q[i], k_codes[:, :T], k_norm16[:, :T], v_codes[:, :T], v_norm16[:, :T], params,
                                    bits, v_bits, variant)
     return out
+
+
+def attention_mixed(q, k16_prefix, v16_prefix, k_codes, k_norm16, v_codes, v_norm16, params, bits=3, v_bits=None,
+                    variant="iso"):
+    """Deferred quantisation ("RotorQuant" sd114.wiki section "2. 延迟量化策略"; [TQ-RQ] section
+    "延迟量化（Deferred Quantization）"): the prompt's K/V are kept in fp16 and only later tokens
+    are quantised.  Attention over positions 0 .. P-1 held as fp16 vectors (k16_prefix,
+    v16_prefix: (Hkv, P, 128)) followed by packed positions P .. T-1 (k_codes etc.: (Hkv, T-P,
+    ...)): plain softmax attention over the concatenation of the fp16 keys and values, promoted
+    to fp64, and the dequantised packed ones.  Returns (Hq, 128) fp64."""
+    v_bits = bits if v_bits is None else v_bits
+    q = np.asarray(q, dtype=np.float64)
+    Hq = q.shape[0]
+    Hkv = np.asarray(k16_prefix).shape[0]
+    G = Hq // Hkv
+    out = np.zeros((Hq, D))
+    for kv in range(Hkv):
+        K = np.concatenate([np.asarray(k16_prefix[kv], dtype=np.float16).astype(np.float64),
+                            dequantise(k_codes[kv], k_norm16[kv], params[kv], bits, variant)])
+        V = np.concatenate([np.asarray(v16_prefix[kv], dtype=np.float16).astype(np.float64),
+                            dequantise(v_codes[kv], v_norm16[kv], params[kv], v_bits, variant)])
+        if K.shape[0] == 0:
+            continue
+        for h in range(kv * G, (kv + 1) * G):
+            s = K @ q[h] / math.sqrt(D)
+            p = np.exp(s - s.max())
+            out[h] = (p / p.sum()) @ V
+    return out

@@ -79,6 +79,15 @@ class iq_cache(ctypes.Structure):
     ]
 
 
+class iq_fp16_prefix(ctypes.Structure):
+    _fields_ = [
+        ("k_dev", ctypes.c_void_p),
+        ("v_dev", ctypes.c_void_p),
+        ("len_dev", ctypes.c_void_p),
+        ("max_len", ctypes.c_int32),
+    ]
+
+
 _lib = None
 
 
@@ -113,6 +122,11 @@ def lib():
         L.iq_decode_step.argtypes = [P, i32, vp, ctypes.c_int, vp, vp, i32, i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_decode_attention_noalloc.restype = ctypes.c_int
         L.iq_decode_attention_noalloc.argtypes = [P, i32, vp, ctypes.c_int, i32, i32, vp, i32, vp, vp, vp]
+        L.iq_decode_deferred_workspace_size.restype = sz
+        L.iq_decode_deferred_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.iq_decode_step_deferred.restype = ctypes.c_int
+        L.iq_decode_step_deferred.argtypes = [P, i32, ctypes.POINTER(iq_fp16_prefix), vp, ctypes.c_int, vp, vp, i32,
+                                              i32, vp, i32, vp, vp, vp, sz, vp]
         L.iq_prefill_workspace_size.restype = sz
         L.iq_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
         L.iq_prefill_attention.restype = ctypes.c_int
@@ -214,6 +228,24 @@ def iq_decode_step(cache, layer, q, k_new, v_new, ctx_len, max_ctx, params, out,
     _check("iq_decode_step", lib().iq_decode_step(
         ctypes.byref(cache.c), layer, _ptr(q), dtype, _ptr(k_new), _ptr(v_new), int(q.shape[0]), int(q.shape[1]),
         _ptr(ctx_len), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace),
+        int(workspace.numel() * workspace.element_size()), _stream(stream)))
+
+
+def iq_decode_deferred_workspace_size(batch, n_q_heads, n_kv_heads, max_ctx, max_len):
+    return int(lib().iq_decode_deferred_workspace_size(batch, n_q_heads, n_kv_heads, max_ctx, max_len))
+
+
+def iq_decode_step_deferred(cache, layer, k16, v16, prefix_len, q, k_new, v_new, ctx_len, max_ctx, params, out,
+                            workspace, stream=None):
+    """Decode step over an fp16 prefix (k16, v16: fp16 [batch][Hkv][max_len][128], prefix_len: int32
+    [batch]) followed by the packed cache; the new token is appended (quantised) as by iq_decode_step."""
+    import torch
+
+    dtype = IQ_F32 if q.dtype == torch.float32 else IQ_F16
+    pre = iq_fp16_prefix(k16.data_ptr(), v16.data_ptr(), prefix_len.data_ptr(), int(k16.shape[2]))
+    _check("iq_decode_step_deferred", lib().iq_decode_step_deferred(
+        ctypes.byref(cache.c), layer, ctypes.byref(pre), _ptr(q), dtype, _ptr(k_new), _ptr(v_new), int(q.shape[0]),
+        int(q.shape[1]), _ptr(ctx_len), int(max_ctx), _ptr(params), _ptr(out), _ptr(workspace),
         int(workspace.numel() * workspace.element_size()), _stream(stream)))
 
 

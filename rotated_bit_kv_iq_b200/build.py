@@ -8,7 +8,7 @@ from concurrent.futures import ThreadPoolExecutor
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libiq.so")
-CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu", "iq_noalloc.cu",
+CUDA_SOURCES = ["iq_api.cu", "iq_encode.cu", "iq_decode.cu", "iq_export.cu", "iq_noalloc.cu", "iq_deferred.cu",
                 # decode kernels, one unit per (K bits, V bits) pair
                 "iq_decode_k2v2.cu", "iq_decode_k3v2.cu", "iq_decode_k3v3.cu", "iq_decode_k4v2.cu",
                 "iq_decode_k4v3.cu", "iq_decode_k4v4.cu"]

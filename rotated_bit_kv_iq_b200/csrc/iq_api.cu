@@ -246,6 +246,46 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
   return e ? IQ_ERR_CUDA : IQ_OK;
 }
 
+size_t iq_decode_deferred_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads, int32_t max_ctx,
+                                         int32_t max_len) {
+  if (batch < 0 || n_q_heads < 0 || n_kv_heads < 1 || max_ctx < 0 || max_len < 0) return 0;
+  const int extra = batch * n_kv_heads * prefix_splits(batch, n_kv_heads, max_len, sm_count());
+  return decode_workspace_bytes(batch, n_q_heads, n_kv_heads, max_ctx, extra);
+}
+
+iq_status iq_decode_step_deferred(const iq_cache* cache, int32_t layer, const iq_fp16_prefix* prefix, const void* q_dev,
+                                  iq_dtype q_dtype, const void* k_new_dev, const void* v_new_dev, int32_t batch,
+                                  int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
+                                  const float* params_dev, float* out_dev, void* workspace_dev, size_t workspace_bytes,
+                                  iq_stream_t stream) {
+  iq_status st = check_cache(cache, layer);
+  if (st != IQ_OK) return st;
+  if (!prefix || !prefix->k_dev || !prefix->v_dev || !prefix->len_dev || prefix->max_len < 0) return IQ_ERR_INVALID_ARG;
+  if (batch < 0 || n_q_heads < 1 || max_ctx < 1 || !q_dev || !ctx_len_dev || !params_dev || !out_dev || !k_new_dev ||
+      !v_new_dev)
+    return IQ_ERR_INVALID_ARG;
+  if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
+  if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
+  if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
+  const int G = n_q_heads / cache->n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
+  if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
+  if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(ctx_len_dev, 4) ||
+      !aligned(k_new_dev, 16) || !aligned(v_new_dev, 16) || !aligned(prefix->k_dev, 16) ||
+      !aligned(prefix->v_dev, 16) || !aligned(prefix->len_dev, 4))
+    return IQ_ERR_ALIGNMENT;
+  const size_t need = iq_decode_deferred_workspace_size(batch, n_q_heads, cache->n_kv_heads, max_ctx, prefix->max_len);
+  if (!workspace_dev || workspace_bytes < need) return IQ_ERR_WORKSPACE;
+  if (!aligned(workspace_dev, 256)) return IQ_ERR_ALIGNMENT;
+  const LayerView v = view(cache, layer);
+  const int e = launch_decode_deferred(v, q_dev, q_dtype == IQ_F32, k_new_dev, v_new_dev, batch, n_q_heads, ctx_len_dev,
+                                       max_ctx, layer_params(cache, params_dev, layer), out_dev, workspace_dev,
+                                       kernel_consts(v.kb, v.vb), stream, prefix->k_dev, prefix->v_dev,
+                                       prefix->len_dev, prefix->max_len);
+  return e ? IQ_ERR_CUDA : IQ_OK;
+}
+
 size_t iq_prefill_workspace_size(int32_t batch, int32_t n_tokens, int32_t n_kv_heads, int32_t max_ctx) {
   if (batch < 0 || n_tokens < 0 || n_kv_heads < 1 || max_ctx < 0) return 0;
   return prefill_workspace_bytes(batch, n_tokens, n_kv_heads, max_ctx);

@@ -14,7 +14,7 @@ namespace iq {
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-static int sm_count() {
+int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
@@ -53,17 +53,19 @@ int decode_ctas(int batch, int n_kv_heads, int max_ctx, int resident) {
 // slot c + gid (a CTA's run covers consecutive groups), so 2 * #SMs + groups slots suffice.
 static size_t ws_slots(int batch, int n_kv_heads) { return (size_t)2 * sm_count() + (size_t)batch * n_kv_heads; }
 
-size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx) {
+int workspace_base_slots(int batch, int n_kv_heads) { return (int)ws_slots(batch, n_kv_heads); }
+
+size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx, int extra_slots) {
   (void)n_q_heads;
   (void)max_ctx;
-  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
+  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads) + (size_t)extra_slots;
   return align256(groups * 8) + align256(slots * HMAX * sizeof(float2)) + align256(slots * HMAX * D * sizeof(float));
 }
 
 size_t decode_counter_bytes(int batch, int n_kv_heads) { return align256((size_t)batch * n_kv_heads * 8); }
 
-Workspace carve_workspace(void* ws, int batch, int n_kv_heads) {
-  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads);
+Workspace carve_workspace(void* ws, int batch, int n_kv_heads, int extra_slots) {
+  const size_t groups = (size_t)batch * n_kv_heads, slots = ws_slots(batch, n_kv_heads) + (size_t)extra_slots;
   Workspace w;
   char* p = (char*)ws;
   w.counters = (uint32_t*)p;
@@ -78,7 +80,7 @@ Workspace carve_workspace(void* ws, int batch, int n_kv_heads) {
 #define IQ_DECL(KB, VB)                                                                                      \
   extern template int launch_decode_kv<KB, VB>(const LayerView&, const void*, int, int, int, const int32_t*, \
                                                int, const float*, float*, void*, const KernelConsts&, void*,  \
-                                               const void*, const void*);
+                                               const void*, const void*, const DeferredInfo*);
 IQ_DECODE_WIDTHS(IQ_DECL)
 #undef IQ_DECL
 #define IQ_DECL(KB, VB)                                                                                         \
@@ -89,11 +91,11 @@ IQ_DECODE_WIDTHS(IQ_DECL)
 
 static int dispatch(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads, const int32_t* ctx_len,
                     int max_ctx, const float* params_layer, float* out, void* workspace, const KernelConsts& kc,
-                    void* stream, const void* k_new, const void* v_new) {
+                    void* stream, const void* k_new, const void* v_new, const DeferredInfo* def = nullptr) {
 #define IQ_CASE(KB, VB)                                                                                          \
   if (v.kb == KB && v.vb == VB)                                                                                 \
     return launch_decode_kv<KB, VB>(v, q, q_f32, batch, n_q_heads, ctx_len, max_ctx, params_layer, out, workspace, \
-                                    kc, stream, k_new, v_new);
+                                    kc, stream, k_new, v_new, def);
   IQ_DECODE_WIDTHS(IQ_CASE)
 #undef IQ_CASE
   return (int)cudaErrorInvalidValue;
@@ -111,6 +113,22 @@ int launch_decode_step(const LayerView& v, const void* q, int q_f32, const void*
                        void* workspace, const KernelConsts& kc, void* stream) {
   return dispatch(v, q, q_f32, batch, n_q_heads, ctx_len, max_ctx, params_layer, out, workspace, kc, stream, k_new,
                   v_new);
+}
+
+// Deferred quantisation: the fp16-prefix kernel writes its split partials into the extra slots,
+// then the fused step (which waits for it) attends over the packed tail and merges both.
+int launch_decode_deferred(const LayerView& v, const void* q, int q_f32, const void* k_new, const void* v_new,
+                           int batch, int n_q_heads, const int32_t* ctx_len, int max_ctx, const float* params_layer,
+                           float* out, void* workspace, const KernelConsts& kc, void* stream, const void* k16,
+                           const void* v16, const int32_t* len, int max_len) {
+  if (batch == 0 || n_q_heads == 0) return 0;
+  const int splits = prefix_splits(batch, v.n_kv_heads, max_len, sm_count());
+  int e = launch_prefix(v, k16, v16, len, max_len, ctx_len, max_ctx, q, q_f32, batch, n_q_heads, params_layer, kc,
+                        workspace, splits, workspace_base_slots(batch, v.n_kv_heads), stream);
+  if (e) return e;
+  DeferredInfo def{len, splits};
+  return dispatch(v, q, q_f32, batch, n_q_heads, ctx_len, max_ctx, params_layer, out, workspace, kc, stream, k_new,
+                  v_new, &def);
 }
 
 // Prefill workspace: per (group, split, query token, head) one (m, l) pair and one 128-float O.

@@ -64,11 +64,11 @@ struct DecSmem {
   static constexpr int kappa = qfrag + 32 * QF_WORDS * 4;                 // float [head] score scales
   static constexpr int sparams = kappa + HMAX * 4;                        // float [256] one head's parameters
   static constexpr int flags = sparams + 256 * 4;                         // int [4]
-  static constexpr int valid = flags + 16;                                // uint8 [warp][slot] half masks
-  static constexpr int bars = (valid + DEC_WARPS * NSLOT + 7) / 8 * 8;    // uint64 [warp][slot]
+  static constexpr int valid = flags + 16;                                // uint32 [warp][slot] token masks
+  static constexpr int bars = valid + DEC_WARPS * NSLOT * 4;              // uint64 [warp][slot]
   static constexpr int cursors = bars + DEC_WARPS * NSLOT * 8;           // Cursor [warp]
-  static constexpr int plan = cursors + DEC_WARPS * 48;                   // int [batch+1] tile prefix, [batch] ctx
-  static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(2 * batch + 1); }
+  static constexpr int plan = cursors + DEC_WARPS * 48;  // int [batch+1] tile prefix, [batch] ctx, [batch] fp16 prefix
+  static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(3 * batch + 1); }
 };
 
 struct Workspace {
@@ -76,7 +76,8 @@ struct Workspace {
   float2* part_ml;     // [slots][HMAX] (max in log2 units, sum of 2^(s-max))
   float* part_o;       // [slots][HMAX][128]
 };
-Workspace carve_workspace(void* ws, int batch, int n_kv_heads);
+Workspace carve_workspace(void* ws, int batch, int n_kv_heads, int extra_slots = 0);
+int workspace_base_slots(int batch, int n_kv_heads);  // partial slots of the CTAs; extra slots follow
 int resident_per_sm(const void* fn, size_t smem, int threads);
 
 struct DecArgs {
@@ -90,23 +91,44 @@ struct DecArgs {
   const __half* k_new;
   const __half* v_new;
   KernelConsts kc;
+  // deferred quantisation: positions 0 .. pre_len[b]-1 of sequence b are held in fp16 outside the
+  // packed cache (NULL: none); their attention arrives as n_extra partials per group, at partial
+  // slots extra_base + gid * n_extra + s, written by the preceding kernel
+  const int32_t* pre_len;
+  int n_extra, extra_base;
 };
 
 // ------------------------------------------------------------------ work plan
 // pre[b] = tiles of sequences 0..b-1 (per kv head) and pre[B + 1 + b] = the clamped context
 // length of sequence b; every CTA builds the same table.
+static // Clamped context length and fp16 prefix length of sequence b (flags out-of-range values once).
+__device__ __forceinline__ void seq_lengths(const DecArgs& a, int b, int& c, int& p) {
+  c = a.ctx_len[b];
+  if (c < 0 || c > a.max_ctx) {
+    if (a.v.status && blockIdx.x == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
+    c = c < 0 ? 0 : a.max_ctx;
+  }
+  p = 0;
+  if (a.pre_len) {  // 0 <= prefix < ctx: the step's new token is always packed
+    p = a.pre_len[b];
+    if (p < 0 || (c > 0 && p >= c)) {
+      if (a.v.status && blockIdx.x == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
+      p = p < 0 ? 0 : max(c - 1, 0);
+    }
+  }
+}
+// Packed tiles of a sequence: absolute tiles p/32 .. ceil(c/32)-1.
+__device__ __forceinline__ int seq_tiles(int c, int p) { return c > 0 ? (c + TT - 1) / TT - p / TT : 0; }
+
 static __device__ void build_plan(const DecArgs& a, int* pre) {
   const int B = a.batch;
   const int per = (B + DEC_THREADS - 1) / DEC_THREADS;
   const int lo = threadIdx.x * per, hi = min(B, lo + per);
   int sum = 0;
   for (int b = lo; b < hi; ++b) {
-    int c = a.ctx_len[b];
-    if (c < 0 || c > a.max_ctx) {
-      if (a.v.status && blockIdx.x == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
-      c = c < 0 ? 0 : a.max_ctx;
-    }
-    sum += (c + TT - 1) / TT;
+    int c, p;
+    seq_lengths(a, b, c, p);
+    sum += seq_tiles(c, p);
   }
   // block-wide exclusive scan of the per-thread sums
   __shared__ int warp_tot[DEC_WARPS];
@@ -124,10 +146,12 @@ static __device__ void build_plan(const DecArgs& a, int* pre) {
   int run = base + incl - sum;
   for (int b = lo; b < hi; ++b) {
     pre[b] = run;
-    int c = a.ctx_len[b];
+    int c = a.ctx_len[b], p = a.pre_len ? a.pre_len[b] : 0;
     c = c < 0 ? 0 : (c > a.max_ctx ? a.max_ctx : c);
+    p = p < 0 ? 0 : ((c > 0 && p >= c) ? max(c - 1, 0) : p);
     pre[B + 1 + b] = c;
-    run += (c + TT - 1) / TT;
+    pre[2 * B + 1 + b] = p;
+    run += seq_tiles(c, p);
   }
   if (threadIdx.x == DEC_THREADS - 1) pre[B] = run;
   __syncthreads();
@@ -137,6 +161,7 @@ static __device__ void build_plan(const DecArgs& a, int* pre) {
 struct Seg {
   int b, kvh, ntiles, lo, hi;  // tiles [lo, hi) of the group's ntiles lie in this CTA
   int ctx;                     // context length of sequence b (clamped)
+  int plo, first;              // fp16 prefix length (packed positions start there) and its tile
   long long gstart;
 };
 __device__ __forceinline__ Seg segment_at(const DecArgs& a, const int* pre, int B, int Hkv, long long x, long long c1) {
@@ -155,6 +180,8 @@ __device__ __forceinline__ Seg segment_at(const DecArgs& a, const int* pre, int 
   s.lo = (int)(x - s.gstart);
   s.hi = (int)min((long long)s.ntiles, c1 - s.gstart);
   s.ctx = pre[B + 1 + s.b];
+  s.plo = pre[2 * B + 1 + s.b];
+  s.first = s.plo / TT;
   return s;
 }
 
@@ -178,7 +205,7 @@ static_assert(sizeof(Cursor) <= 48, "one cursor slot per warp");
 // flight while the warp computes (the entry is checked when the copy is issued).
 __device__ __forceinline__ int cursor_page(const Cursor& c, const LayerView& v) {
   if (c.done || (threadIdx.x & 31) != 0) return -1;
-  const int t = TT * c.i;
+  const int t = TT * (c.s.first + c.i);
   int pg = c.s.b;
   if (v.block_table && t < c.s.ctx) {
     const int idx = t / v.page_size;
@@ -202,11 +229,18 @@ __device__ __forceinline__ bool is_new_token_tile(const Seg& s, int i) {
   return FUSED && i == s.ntiles - 1;
 }
 
-// Copy tile i of group (b, kvh) -- one tile record, 3200 bytes -- into slot `st` with one bulk
-// copy (lane 0).  raw_pg is the tile's block-table entry (or b without a table), validated
-// here; the half mask marks the 16-token halves that lie before ctx.
-__device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, int i, int ctx, int raw_pg, uint8_t* st,
-                                           uint8_t* valid, uint64_t* bar, uint32_t tbytes) {
+// Copy tile i (absolute: positions 32i .. 32i+31) of group (b, kvh) -- one tile record -- into slot
+// `st` with one bulk copy (lane 0).  raw_pg is the tile's block-table entry (or b without a table),
+// validated here; the token mask has bit u set when position 32i + u lies in [lo, ctx) on a valid
+// page (lo > 0: the positions below are not in the packed cache).
+__device__ __forceinline__ uint32_t token_range_mask(int a, int e) {  // bits [max(a,0), min(e,32))
+  a = max(a, 0);
+  e = min(e, 32);
+  if (e <= a) return 0u;
+  return (e == 32 ? 0xFFFFFFFFu : ((1u << e) - 1u)) & ~((1u << a) - 1u);
+}
+__device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, int i, int ctx, int lo, int raw_pg,
+                                           uint8_t* st, uint32_t* valid, uint64_t* bar, uint32_t tbytes) {
   const int t = TT * i;
   int page = -1;
   if (t < ctx) {
@@ -219,8 +253,8 @@ __device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, i
       page = -1;
     }
   }
-  const uint32_t mask = page < 0 ? 0u : (t + 16 < ctx ? 3u : 1u);
-  *valid = (uint8_t)mask;
+  const uint32_t mask = page < 0 ? 0u : token_range_mask(lo - t, ctx - t);
+  *valid = mask;
   mbar_arrive_expect_tx(bar, mask ? tbytes : 0);
   if (mask) bulk_g2s(st, tile_record(v, page, kvh, t % v.page_size), tbytes, bar);
 }
@@ -257,7 +291,7 @@ __device__ __forceinline__ uint32_t pack4(uint32_t x0, uint32_t x1, uint32_t x2,
 // head n, n >= 4 = P' lo of head n - 4; lanes t < 2 accumulate the hi columns, t >= 2 the
 // lo columns of the same heads (added together at the segment end).
 template <bool P4, int KB, int VB>
-__device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uint32_t vmask, int tok_end,
+__device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uint32_t tmask,
                                              const uint32_t* __restrict__ qf, float kappa,
                                              const KernelConsts& kc, WarpState& ws) {
   using SM = DecSmem<KB, VB>;
@@ -337,11 +371,11 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
     nv[2 * nt] = nvv.x;
     nv[2 * nt + 1] = nvv.y;
   }
-  if (vmask != 3u || tok_end < TT) {  // a partial tile: tokens past the context or on bad pages
+  if (tmask != 0xFFFFFFFFu) {  // a partial tile: tokens outside the context or on bad pages
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int tok = 8 * (i >> 1) + 2 * t + (i & 1);
-      if (!((vmask >> (tok >> 4)) & 1u) || tok >= tok_end) {
+      if (!((tmask >> tok) & 1u)) {
         s[i] = -CUDART_INF_F;
         nv[i] = 0.f;
       }
@@ -509,6 +543,11 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
 // two at a time, four warps each, one coordinate per lane; when only one of the two exists,
 // both warp groups work on it, each over half of the partials, and meet in shared memory.
 // O = sum_c 2^(m_c - M) O_c and L likewise, then R^T per head.
+// Partial slot of the k-th partial of group gid: the group's CTAs first, then its extra partials.
+__device__ __forceinline__ size_t part_slot(const DecArgs& a, int gid, int c_first, int n_parts, int k) {
+  return k < n_parts ? (size_t)(c_first + k + gid) : (size_t)a.extra_base + (size_t)gid * a.n_extra + (k - n_parts);
+}
+
 __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, int gid, int c_first, int n_parts, int k,
                                             float* buf, const float* prm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, grp = warp >> 2;  // groups 0, 1 work
@@ -519,15 +558,18 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
     const bool split = h0 + n_parts >= a.g_real;
     const int h = split ? h0 : h0 + grp * n_parts;
     const int half = (n_parts + 1) >> 1;
-    const int p_lo = split ? grp * half : 0, p_hi = split ? (grp ? n_parts : half) : n_parts;
+    const int n_all = n_parts + a.n_extra;
+    const int half_all = (n_all + 1) >> 1;
+    const int p_lo = split ? grp * half_all : 0, p_hi = split ? (grp ? n_all : half_all) : n_all;
+    (void)half;
     float acc = 0.f, M = -CUDART_INF_F, L = 0.f;
     for (int c0 = p_lo; c0 < p_hi && grp < 2; c0 += 32) {
       const int nb = min(32, p_hi - c0);
       float ov[32];
 #pragma unroll
       for (int u = 0; u < 32; ++u)
-        ov[u] = __ldcg(a.ws.part_o + (((size_t)(c_first + c0 + min(u, nb - 1)) + gid) * HMAX + h) * D + coord);
-      const float2 ml = lane < nb ? __ldcg(a.ws.part_ml + ((size_t)(c_first + c0 + lane) + gid) * HMAX + h)
+        ov[u] = __ldcg(a.ws.part_o + (part_slot(a, gid, c_first, n_parts, c0 + min(u, nb - 1)) * HMAX + h) * D + coord);
+      const float2 ml = lane < nb ? __ldcg(a.ws.part_ml + part_slot(a, gid, c_first, n_parts, c0 + lane) * HMAX + h)
                                   : make_float2(-CUDART_INF_F, 0.f);
       float Mb = ml.x;
 #pragma unroll
@@ -597,7 +639,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.v.n_kv_heads, B = a.batch;
   uint8_t* ring = smem + DecSmem::ring + warp * NSLOT * SLOT_BYTES;
-  uint8_t* valid = smem + DecSmem::valid + warp * NSLOT;
+  uint32_t* valid = reinterpret_cast<uint32_t*>(smem + DecSmem::valid) + warp * NSLOT;
   uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + DecSmem::bars) + warp * NSLOT;
   if (lane == 0) {
     for (int s = 0; s < NSLOT; ++s) mbar_init(&wbar[s], 1);
@@ -624,7 +666,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     // lanes 1.. request the block-table entries of the warp's next tiles now, so that the
     // dependent lookups of the first copies below find them in L1
     if (!fc.done && a.v.block_table && lane > 0 && lane < NSLOT) {
-      const int t = TT * (fc.i + lane * DEC_WARPS);
+      const int t = TT * (fc.s.first + fc.i + lane * DEC_WARPS);
       if (fc.i + lane * DEC_WARPS < fc.s.hi && t < fc.s.ctx && t / a.v.page_size < a.v.max_pages)
         asm volatile("prefetch.global.L1 [%0];" ::"l"(a.v.block_table + (size_t)fc.s.b * a.v.max_pages + t / a.v.page_size));
     }
@@ -644,7 +686,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       if (is_new_token_tile<FUSED>(fc.s, fc.i) && fc.s.gstart != app_done) break;
       const int sl_i = k_fetch % NSLOT;
       if (lane == 0)
-        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.i, ctx, pg, ring + sl_i * SLOT_BYTES, &valid[sl_i], &wbar[sl_i],
+        issue_tile(a.v, fc.s.b, fc.s.kvh, fc.s.first + fc.i, ctx, fc.s.plo, pg, ring + sl_i * SLOT_BYTES, &valid[sl_i],
+                   &wbar[sl_i],
                    SLOT_BYTES);
       ++k_fetch;
       fc.i += DEC_WARPS;
@@ -726,7 +769,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) st.acc[j][e] = 0.f;
 
-    const int ctx = seg.ctx;
     for (int i = seg.lo + warp; i < seg.hi; i += DEC_WARPS) {
       top_up();  // issues this tile if it is not in flight yet, and refills the ring
       const int sl_i = k_done % NSLOT;
@@ -735,7 +777,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
         if (landed) ++k_wait; else aborted = true;
       }
       if (!aborted)
-        process_tile<P4, KB, VB>(ring + sl_i * SLOT_BYTES, valid[sl_i], ctx - TT * i, qfrag + lane * QF_WORDS, kap,
+        process_tile<P4, KB, VB>(ring + sl_i * SLOT_BYTES, valid[sl_i], qfrag + lane * QF_WORDS, kap,
                                  a.kc, st);
       ++k_done;
       __syncwarp();
@@ -892,11 +934,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   }
 }
 
-// One decode launch for code widths (KB, VB); k_new / v_new select the fused step.
+// One decode launch for code widths (KB, VB); k_new / v_new select the fused step; def (or NULL)
+// describes an fp16 prefix whose partials a preceding kernel has written.
 template <int KB, int VB>
 int launch_decode_kv(const LayerView& v, const void* q, int q_f32, int batch, int n_q_heads, const int32_t* ctx_len,
                      int max_ctx, const float* params_layer, float* out, void* workspace, const KernelConsts& kc,
-                     void* stream, const void* k_new, const void* v_new) {
+                     void* stream, const void* k_new, const void* v_new, const DeferredInfo* def) {
   if (batch == 0 || n_q_heads == 0) return 0;
   DecArgs a;
   a.v = v;
@@ -909,7 +952,10 @@ int launch_decode_kv(const LayerView& v, const void* q, int q_f32, int batch, in
   a.ctx_len = ctx_len;
   a.params_layer = params_layer;
   a.out = out;
-  a.ws = carve_workspace(workspace, batch, v.n_kv_heads);
+  a.ws = carve_workspace(workspace, batch, v.n_kv_heads, def ? batch * v.n_kv_heads * def->n_extra : 0);
+  a.pre_len = def ? def->len : nullptr;
+  a.n_extra = def ? def->n_extra : 0;
+  a.extra_base = def ? workspace_base_slots(batch, v.n_kv_heads) : 0;
   a.k_new = (const __half*)k_new;
   a.v_new = (const __half*)v_new;
   a.kc = kc;

@@ -3,7 +3,8 @@
 
 namespace iq {
 template int launch_decode_kv<2, 2>(const LayerView&, const void*, int, int, int, const int32_t*, int, const float*,
-                                   float*, void*, const KernelConsts&, void*, const void*, const void*);
+                                   float*, void*, const KernelConsts&, void*, const void*, const void*,
+                                   const DeferredInfo*);
 template int launch_prefill_kv<2, 2>(const LayerView&, const void*, int, int, int, int, const int32_t*, int,
                                     const float*, float*, void*, const KernelConsts&, void*, int);
 }  // namespace iq

@@ -84,6 +84,14 @@ struct LayerView {
   int32_t rot;                 // rotation variant
 };
 
+// An fp16 prefix of the cache (deferred quantisation), resolved on the host: positions
+// 0 .. len[b]-1 of sequence b live in fp16 [batch][Hkv][max_len][128] K and V arrays; their
+// attention arrives as n_extra partials per (sequence, kv head).
+struct DeferredInfo {
+  const int32_t* len;
+  int n_extra;
+};
+
 // Kernel launchers (defined in the .cu files); return the launch error.
 int launch_encode(const LayerView& v, const void* k, const void* vsrc, int batch, int n_new,
                   const int32_t* start_pos, const float* params_layer, const KernelConsts& kc,
@@ -104,7 +112,17 @@ int launch_export(const LayerView& v, int kv, int seq, int t0, int n, uint8_t* c
 // Decode grid (host): CTAs of one decode launch on the current device, given how many CTAs of
 // the kernel an SM holds at once.
 int decode_ctas(int batch, int n_kv_heads, int max_ctx, int resident_per_sm);
-size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx);
+size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx, int extra_slots = 0);
+int prefix_splits(int batch, int n_kv_heads, int max_len, int n_sm);
+int sm_count();
+int launch_prefix(const LayerView& v, const void* k16, const void* v16, const int32_t* len, int max_len,
+                  const int32_t* ctx_len, int max_ctx, const void* q, int q_f32, int batch, int n_q_heads,
+                  const float* params_layer, const KernelConsts& kc, void* workspace, int splits, int extra_base,
+                  void* stream);
+int launch_decode_deferred(const LayerView& v, const void* q, int q_f32, const void* k_new, const void* v_new,
+                           int batch, int n_q_heads, const int32_t* ctx_len, int max_ctx, const float* params_layer,
+                           float* out, void* workspace, const KernelConsts& kc, void* stream, const void* k16,
+                           const void* v16, const int32_t* len, int max_len);
 size_t decode_counter_bytes(int batch, int n_kv_heads);  // leading bytes that must be zero between calls
 constexpr int DECODE_MAX_BATCH = 2048;  // sequences per decode call (per-CTA plan in shared memory)
 

@@ -43,8 +43,8 @@ struct PreSmem {
   static constexpr int qfrag = ring + PF_NSLOT * SLOT_BYTES;            // uint32 [QB][32][QF_WORDS]
   static constexpr int kappa = qfrag + PF_QB * 32 * QF_WORDS * 4;       // float [QB][HMAX]
   static constexpr int sparams = kappa + PF_QB * HMAX * 4;              // float [256]
-  static constexpr int valid = sparams + 256 * 4;                       // uint8 [slot]
-  static constexpr int bars = (valid + PF_NSLOT + 7) / 8 * 8;           // uint64 [slot]
+  static constexpr int valid = sparams + 256 * 4;                       // uint32 [slot] token masks
+  static constexpr int bars = valid + PF_NSLOT * 4;                     // uint64 [slot]
   static constexpr int bytes = bars + PF_NSLOT * 8;
 };
 
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) prefill_kernel(PreArgs a) {
   uint32_t* qfrag = reinterpret_cast<uint32_t*>(smem + SM::qfrag);
   float* kappa = reinterpret_cast<float*>(smem + SM::kappa);
   float* sprm = reinterpret_cast<float*>(smem + SM::sparams);
-  uint8_t* valid = smem + SM::valid;
+  uint32_t* valid = reinterpret_cast<uint32_t*>(smem + SM::valid);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bars);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.v.n_kv_heads;
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) prefill_kernel(PreArgs a) {
       pg = idx < a.v.max_pages ? a.v.block_table[(size_t)b * a.v.max_pages + idx] : -1;
     }
     const int sl = (i - t_lo) % PF_NSLOT;
-    issue_tile(a.v, b, kvh, i, kv_end, pg, ring + sl * SLOT, &valid[sl], &bars[sl], SLOT);
+    issue_tile(a.v, b, kvh, i, kv_end, 0, pg, ring + sl * SLOT, &valid[sl], &bars[sl], SLOT);
   };
   if (threadIdx.x == 0)
     for (int i = t_lo; i < min(t_hi, t_lo + PF_NSLOT); ++i) issue(i);
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) prefill_kernel(PreArgs a) {
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[sl], (k / PF_NSLOT) & 1, a.v.status));
     const int tok_end = my_pos + 1 - TT * i;  // causal limit inside this tile
     if (ok && live && tok_end > 0)
-      process_tile<P4, KB, VB>(ring + sl * SLOT, valid[sl], tok_end, qf, kap, a.kc, st);
+      process_tile<P4, KB, VB>(ring + sl * SLOT, valid[sl] & token_range_mask(0, tok_end), qf, kap, a.kc, st);
     __syncthreads();  // every warp is done with slot sl
     if (threadIdx.x == 0 && i + PF_NSLOT < t_hi) issue(i + PF_NSLOT);
   }

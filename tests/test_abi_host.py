@@ -29,7 +29,7 @@ def test_library_exports_every_declared_symbol(lib):
     assert {"iq_init_rotation", "iq_encode_append", "iq_decode_attention", "iq_decode_workspace_size",
             "iq_export_codes", "iq_status_string", "iq_cache_bytes", "iq_version", "iq_decode_step",
             "iq_init_rotation_variant", "iq_rotation_params_per_head", "iq_prefill_attention",
-            "iq_prefill_workspace_size"} <= names
+            "iq_prefill_workspace_size", "iq_decode_step_deferred", "iq_decode_deferred_workspace_size"} <= names
     for n in names:
         assert hasattr(lib, n), n
         assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
@@ -185,6 +185,27 @@ def test_prefill_rejects_bad_arguments(lib):
     assert pre(_fake_cache(k_bits=5)) == B.IQ_ERR_UNSUPPORTED
     assert pre(_fake_cache(), batch=5) == B.IQ_ERR_CAPACITY
     assert B.iq_prefill_workspace_size(1, 512, 8, 8192) > 0
+
+
+@cpu_only
+def test_deferred_step_rejects_bad_arguments(lib):
+    f = B.lib().iq_decode_step_deferred
+
+    def step(c, pre, max_ctx=32, hq=8, ws=0xA0000, ws_bytes=1 << 30):
+        return f(ctypes.byref(c), 0, ctypes.byref(pre) if pre is not None else None, 0x50000, 0, 0x58000, 0x5C000, 1,
+                 hq, 0x70000, max_ctx, 0x80000, 0x90000, ws, ws_bytes, None)
+
+    good = B.iq_fp16_prefix(0x100000, 0x200000, 0x300000, 16)
+    assert step(_fake_cache(), None) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), B.iq_fp16_prefix(None, 0x200000, 0x300000, 16)) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), B.iq_fp16_prefix(0x100000, 0x200000, None, 16)) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), B.iq_fp16_prefix(0x100008, 0x200000, 0x300000, 16)) == B.IQ_ERR_ALIGNMENT
+    assert step(_fake_cache(), B.iq_fp16_prefix(0x100000, 0x200000, 0x300000, -1)) == B.IQ_ERR_INVALID_ARG
+    assert step(_fake_cache(), good, max_ctx=65) == B.IQ_ERR_CAPACITY
+    assert step(_fake_cache(), good, hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert step(_fake_cache(), good, ws_bytes=64) == B.IQ_ERR_WORKSPACE
+    assert step(_fake_cache(k_bits=1), good) == B.IQ_ERR_UNSUPPORTED
+    assert B.iq_decode_deferred_workspace_size(1, 32, 8, 8704, 8192) > B.iq_decode_workspace_size(1, 32, 8, 8704)
 
 
 @cpu_only

@@ -617,3 +617,35 @@ def test_prefill_attention_is_causal_sdpa():
             np.testing.assert_allclose(out[:, h], ref.numpy(), rtol=1e-12, atol=1e-12)
     # the last query token sees the whole cache: plain decode attention
     np.testing.assert_allclose(out[-1], attention.attention_rotated(q[-1], kc, kn, vc, vn, P), atol=1e-13)
+
+
+def test_mixed_attention_pins():
+    """Attention over an fp16 prefix plus packed positions: equals torch SDPA (fp64) on the
+    concatenated keys and values; with no prefix it is the packed attention; with no packed
+    positions it is plain attention on the fp16 vectors."""
+    rng = np.random.default_rng(41)
+    Hkv, G, P, T2 = 2, 4, 13, 9
+    Pr = rotation.init_rotation(3, 1, Hkv)[0]
+    k16 = (rng.standard_normal((Hkv, P, 128)) * 2).astype(np.float16)
+    v16 = rng.standard_normal((Hkv, P, 128)).astype(np.float16)
+    kc = rng.integers(0, 8, (Hkv, T2, 128)).astype(np.uint8)
+    vc = rng.integers(0, 8, (Hkv, T2, 128)).astype(np.uint8)
+    kn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 30, (Hkv, T2)))
+    vn, _ = encode.norm_to_fp16_bits(rng.uniform(1, 10, (Hkv, T2)))
+    q = rng.standard_normal((Hkv * G, 128))
+    out = attention.attention_mixed(q, k16, v16, kc, kn, vc, vn, Pr)
+    for kv in range(Hkv):
+        K = torch.from_numpy(np.concatenate([k16[kv].astype(np.float64), attention.dequantise(kc[kv], kn[kv], Pr[kv])]))
+        V = torch.from_numpy(np.concatenate([v16[kv].astype(np.float64), attention.dequantise(vc[kv], vn[kv], Pr[kv])]))
+        Q = torch.from_numpy(q[kv * G:(kv + 1) * G])
+        ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None])[0]
+        np.testing.assert_allclose(out[kv * G:(kv + 1) * G], ref.numpy(), rtol=1e-12, atol=1e-12)
+    none = attention.attention_mixed(q, k16[:, :0], v16[:, :0], kc, kn, vc, vn, Pr)
+    np.testing.assert_allclose(none, attention.attention_rotated(q, kc, kn, vc, vn, Pr), atol=1e-12)
+    only = attention.attention_mixed(q, k16, v16, kc[:, :0], kn[:, :0], vc[:, :0], vn[:, :0], Pr)
+    for kv in range(Hkv):
+        K = torch.from_numpy(k16[kv].astype(np.float64))
+        V = torch.from_numpy(v16[kv].astype(np.float64))
+        Q = torch.from_numpy(q[kv * G:(kv + 1) * G])
+        ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None])[0]
+        np.testing.assert_allclose(only[kv * G:(kv + 1) * G], ref.numpy(), rtol=1e-12, atol=1e-12)
