@@ -30,13 +30,14 @@ if ROOT not in sys.path:
 
 BYTES_PER_TOKEN_HEAD = 100  # 48 B K codes + 2 B K norm + 48 B V codes + 2 B V norm
 BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
-# DRAM bytes (read + write) of one decode_kernel launch of the headline layer, from an ncu
-# capture (dram__bytes_read.sum + dram__bytes_write.sum, one 13.1 MB layer), valid only for the
-# kernel sources it was taken on: reported as roofline.traffic while their code hash matches.
-DECODE_TRAFFIC = {"sources": ["rotated_bit_kv_iq_b200/csrc/iq_decode.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
-                              "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"],
-                  "sha256": "b66e8e08151dd41a269d3d625650ec35aa53c10118573fe62a728c3915db9035",
-                  "bytes": 13215744}
+# DRAM bytes (read + write) of one decode_kernel launch of the headline layer and of the serving
+# layer, from ncu captures (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the
+# kernel sources they were taken on: reported as roofline.traffic while their code hash matches.
+DECODE_SOURCES = ["rotated_bit_kv_iq_b200/csrc/iq_decode_impl.cuh", "rotated_bit_kv_iq_b200/csrc/iq_decode.cu",
+                  "rotated_bit_kv_iq_b200/csrc/iq_decode_k3v3.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
+                  "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"]
+DECODE_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "a5fd3c8e32199eb65aa31b5b4068cf2a2a8fba8b6a724a2b1979c163e114ad28", "bytes": 13240832}
+SERVING_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "a5fd3c8e32199eb65aa31b5b4068cf2a2a8fba8b6a724a2b1979c163e114ad28", "bytes": 235557120 + 4064000}
 
 
 def kernel_source_hash(paths):
@@ -56,13 +57,14 @@ def kernel_source_hash(paths):
     return h.hexdigest()
 
 
-def decode_traffic():
+def decode_traffic(rec=None):
     """Captured DRAM bytes per decode launch, or None once the kernel sources have changed."""
+    rec = rec or DECODE_TRAFFIC
     try:
-        digest = kernel_source_hash(DECODE_TRAFFIC["sources"])
+        digest = kernel_source_hash(rec["sources"])
     except OSError:
         return None
-    return DECODE_TRAFFIC["bytes"] if digest == DECODE_TRAFFIC["sha256"] else None
+    return rec["bytes"] if digest == rec["sha256"] else None
 
 
 HEADLINE = "qwen30b_32k"
@@ -498,7 +500,7 @@ def bench_serving(steps, warmup, device, stream, seed=0, world=1, n_layers=0):
         "value": job_gbs(world, stack.bytes_per_step, ms), "unit": "GB/s", "ms_per_step": ms,
         "bytes_per_step": stack.bytes_per_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "decode_kernel, CUDA-graph step time / layers",
+                     "traffic": decode_traffic(SERVING_TRAFFIC), "kernel": "decode_kernel, CUDA-graph step time / layers",
                      "peak_kind": peak_kind, "bytes_per_launch": layer_bytes, "launch_ms": kern_ms},
         "launches": stack.L * DecodeStack.launches_per_layer * steps,
     }

@@ -411,7 +411,7 @@ __device__ __forceinline__ void process_tile(const uint8_t* __restrict__ st, uin
   }
   pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 1));
   pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 2));
-  const float gam = pmax > 0.f ? 127.f / pmax : 0.f;
+  const float gam = pmax > 0.f ? __fdividef(127.f, pmax) : 0.f;  // x = pv gam stays <= 127 (1-ulp quotient)
   const float ig = pmax > 0.f ? pmax * (1.0f / 127.0f) : 0.f;
   const int hl = P4 ? 8 * (t & 1) : 8 * t;
   const float igs = (P4 && t >= 2) ? 1.0f / 254.0f : 1.0f;  // P4: lo columns carry P' lo

@@ -9,8 +9,10 @@
 //
 // Two kernels per call.  prefix_kernel computes, on CUDA cores in fp32, the attention of every
 // query head of a kv head over a split of the fp16 prefix, exactly (fp16 inputs, fp32 products
-// and sums): online softmax over 32-token tiles in shared memory, then the value sum rotated
-// forward (R) and scaled to the packed kernel's units, written as extra split partials.  The
+// and sums): 32-token K and V tiles stream into shared memory by bulk copies, two rounds in
+// flight, each warp keeping the online softmax of one head over one stream of tiles; the value
+// sum is rotated forward (R) and scaled to the packed kernel's units, and written as extra split
+// partials.  The
 // fused decode step (decode_kernel) then appends the new token, attends over the packed tiles
 // from the prefix's tile onward (positions below len masked) and merges its own partials with
 // the extra ones before the single inverse rotation.
@@ -26,7 +28,9 @@
 namespace iq {
 
 constexpr int PX_THREADS = 256;
-constexpr int PX_ROW = D + 8;  // halves per token row in shared memory (16-byte rows, staggered banks)
+constexpr int PX_NB = 2;       // rounds of tiles in flight
+constexpr int PX_RMAX = 4;     // replicas (tile streams) per CTA
+constexpr int PX_TILE = TT * D * 2;  // bytes of one fp16 tile (32 tokens x 128)
 
 struct PrefixArgs {
   const __half* k;  // [batch][Hkv][max_len][128]
@@ -44,21 +48,27 @@ struct PrefixArgs {
   uint32_t* status;
 };
 
+// Replicas: tile streams per CTA; warp w works on head w % G of stream w / G.
+__host__ __device__ inline int px_replicas(int G) { return (HMAX / G) < PX_RMAX ? (HMAX / G) : PX_RMAX; }
+
 __global__ void __launch_bounds__(PX_THREADS) prefix_kernel(PrefixArgs a) {
   // wait before letting the decode kernel start, so that the kernel before this one is the only
   // one the decode kernel's early reads can overlap
   pdl_wait();
   pdl_launch_dependents();
-  constexpr int R_MAX = 8;
   __shared__ __align__(16) float sq[HMAX][D];
-  __shared__ float sml[R_MAX][HMAX][2];
+  __shared__ float sml[PX_RMAX][HMAX][2];
   __shared__ float sprm[256];
+  __shared__ __align__(8) uint64_t bars[PX_NB][PX_RMAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = a.g_real, R = HMAX / G;  // warp w: head w % G, replica w / G
-  // dynamic: R K tiles then R V tiles, [R][32][PX_ROW] halves each
-  extern __shared__ __align__(16) uint8_t px_smem[];
-  __half(*sk)[TT][PX_ROW] = reinterpret_cast<__half(*)[TT][PX_ROW]>(px_smem);
-  __half(*sv)[TT][PX_ROW] = reinterpret_cast<__half(*)[TT][PX_ROW]>(px_smem + (size_t)R * TT * PX_ROW * 2);
+  const int G = a.g_real, R = px_replicas(G);
+  const int h = warp % G, r = warp / G;  // r >= R: idle warp (group size 1 only)
+  // dynamic: [PX_NB][R] K tiles, then [PX_NB][R] V tiles, each [32][128] halves as stored
+  extern __shared__ __align__(128) uint8_t px_smem[];
+  auto ktile = [&](int buf, int rr) { return reinterpret_cast<__half*>(px_smem + (size_t)(buf * R + rr) * PX_TILE); };
+  auto vtile = [&](int buf, int rr) {
+    return reinterpret_cast<__half*>(px_smem + (size_t)(PX_NB * R + buf * R + rr) * PX_TILE);
+  };
   const int gid = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
   const int b = gid / a.n_kv_heads, kvh = gid % a.n_kv_heads;
   // prefix length, clamped as the decode kernel clamps it (0 <= len < ctx)
@@ -72,89 +82,114 @@ __global__ void __launch_bounds__(PX_THREADS) prefix_kernel(PrefixArgs a) {
   }
   const int ntiles = (p + TT - 1) / TT;
   const int t_lo = (int)((long long)split * ntiles / a.splits), t_hi = (int)((long long)(split + 1) * ntiles / a.splits);
+  const int n_rounds = (t_hi - t_lo + R - 1) / R;
+  const size_t seq_base = ((size_t)b * a.n_kv_heads + kvh) * a.max_len;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < PX_NB; ++i)
+      for (int rr = 0; rr < R; ++rr) mbar_init(&bars[i][rr], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  // round rd: tiles t_lo + rd R + rr, rr < R; each K and V tile is one bulk copy of its valid rows
+  auto issue_round = [&](int rd) {
+    const int buf = rd % PX_NB;
+    for (int rr = 0; rr < R; ++rr) {
+      const int tile = t_lo + rd * R + rr;
+      const int rows = tile < t_hi ? min(TT, p - TT * tile) : 0;
+      mbar_arrive_expect_tx(&bars[buf][rr], 2u * rows * D * 2);
+      if (rows > 0) {
+        bulk_g2s(ktile(buf, rr), a.k + (seq_base + (size_t)TT * tile) * D, rows * D * 2, &bars[buf][rr]);
+        bulk_g2s(vtile(buf, rr), a.v + (seq_base + (size_t)TT * tile) * D, rows * D * 2, &bars[buf][rr]);
+      }
+    }
+  };
+  if (threadIdx.x == 0)
+    for (int rd = 0; rd < min(PX_NB, n_rounds); ++rd) issue_round(rd);
 
   // queries of the group, scaled so that q.k gives scores in log2 units: log2(e) / sqrt(128)
   const float qs = kLog2e * 0.08838834764831845f;
   for (int i = threadIdx.x; i < HMAX * D; i += PX_THREADS) {
-    const int h = i / D, x = i % D;
+    const int hh = i / D, x = i % D;
     float val = 0.f;
-    if (h < G) {
-      const size_t row = ((size_t)b * a.n_q_heads + (size_t)kvh * G + h) * D + x;
+    if (hh < G) {
+      const size_t row = ((size_t)b * a.n_q_heads + (size_t)kvh * G + hh) * D + x;
       val = a.q_f32 ? ((const float*)a.q)[row] : __half2float(((const __half*)a.q)[row]);
     }
-    sq[h][x] = val * qs;
+    sq[hh][x] = val * qs;
   }
   if (threadIdx.x < params_per_head(a.rot) / 4)
     reinterpret_cast<float4*>(sprm)[threadIdx.x] =
         reinterpret_cast<const float4*>(a.params_layer + (size_t)kvh * params_per_head(a.rot))[threadIdx.x];
-
-  const int h = warp % G, r = warp / G;
-  float m = -CUDART_INF_F, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const size_t seq_base = ((size_t)b * a.n_kv_heads + kvh) * a.max_len;
-  for (int base = t_lo; base < t_hi; base += R) {
-    __syncthreads();  // the previous tiles are consumed (and sq, sprm written, on the first pass)
-    // the R tiles base .. base+R-1: rows of 16-byte pieces, all threads
-    for (int i = threadIdx.x; i < R * TT * (D / 8); i += PX_THREADS) {
-      const int rr = i / (TT * (D / 8)), t = (i / (D / 8)) % TT, piece = i % (D / 8);
-      const int pos = TT * (base + rr) + t;
-      uint4 kk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-      if (base + rr < t_hi && pos < p) {
-        kk = reinterpret_cast<const uint4*>(a.k + (seq_base + pos) * D)[piece];
-        vv = reinterpret_cast<const uint4*>(a.v + (seq_base + pos) * D)[piece];
-      }
-      *reinterpret_cast<uint4*>(&sk[rr][t][8 * piece]) = kk;
-      *reinterpret_cast<uint4*>(&sv[rr][t][8 * piece]) = vv;
-    }
-    __syncthreads();
-    const int tile = base + r;
-    if (tile < t_hi) {
-      // score of token `lane`: coordinates visited from a lane-dependent start (no bank conflicts)
-      float s = 0.f;
-#pragma unroll 8
-      for (int c2 = 0; c2 < D / 2; ++c2) {
-        const int x = 2 * ((c2 + lane) & (D / 2 - 1));
-        const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&sk[r][lane][x]));
-        s = fmaf(sq[h][x], kf.x, s);
-        s = fmaf(sq[h][x + 1], kf.y, s);
-      }
-      const int pos = TT * tile + lane;
-      if (pos >= p) s = -CUDART_INF_F;
-      float mx = s;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_new = fmaxf(m, mx);
-      const float sc = (m == -CUDART_INF_F) ? 0.f : exp2f(m - m_new);
-      const float pw = (s == -CUDART_INF_F) ? 0.f : exp2f(s - m_new);
-      float ps = pw;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-      l = l * sc + ps;
-      m = m_new;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] *= sc;
-      // values: lane holds coordinates 4 lane .. 4 lane + 3
-#pragma unroll 4
-      for (int t = 0; t < TT; ++t) {
-        const float pt = __shfl_sync(0xffffffffu, pw, t);
-        const uint2 raw = *reinterpret_cast<const uint2*>(&sv[r][t][4 * lane]);
-        const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-        const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-        acc[0] = fmaf(pt, v0.x, acc[0]);
-        acc[1] = fmaf(pt, v0.y, acc[1]);
-        acc[2] = fmaf(pt, v1.x, acc[2]);
-        acc[3] = fmaf(pt, v1.y, acc[3]);
-      }
-    }
-  }
-  // merge the replicas of each head (shared memory), then R, scale and write the partial
   __syncthreads();
-  float* so = reinterpret_cast<float*>(&sk[0][0][0]);  // [R][G][128] floats, reused
-  if (lane == 0) {
-    sml[r][h][0] = m;
-    sml[r][h][1] = l;
-  }
+
+  float m = -CUDART_INF_F, l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+  bool ok = true;
+  for (int rd = 0; rd < n_rounds; ++rd) {
+    const int buf = rd % PX_NB, tile = t_lo + rd * R + r;
+    if (r < R && tile < t_hi) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[buf][r], (rd / PX_NB) & 1, a.status));
+      const int n_valid = min(TT, p - TT * tile);  // rows of this tile in the prefix
+      const __half* kt = ktile(buf, r);
+      const __half* vt = vtile(buf, r);
+      if (ok) {
+        // score of token `lane`: coordinates visited from a lane-dependent start, so the 32 lanes
+        // read 32 different banks of their 256-byte rows
+        float s = 0.f;
+#pragma unroll 8
+        for (int c2 = 0; c2 < D / 2; ++c2) {
+          const int x = 2 * ((c2 + lane) & (D / 2 - 1));
+          const float2 kf = __half22float2(*reinterpret_cast<const __half2*>(kt + lane * D + x));
+          const float2 qv = *reinterpret_cast<const float2*>(&sq[h][x]);
+          s = fmaf(qv.x, kf.x, s);
+          s = fmaf(qv.y, kf.y, s);
+        }
+        if (lane >= n_valid) s = -CUDART_INF_F;  // rows past the prefix were not copied
+        float mx = s;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) so[(r * G + h) * D + 4 * lane + i] = acc[i];
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = fmaxf(m, mx);
+        const float sc = (m == -CUDART_INF_F) ? 0.f : exp2f(m - m_new);
+        const float pw = (s == -CUDART_INF_F) ? 0.f : exp2f(s - m_new);
+        float ps = pw;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l = l * sc + ps;
+        m = m_new;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] *= sc;
+        // values: lane holds coordinates 4 lane .. 4 lane + 3; only the copied rows are read
+        for (int t = 0; t < n_valid; ++t) {
+          const float pt = __shfl_sync(0xffffffffu, pw, t);
+          const uint2 raw = *reinterpret_cast<const uint2*>(vt + t * D + 4 * lane);
+          const float2 v0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+          const float2 v1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+          acc[0] = fmaf(pt, v0.x, acc[0]);
+          acc[1] = fmaf(pt, v0.y, acc[1]);
+          acc[2] = fmaf(pt, v1.x, acc[2]);
+          acc[3] = fmaf(pt, v1.y, acc[3]);
+        }
+      }
+    }
+    __syncthreads();  // every stream is done with buffer buf
+    if (threadIdx.x == 0 && rd + PX_NB < n_rounds) issue_round(rd + PX_NB);
+  }
+  // leave no bulk copy in flight (only after a timed-out wait can one be pending)
+  if (!__syncthreads_and(ok) && threadIdx.x == 0)
+    for (int rd = 0; rd < n_rounds; ++rd)
+      for (int rr = 0; rr < R; ++rr)
+        if (t_lo + rd * R + rr < t_hi) mbar_wait(&bars[rd % PX_NB][rr], (rd / PX_NB) & 1, nullptr);
+  // merge the streams of each head (shared memory), then R, scale and write the partial
+  __syncthreads();
+  float* so = reinterpret_cast<float*>(px_smem);  // [R][G][128] floats, over the tile buffers
+  if (r < R) {
+    if (lane == 0) {
+      sml[r][h][0] = m;
+      sml[r][h][1] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) so[(r * G + h) * D + 4 * lane + i] = acc[i];
+  }
   __syncthreads();
   if (r == 0) {
     float M = -CUDART_INF_F;
@@ -214,10 +249,10 @@ int launch_prefix(const LayerView& v, const void* k16, const void* v16, const in
   a.part_o = w.part_o;
   a.extra_base = extra_base;
   a.status = v.status;
-  const size_t smem = (size_t)(HMAX / a.g_real) * 2 * TT * PX_ROW * sizeof(__half);
+  const size_t smem = (size_t)2 * PX_NB * px_replicas(a.g_real) * PX_TILE;
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HMAX * 2 * TT * PX_ROW * 2);
+    cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2 * PX_NB * PX_RMAX * PX_TILE);
   });
   return (int)launch_pdl(prefix_kernel, dim3(batch * v.n_kv_heads * splits), dim3(PX_THREADS), smem,
                          (cudaStream_t)stream, a);
