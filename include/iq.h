@@ -89,8 +89,8 @@ typedef struct CUstream_st* iq_stream_t; /* same type as cudaStream_t */
 typedef enum {
   IQ_OK = 0,
   IQ_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, inconsistent shapes */
-  IQ_ERR_UNSUPPORTED = 2, /* head_dim != 128, GQA group size not 1, 2, 4 or 8, bad dtype, code widths
-                             or rotation variant not supported */
+  IQ_ERR_UNSUPPORTED = 2, /* head_dim != 128, GQA group size above 8, bad dtype, code widths or
+                             rotation variant not supported */
   IQ_ERR_CAPACITY = 3,    /* a host-known size exceeds the cache's capacity */
   IQ_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than iq_decode_workspace_size */
   IQ_ERR_ALIGNMENT = 5,   /* a device pointer is not 16-byte aligned (workspace: 256) */
@@ -203,7 +203,8 @@ size_t iq_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_h
  *                  zero-filled before its first use (see iq_decode_workspace_size); calls
  *                  that overlap on the GPU must not share one.
  *   batch        : at most 2048 (IQ_ERR_UNSUPPORTED above).
- * q head h reads kv head h / (n_q_heads / n_kv_heads); that group size must be 1, 2, 4 or 8.
+ * q head h reads kv head h / (n_q_heads / n_kv_heads); that group size must be 1 .. 8 (every call
+ * below has the same limit).
  * out[b][h] = sum_t softmax_t(<q, K_t>/sqrt(128)) V_t with K_t, V_t the dequantised
  * vectors n * R^T c[codes] / sqrt(128), computed without forming them: q is rotated once,
  * scores and the value sum are formed in the rotated basis from codes and norms,

@@ -202,7 +202,7 @@ iq_status iq_decode_attention(const iq_cache* cache, int32_t layer, const void* 
   if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return IQ_ERR_UNSUPPORTED;  // at most 8 query heads per kv head (one mma row block)
   if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
   if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
   if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(ctx_len_dev, 4))
@@ -230,7 +230,7 @@ iq_status iq_decode_step(const iq_cache* cache, int32_t layer, const void* q_dev
   if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return IQ_ERR_UNSUPPORTED;  // at most 8 query heads per kv head (one mma row block)
   if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
   if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
   if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(ctx_len_dev, 4) ||
@@ -268,7 +268,7 @@ iq_status iq_decode_step_deferred(const iq_cache* cache, int32_t layer, const iq
   if (batch > DECODE_MAX_BATCH) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return IQ_ERR_UNSUPPORTED;  // at most 8 query heads per kv head (one mma row block)
   if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
   if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
   if (!aligned(q_dev, 16) || !aligned(out_dev, 16) || !aligned(params_dev, 16) || !aligned(ctx_len_dev, 4) ||
@@ -303,7 +303,7 @@ iq_status iq_prefill_attention(const iq_cache* cache, int32_t layer, const void*
   if (q_dtype != IQ_F16 && q_dtype != IQ_F32) return IQ_ERR_UNSUPPORTED;
   if (n_q_heads % cache->n_kv_heads != 0) return IQ_ERR_INVALID_ARG;
   const int G = n_q_heads / cache->n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return IQ_ERR_UNSUPPORTED;
+  if (G < 1 || G > 8) return IQ_ERR_UNSUPPORTED;  // at most 8 query heads per kv head (one mma row block)
   if (!cache->block_table_dev && batch > cache->n_pages) return IQ_ERR_CAPACITY;
   if ((int64_t)max_ctx > seq_capacity(cache)) return IQ_ERR_CAPACITY;
   if ((int64_t)batch * cache->n_kv_heads * ((n_tokens + 7) / 8) > (int64_t)1 << 24) return IQ_ERR_UNSUPPORTED;

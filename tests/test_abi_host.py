@@ -133,7 +133,7 @@ def test_calls_reject_unsupported_formats(lib):
 def test_decode_rejects_bad_arguments(lib):
     assert _dec(None) == B.IQ_ERR_INVALID_ARG
     assert _dec(_fake_cache(head_dim=96)) == B.IQ_ERR_UNSUPPORTED
-    assert _dec(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED          # group size 3
+    assert _dec(_fake_cache(), hq=18) == B.IQ_ERR_UNSUPPORTED         # group size 9
     assert _dec(_fake_cache(), hq=5) == B.IQ_ERR_INVALID_ARG          # not a multiple of Hkv
     assert _dec(_fake_cache(), dtype=7) == B.IQ_ERR_UNSUPPORTED
     assert _dec(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
@@ -160,7 +160,7 @@ def test_decode_step_rejects_bad_arguments(lib):
     assert step(_fake_cache(), k=0x58008) == B.IQ_ERR_ALIGNMENT
     assert step(_fake_cache(), max_ctx=0) == B.IQ_ERR_INVALID_ARG   # the new token needs a slot
     assert step(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
-    assert step(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert step(_fake_cache(), hq=18) == B.IQ_ERR_UNSUPPORTED
     assert step(_fake_cache(), ws_bytes=8) == B.IQ_ERR_WORKSPACE
     assert step(_fake_cache(head_dim=64)) == B.IQ_ERR_UNSUPPORTED
 
@@ -174,7 +174,7 @@ def test_prefill_rejects_bad_arguments(lib):
 
     assert pre(_fake_cache(), n_tok=40) == B.IQ_ERR_INVALID_ARG      # max_ctx below the chunk
     assert pre(_fake_cache(), max_ctx=65) == B.IQ_ERR_CAPACITY
-    assert pre(_fake_cache(), hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert pre(_fake_cache(), hq=18) == B.IQ_ERR_UNSUPPORTED
     assert pre(_fake_cache(), hq=5) == B.IQ_ERR_INVALID_ARG
     assert pre(_fake_cache(), dtype=3) == B.IQ_ERR_UNSUPPORTED
     assert pre(_fake_cache(), start=None) == B.IQ_ERR_INVALID_ARG
@@ -202,7 +202,7 @@ def test_deferred_step_rejects_bad_arguments(lib):
     assert step(_fake_cache(), B.iq_fp16_prefix(0x100008, 0x200000, 0x300000, 16)) == B.IQ_ERR_ALIGNMENT
     assert step(_fake_cache(), B.iq_fp16_prefix(0x100000, 0x200000, 0x300000, -1)) == B.IQ_ERR_INVALID_ARG
     assert step(_fake_cache(), good, max_ctx=65) == B.IQ_ERR_CAPACITY
-    assert step(_fake_cache(), good, hq=6) == B.IQ_ERR_UNSUPPORTED
+    assert step(_fake_cache(), good, hq=18) == B.IQ_ERR_UNSUPPORTED
     assert step(_fake_cache(), good, ws_bytes=64) == B.IQ_ERR_WORKSPACE
     assert step(_fake_cache(k_bits=1), good) == B.IQ_ERR_UNSUPPORTED
     assert B.iq_decode_deferred_workspace_size(1, 32, 8, 8704, 8192) > B.iq_decode_workspace_size(1, 32, 8, 8704)

@@ -257,10 +257,11 @@ def test_decode_gqa8_qwen_32k_layer_full():
     assert err < TOL, err
 
 
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_decode_ragged_paged_batch(G):
-    """Ragged contexts (0, 1, 15, 17, 300, 1000) over shuffled 64-token pages, every supported
-    group size (both mma layouts: G <= 4 packs the lower terms into the free rows and columns)."""
+    """Ragged contexts (0, 1, 15, 17, 300, 1000) over shuffled 64-token pages, every group size
+    1 .. 8 (both mma layouts: G <= 4 packs the lower terms into the free rows and columns; groups
+    that do not fill a layout leave rows unused)."""
     Hkv = 2
     Hq = G * Hkv
     ctx = [0, 1, 15, 17, 300, 1000]
@@ -414,7 +415,7 @@ def _check_appended(cache, layer, b, pos, knew_b, vnew_b, P_layer, rec):
             _check_codes(codes[h], n16[h], e, f"b={b} kv={kv} h={h}", cap=False, record=rec)
 
 
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_decode_step_matches_oracle(G):
     """Fused append + attention: new tokens at odd and even positions, page boundaries, ctx = 1."""
     ctx = [1, 2, 64, 65, 129, 700]
