@@ -78,7 +78,6 @@ struct Workspace {
 };
 Workspace carve_workspace(void* ws, int batch, int n_kv_heads, int extra_slots = 0);
 int workspace_base_slots(int batch, int n_kv_heads);  // partial slots of the CTAs; extra slots follow
-int resident_per_sm(const void* fn, size_t smem, int threads);
 
 struct DecArgs {
   LayerView v;

@@ -154,15 +154,17 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
       for (int i = 0; i < BITS; ++i) dst[i] = make_uint4(rec[4 * i], rec[4 * i + 1], rec[4 * i + 2], rec[4 * i + 3]);
     }
   } else {
-    // V block (16 tokens = 16 consecutive lanes): token u = lane mod 16 owns nibbles j and
-    // j+4 of the selector words of chunks (g, tq, h), tq = (u mod 8)/2, j = 2 (u/8) + (u mod 2);
-    // nibble j of selector word w holds coordinate 32w + g + 8h and nibble j+4 coordinate
-    // 32w + 16 + g + 8h.  Packing keeps nibble positions, so the four tokens of a quad (lanes
-    // u, u^1, u^8, u^9) pack their own nibbles, OR the storage words together and member j
-    // stores the two chunks (h = 0, 1) of g = 2j, 2j+1 (2 BITS contiguous words each g).
+    // V block (16 tokens = 16 consecutive lanes).  Chunk (g, tq, h) holds the codes of the
+    // quad of tokens u with (u mod 8)/2 = tq (lanes u, u^1, u^8, u^9; token u is quad member
+    // m = 2 (u/8) + (u mod 2)): nibble m of selector word w = coordinate 32w + g + 8h, nibble
+    // m + 4 = coordinate 32w + 16 + g + 8h.  Member m stores the chunks of g = 2m, 2m+1, whose
+    // codes are byte m of every code word cw[r] of the four members: a 4 x 4 byte transpose
+    // in the quad (two shuffles and two permutes per word) gives it T[r], byte s = byte m of
+    // member s's cw[r].  Packing keeps nibble positions, so the selector words are the bytes'
+    // low (g even) or high (g odd) nibbles side by side.
     const unsigned lane = threadIdx.x & 31;
-    const int u = lane & 15, tq = (u & 7) >> 1, j = 2 * (u >> 3) + (u & 1);
-    uint32_t qmask = active ? ((0xFu << (4 * j)) | (0xFu << (16 + 4 * j))) : 0u;
+    const int u = lane & 15, tq = (u & 7) >> 1, m = 2 * (u >> 3) + (u & 1);
+    uint32_t qmask = active ? ((0xFu << (4 * m)) | (0xFu << (16 + 4 * m))) : 0u;
     qmask |= __shfl_xor_sync(0xffffffffu, qmask, 1);
     qmask |= __shfl_xor_sync(0xffffffffu, qmask, 8);
     // the storing member may lie outside the launch: take the block's page from an active one
@@ -170,27 +172,31 @@ encode_kernel(LayerView v, const __half* __restrict__ k_src, const __half* __res
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 1));
     qpage = max(qpage, __shfl_xor_sync(0xffffffffu, qpage, 8));
     uint8_t* blk = v_block(v, qpage < 0 ? 0 : qpage, head, slot);
-#pragma unroll 1
-    for (int g = 0; g < 8; ++g) {  // rolled: keeps the kernel's code small
+    const uint32_t sel1 = (u & 1) ? 0x3715u : 0x6240u, sel2 = (u >> 3) ? 0x3276u : 0x5410u;
+    uint32_t T[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const uint32_t x = active ? cw[r] : 0u;  // members outside the launch contribute nothing
+      const uint32_t w1 = prmt(x, __shfl_xor_sync(0xffffffffu, x, 1), sel1);
+      T[r] = prmt(w1, __shfl_xor_sync(0xffffffffu, w1, 8), sel2);
+    }
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
       uint32_t wd[2 * BITS];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        // codes of coordinates 16m + g + 8h: nibble g of cw[2m + h]
         uint32_t sw[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const uint32_t a = (cw[4 * w + h] >> (4 * g)) & 0xFu, c = (cw[4 * w + 2 + h] >> (4 * g)) & 0xFu;
-          sw[w] = active ? ((a << (4 * j)) | (c << (16 + 4 * j))) : 0u;
+          const uint32_t xa = (gg ? T[4 * w + h] >> 4 : T[4 * w + h]) & 0x0F0F0F0Fu;
+          const uint32_t xb = (gg ? T[4 * w + 2 + h] >> 4 : T[4 * w + 2 + h]) & 0x0F0F0F0Fu;
+          sw[w] = prmt(xa | (xa >> 4), xb | (xb >> 4), 0x6420u);
         }
 #pragma unroll
-        for (int k = 0; k < BITS; ++k) {
-          uint32_t part = pack_word<BITS>(k, sw[0], sw[1], sw[2], sw[3]);
-          part |= __shfl_xor_sync(0xffffffffu, part, 1);
-          part |= __shfl_xor_sync(0xffffffffu, part, 8);
-          wd[BITS * h + k] = part;
-        }
+        for (int k = 0; k < BITS; ++k) wd[BITS * h + k] = pack_word<BITS>(k, sw[0], sw[1], sw[2], sw[3]);
       }
-      if (j == (g >> 1) && qmask != 0u) {
+      if (qmask != 0u) {
+        const int g = 2 * m + gg;
         uint32_t* dst = reinterpret_cast<uint32_t*>(blk + 2 * chunk_bytes(BITS) * (4 * g + tq));
         if (qmask == 0xFFFFFFFFu) {
           uint2* d2 = reinterpret_cast<uint2*>(dst);

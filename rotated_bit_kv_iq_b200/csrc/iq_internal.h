@@ -115,6 +115,8 @@ int decode_ctas(int batch, int n_kv_heads, int max_ctx, int resident_per_sm);
 size_t decode_workspace_bytes(int batch, int n_q_heads, int n_kv_heads, int max_ctx, int extra_slots = 0);
 int prefix_splits(int batch, int n_kv_heads, int max_len, int n_sm);
 int sm_count();
+// CTAs of kernel fn with the given dynamic shared memory and block size that fit on one SM.
+int resident_per_sm(const void* fn, size_t smem, int threads);
 int launch_prefix(const LayerView& v, const void* k16, const void* v16, const int32_t* len, int max_len,
                   const int32_t* ctx_len, int max_ctx, const void* q, int q_f32, int batch, int n_q_heads,
                   const float* params_layer, const KernelConsts& kc, void* workspace, int splits, int extra_base,
