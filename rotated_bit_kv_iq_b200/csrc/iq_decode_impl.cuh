@@ -49,12 +49,15 @@ constexpr int SO_STRIDE = 132;              // floats per (warp, head) row of th
 constexpr int QF_WORDS = 28;  // query fragment words per lane: 16 (hi, lo) + 8 (lo2) + 4 (bank skew)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Tiles in flight per warp by default: three while a tile record is at most 3200 bytes.
+IQ_HD constexpr int dec_nslot(int kb, int vb) { return tile_bytes(kb, vb) <= 3200 ? 3 : 2; }
+
 // Shared memory of one decode CTA for code widths (KB, VB).  A ring slot holds one tile record as
-// stored (one bulk copy); each warp has NSLOT of them.
-template <int KB, int VB>
+// stored (one bulk copy); each warp has NS of them.
+template <int KB, int VB, int NS = dec_nslot(KB, VB)>
 struct DecSmem {
   static constexpr int SLOT_BYTES = tile_bytes(KB, VB);
-  static constexpr int NSLOT = SLOT_BYTES <= 3200 ? 3 : 2;                // tiles in flight per warp
+  static constexpr int NSLOT = NS;                                        // tiles in flight per warp
   static constexpr int SL_K = 0, SL_V = tr_v(KB), SL_KN = tr_kn(KB, VB), SL_VN = tr_vn(KB, VB);
   static constexpr int ring = 0;                                          // [warp][slot] tiles
   static constexpr int so = ring + DEC_WARPS * NSLOT * SLOT_BYTES;        // float [warp-4][head][SO_STRIDE]
@@ -481,10 +484,10 @@ __device__ __forceinline__ void rotate_query_row(const void* q, int q_f32, size_
   if (live) {
     const size_t row = row0 + 4 * lane;
     if (q_f32) {
-      const float4 f = *reinterpret_cast<const float4*>((const float*)q + row);
+      const float4 f = __ldcg(reinterpret_cast<const float4*>((const float*)q + row));
       x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
     } else {
-      const uint2 u = *reinterpret_cast<const uint2*>((const __half*)q + row);
+      const uint2 u = __ldcg(reinterpret_cast<const uint2*>((const __half*)q + row));
       const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
       const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
       x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
@@ -621,9 +624,9 @@ __device__ __forceinline__ void merge_group(const DecArgs& a, const Seg& seg, in
 }
 
 // ------------------------------------------------------------------ the kernel
-template <bool FUSED, bool P4, int KB, int VB>
+template <bool FUSED, bool P4, int KB, int VB, int NS = dec_nslot(KB, VB)>
 __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
-  using DecSmem = iq::DecSmem<KB, VB>;
+  using DecSmem = iq::DecSmem<KB, VB, NS>;
   constexpr int NSLOT = DecSmem::NSLOT, SLOT_BYTES = DecSmem::SLOT_BYTES;
   pdl_launch_dependents();
   if (!FUSED) pdl_wait();  // a plain call may read anything the previous kernel wrote
@@ -717,7 +720,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       const char* p = a.q_f32 ? (const char*)((const float*)a.q + row) : (const char*)((const __half*)a.q + row);
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * (threadIdx.x & 1) * (a.q_f32 ? 2 : 1)));
     }
-    pdl_wait();
+    // After an fp16 prefix's kernel (a.n_extra > 0) the wait moves to the final merge, the first
+    // read of what that kernel writes (its partials): it starts only once it has waited for the
+    // kernel before it, so q and the new token (read through L2) are already final.  The tile
+    // work of this kernel then runs while the prefix's kernel is still running.
+    if (a.n_extra == 0) pdl_wait();
   }
 
   // ---- outputs of groups with no tiles (empty context): zeros
@@ -884,6 +891,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 
   // ---- final merges: for every group of the run, the heads given to this CTA, once all of
   // the group's partials are in (every CTA has written all of its partials before waiting)
+  if (FUSED && a.n_extra > 0) pdl_wait();  // the fp16 prefix's partials
   x = c0;
   while (x < c1) {
     const Seg seg = segment_at(a, pre, B, Hkv, x, c1);
@@ -961,17 +969,21 @@ int launch_decode_kv(const LayerView& v, const void* q, int q_f32, int batch, in
   static std::once_flag attr_once;
   std::call_once(attr_once, [] {
     const int maxb = (int)DecSmem<KB, VB>::bytes(DECODE_MAX_BATCH);
-    void (*ks[4])(DecArgs) = {decode_kernel<false, false, KB, VB>, decode_kernel<false, true, KB, VB>,
-                              decode_kernel<true, false, KB, VB>, decode_kernel<true, true, KB, VB>};
+    void (*ks[6])(DecArgs) = {decode_kernel<false, false, KB, VB>, decode_kernel<false, true, KB, VB>,
+                              decode_kernel<true, false, KB, VB>,  decode_kernel<true, true, KB, VB>,
+                              decode_kernel<true, false, KB, VB, 2>, decode_kernel<true, true, KB, VB, 2>};
     for (auto k : ks) {
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
       cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     }
   });
   const bool fused = k_new != nullptr;
-  auto kern = fused ? (a.g_real <= 4 ? decode_kernel<true, true, KB, VB> : decode_kernel<true, false, KB, VB>)
-                    : (a.g_real <= 4 ? decode_kernel<false, true, KB, VB> : decode_kernel<false, false, KB, VB>);
-  const size_t smem = DecSmem<KB, VB>::bytes(batch);
+  // After an fp16 prefix's kernel: two ring slots per warp, so that a CTA fits on an SM beside
+  // two of that kernel's CTAs and the two kernels overlap (the packed tail is short)
+  auto kern = def ? (a.g_real <= 4 ? decode_kernel<true, true, KB, VB, 2> : decode_kernel<true, false, KB, VB, 2>)
+              : fused ? (a.g_real <= 4 ? decode_kernel<true, true, KB, VB> : decode_kernel<true, false, KB, VB>)
+                      : (a.g_real <= 4 ? decode_kernel<false, true, KB, VB> : decode_kernel<false, false, KB, VB>);
+  const size_t smem = def ? DecSmem<KB, VB, 2>::bytes(batch) : DecSmem<KB, VB>::bytes(batch);
   const int ctas = decode_ctas(batch, v.n_kv_heads, max_ctx, resident_per_sm((const void*)kern, smem, DEC_THREADS));
   if (ctas == 0) return (int)cudaErrorInvalidConfiguration;
   return (int)launch_pdl(kern, dim3(ctas), dim3(DEC_THREADS), smem, (cudaStream_t)stream, a);

@@ -52,8 +52,8 @@ struct PrefixArgs {
 __host__ __device__ inline int px_replicas(int G) { return (HMAX / G) < PX_RMAX ? (HMAX / G) : PX_RMAX; }
 
 __global__ void __launch_bounds__(PX_THREADS) prefix_kernel(PrefixArgs a) {
-  // wait before letting the decode kernel start, so that the kernel before this one is the only
-  // one the decode kernel's early reads can overlap
+  // Wait before letting the decode kernel start: it reads q and the new token (through L2)
+  // before its own wait, relying on the kernel before this one having completed by then.
   pdl_wait();
   pdl_launch_dependents();
   __shared__ __align__(16) float sq[HMAX][D];

@@ -407,7 +407,7 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
                                                    int side, int page, int slot, const float Mp[4][4],
                                                    const SideConsts& sc) {
   const int lane = threadIdx.x & 31;
-  const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
+  const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(src + 4 * lane));  // through L2 (see decode_kernel)
   const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
   const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
   float x[4] = {f0.x, f0.y, f1.x, f1.y};
