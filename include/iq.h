@@ -261,7 +261,10 @@ size_t iq_decode_deferred_workspace_size(int32_t batch, int32_t n_q_heads, int32
  * position len[b] on (earlier positions of that tile are ignored).  Other arguments, results and
  * errors as for iq_decode_step, with the workspace of iq_decode_deferred_workspace_size.  Two
  * kernels: the prefix's attention (split partials, rotated forward into the packed basis), then
- * the fused step, which merges both before its single inverse rotation. */
+ * the fused step, which merges both before its single inverse rotation.  Ordering: the first
+ * kernel waits for the kernel issued before the call before it reads anything; the second
+ * starts once the first is past that wait, attends over the packed tail while the first is
+ * still running, and waits for it only before merging its partials. */
 iq_status iq_decode_step_deferred(const iq_cache* cache, int32_t layer, const iq_fp16_prefix* prefix, const void* q_dev,
                                   iq_dtype q_dtype, const void* k_new_dev, const void* v_new_dev, int32_t batch,
                                   int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
