@@ -56,6 +56,15 @@ static SideConsts make_side(int bits) {
     sc.lut_lo[k >> 2] |= (uint32_t)(uint8_t)(int8_t)lo[k] << (8 * (k & 3));
   }
   sc.alpha8 = (float)alpha8;
+  for (int k = 0; k < n; ++k) {
+    const __half h = __float2half_rn((float)cb.level[k]);
+    const __half l = __float2half_rn((float)(cb.level[k] - (double)__half2float(h)));
+    const uint16_t bits16[2] = {__half_as_ushort(h), __half_as_ushort(l)};
+    for (int t = 0; t < 2; ++t) {
+      sc.f16_lb[t][k >> 2] |= (uint32_t)(bits16[t] & 0xFFu) << (8 * (k & 3));
+      sc.f16_hb[t][k >> 2] |= (uint32_t)(bits16[t] >> 8) << (8 * (k & 3));
+    }
+  }
   return sc;
 }
 

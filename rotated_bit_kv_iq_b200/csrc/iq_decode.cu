@@ -131,12 +131,12 @@ int launch_decode_deferred(const LayerView& v, const void* q, int q_f32, const v
                   v_new, &def);
 }
 
-// Prefill workspace: per (group, split, query token, head) one (m, l) pair and one 128-float O.
+// Prefill workspace: per (group, split, query row) one (m, l) pair and one 128-float O; the
+// query rows of a group depend on the group size, which the size query does not know, so the
+// largest over group sizes 1 .. 8.
 size_t prefill_workspace_bytes(int batch, int n_tok, int n_kv_heads, int max_ctx) {
-  const int n_qblk = (n_tok + PF_QB - 1) / PF_QB;
-  const int groups = batch * n_kv_heads * n_qblk;
-  const int splits = prefill_splits(groups, (max_ctx + TT - 1) / TT, sm_count());
-  const size_t rows = (size_t)groups * splits * PF_QB * HMAX;
+  size_t rows = 0;
+  for (int g = 1; g <= HMAX; ++g) rows = std::max(rows, prefill_rows(batch, n_tok, n_kv_heads, max_ctx, g, sm_count(), nullptr));
   return align256(rows * sizeof(float2)) + align256(rows * D * sizeof(float));
 }
 

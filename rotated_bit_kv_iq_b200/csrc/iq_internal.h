@@ -65,6 +65,10 @@ struct SideConsts {
   uint32_t lut_lo[4];
   float alpha8;
   int bits;
+  // the N(0,1) centroids as binary16 pairs c = c_hi + c_lo: low bytes (f16_lb) and high bytes
+  // (f16_hb) of term t (0 = hi, 1 = lo) of entry k at byte k % 4 of word k / 4
+  uint32_t f16_lb[2][4];
+  uint32_t f16_hb[2][4];
 };
 struct KernelConsts {
   SideConsts k, v;

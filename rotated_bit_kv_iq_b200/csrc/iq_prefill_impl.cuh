@@ -1,4 +1,4 @@
-// Chunked-prefill attention directly on the packed cache: many query tokens per KV tile.
+// Chunked-prefill attention directly on the packed cache, on the 5th-generation tensor cores.
 //
 // The packed pipeline of "RotaryQuant" (rebasdaily.com, section "妙处不只是压缩，而是不再展开"),
 // applied to a chunk of new prompt tokens instead of one decode token ("RotorQuant",
@@ -6,23 +6,43 @@
 // these caches).  The chunk's own K/V have been appended to the cache first; query token i of
 // sequence b sits at position start[b] + i and attends causally to positions 0 .. start[b] + i.
 //
-// Work: groups (sequence, kv head, block of QB = 8 query tokens), each split over `splits` CTAs
-// along the KV tiles 0 .. ceil(kv_end / 32) - 1 (kv_end = the block's last position + 1).  The CTA
-// streams its tiles through a ring in shared memory with bulk copies; every tile is used by all
-// eight warps, warp w being query token w of the block (its rotated query in its own fragment
-// buffer, its own causal limit, its own online softmax), so the packed K/V are read once per
-// eight query tokens and expanded by each warp on the tensor cores exactly as in decode.  Each
-// warp writes one partial (m, l, O) per head; a second kernel merges the splits, normalises and
-// applies the inverse rotation.
+// Many query tokens share every key, so the contractions are dense: one CTA takes 128 query
+// rows (TQ = 128 / G tokens x the G query heads of one kv head) and streams the keys in steps
+// of 64 (two tile records), with the math on tcgen05 MMAs (M = 128) and fp32 accumulators in
+// tensor memory:
+//   * the rotated queries, scaled per row by a power of two to |q| <= 1, are split into binary16
+//     hi + lo terms once; the step's K codes become binary16 centroid terms c_hi + c_lo in
+//     shared memory (byte-permute table lookups), and S = Q K^T is the sum of the three
+//     products hi.hi, lo.hi and hi.lo (K = 128 coordinates);
+//   * the online softmax runs one thread per row on S read back from tensor memory; the
+//     probabilities times the V norms, P' = 2^(s - m) n_v, are written to shared memory as
+//     binary16 hi + lo terms;
+//   * the V codes become the centroid terms of V^T (coordinates as rows), and O^T = V^T P'^T
+//     (M = 128 coordinates, N = 128 rows, K = 64 keys; products V_hi P_hi, V_lo P_hi and
+//     V_hi P_lo) lands in tensor memory; one thread per coordinate folds each step's tile into
+//     its registers with the rows' rescale factors.  (The output sums terms of both signs, so a
+//     single binary16 term of P' would cost far more relative accuracy than its 2^-11.)
+// Roles (warp-specialised, double-buffered, synchronised by mbarriers): warps 4-7 expand the
+// codes of step i + 1 while warps 0-3 take the softmax of step i and the tensor cores compute
+// S of step i + 1 and O of step i; one thread of warp 8 issues the MMAs.  Splits of the key
+// range leave (m, l, O) partials that a second kernel merges, normalises and rotates back (R^T).
 #pragma once
 #include <algorithm>
 
 #include "iq_decode_impl.cuh"
+#include "iq_tcgen05.cuh"
 
 namespace iq {
 
-constexpr int PF_QB = 8;      // query tokens per block (one per warp)
-constexpr int PF_NSLOT = 4;   // tiles in flight per CTA
+constexpr int PF_ROWS = 128;     // query rows (token, head) per CTA: the MMA's M
+constexpr int PF_BN = 64;        // keys per step (two tile records)
+constexpr int PF_THREADS = 288;  // warps 0-3 softmax and output, 4-7 code expansion, 8 MMA issue
+constexpr int PF_TMEM_COLS = 512;
+constexpr int PF_S_COL = 0;      // scores of buffer b: columns [64 b, 64 b + 64)
+constexpr int PF_O_COL = 128;    // output tile of buffer b: columns [128 + 128 b, 256 + 128 b)
+
+// query tokens per CTA for G heads per kv head
+IQ_HD constexpr int pf_tokens(int g) { return PF_ROWS / g; }
 
 struct PreArgs {
   LayerView v;
@@ -30,183 +50,523 @@ struct PreArgs {
   int q_f32, batch, n_tok, n_q_heads, g_real, n_qblk, splits, max_ctx;
   const int32_t* start;          // [batch] position of each sequence's first chunk token
   const float* params_layer;
-  float2* part_ml;               // [group][split][QB][HMAX]
-  float* part_o;                 // [group][split][QB][HMAX][128]
+  float2* part_ml;               // [group][split][row]: (max in log2 units, sum of 2^(s - max))
+  float* part_o;                 // [group][split][row][128]: sum of 2^(s - max) n_v c (rotated basis)
   float* out;                    // [batch][n_tok][Hq][128]
   KernelConsts kc;
 };
 
+// Shared memory (bytes).  Operand tiles use the no-swizzle K-major layout of iq_tcgen05.cuh.
 template <int KB, int VB>
-struct PreSmem {
-  static constexpr int SLOT_BYTES = tile_bytes(KB, VB);
-  static constexpr int ring = 0;                                        // [slot] tile records
-  static constexpr int qfrag = ring + PF_NSLOT * SLOT_BYTES;            // uint32 [QB][32][QF_WORDS]
-  static constexpr int kappa = qfrag + PF_QB * 32 * QF_WORDS * 4;       // float [QB][HMAX]
-  static constexpr int sparams = kappa + PF_QB * HMAX * 4;              // float [256]
-  static constexpr int valid = sparams + 256 * 4;                       // uint32 [slot] token masks
-  static constexpr int bars = valid + PF_NSLOT * 4;                     // uint64 [slot]
-  static constexpr int bytes = bars + PF_NSLOT * 8;
+struct PfSmem {
+  static constexpr int TB = tile_bytes(KB, VB);
+  static constexpr int q_hi = 0, q_lo = 32768;  // 128 rows x 128 coordinates
+  static constexpr int k0 = 65536;              // hi, lo: 64 keys x 128 coordinates
+  static constexpr int vt0 = 98304;             // [buf] hi, lo: 128 coordinates x 64 keys (32 KB per buf)
+  static constexpr int p = 163840;              // hi, lo: 128 rows x 64 keys (before the steps: parameters, row scales)
+  static constexpr int rec = 196608;            // [buf][2] tile records
+  static constexpr int nk = rec + 4 * TB;       // float [buf][64] K norms of the step's keys
+  static constexpr int nv = nk + 2 * 64 * 4;    // float [buf][64] V norms
+  static constexpr int mrec = nv + 2 * 64 * 4;  // uint32 [buf][2] token masks of the staged records
+  static constexpr int mkv = mrec + 16;         // uint32 [buf][2] token masks of the expanded step
+  static constexpr int alpha = mkv + 16;        // float [128] rows' rescale factors of the last step
+  static constexpr int bars = alpha + 128 * 4;  // uint64 [PB_COUNT]
+  static constexpr int misc = bars + 24 * 8;    // uint32 tensor-memory base, int abort flag
+  static constexpr int bytes = misc + 16;
+  static_assert(bytes <= 232448, "one CTA's shared memory on sm_100");
 };
 
-template <bool P4, int KB, int VB>
-__global__ void __launch_bounds__(DEC_THREADS, 2) prefill_kernel(PreArgs a) {
-  using SM = PreSmem<KB, VB>;
-  constexpr int SLOT = SM::SLOT_BYTES;
-  pdl_launch_dependents();
-  pdl_wait();
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* ring = smem + SM::ring;
-  uint32_t* qfrag = reinterpret_cast<uint32_t*>(smem + SM::qfrag);
-  float* kappa = reinterpret_cast<float*>(smem + SM::kappa);
-  float* sprm = reinterpret_cast<float*>(smem + SM::sparams);
-  uint32_t* valid = reinterpret_cast<uint32_t*>(smem + SM::valid);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bars);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hkv = a.v.n_kv_heads;
+// mbarriers: records staged [buf]; K and V^T expanded [buf]; V^T free again [buf]; scores ready
+// [buf]; scores read [buf]; output tile ready [buf]; output tile read [buf]; P' written; K read
+// (single buffer); the last MMAs done.
+enum { PB_REC = 0, PB_KVFULL = 2, PB_KVFREE = 4, PB_SFULL = 6, PB_SFREE = 8, PB_OFULL = 10, PB_OFREE = 12,
+       PB_PFULL = 14, PB_KFREE = 15, PB_DRAIN = 16, PB_COUNT = 17 };
 
-  const int group = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
-  const int qb = group % a.n_qblk, kvh = (group / a.n_qblk) % Hkv, b = group / (a.n_qblk * Hkv);
-  const int tok0 = qb * PF_QB;
-  const int n_live = min(PF_QB, a.n_tok - tok0);
-  int sp = a.start[b];
-  if (sp < 0 || sp > a.max_ctx - a.n_tok) {  // outside [0, max_ctx - n_tok]: clamped and flagged
-    if (a.v.status && split == 0 && qb == 0 && kvh == 0 && threadIdx.x == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
-    sp = sp < 0 ? 0 : a.max_ctx - a.n_tok;
+// Bounded wait on an mbarrier phase that also gives up once another thread has given up (the
+// abort flag); a timeout flags IQ_DEVERR_TIMEOUT.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 1000000000ull) {
+      if (status) atomicOr(status, IQ_DEVERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
   }
-  const int p0 = sp + tok0;               // position of the block's first query token
-  const int kv_end = p0 + n_live;         // positions 0 .. kv_end - 1 are read
-  const int ntiles = (kv_end + TT - 1) / TT;
-  const int t_lo = (int)((long long)split * ntiles / a.splits), t_hi = (int)((long long)(split + 1) * ntiles / a.splits);
+  return true;
+}
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < PF_NSLOT; ++s) mbar_init(&bars[s], 1);
-    mbar_fence_init();
-  }
-  if (threadIdx.x < params_per_head(a.v.rot) / 4)
-    reinterpret_cast<float4*>(sprm)[threadIdx.x] =
-        reinterpret_cast<const float4*>(a.params_layer + (size_t)kvh * params_per_head(a.v.rot))[threadIdx.x];
-  __syncthreads();
+// AND of `ok` over the 128 threads of named barrier `id` (a barrier for them as well).
+__device__ __forceinline__ bool wg_all(bool ok, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, %2, 128, pi;\n selp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(id)
+      : "memory");
+  return r != 0;
+}
 
-  // first tiles of the range in flight while the queries are rotated
-  auto issue = [&](int i) {
-    const int t = TT * i;
+// Four codes (nibbles 0..3 of s) -> their binary16 centroid terms from the byte tables lb / hb.
+template <int BITS>
+__device__ __forceinline__ uint2 lut_f16x4(const uint32_t* lb, const uint32_t* hb, uint32_t s) {
+  const uint32_t l = lut4<BITS>(lb, s), h = lut4<BITS>(hb, s);
+  return make_uint2(prmt(l, h, 0x5140u), prmt(l, h, 0x7362u));
+}
+
+// Stage the two tile records of step `step` (positions 64 step .. 64 step + 63 of group (b, kvh))
+// into dst with bulk copies completing on `bar` (two arrivals); their token masks go to `mask`.
+__device__ __forceinline__ void pf_stage(const PreArgs& a, int b, int kvh, int step, int kv_end, uint8_t* dst,
+                                         uint32_t* mask, uint64_t* bar, uint32_t tbytes) {
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int i = 2 * step + t, pos = TT * i;
     int pg = b;
-    if (a.v.block_table) {
-      const int idx = t / a.v.page_size;
+    if (a.v.block_table && pos < kv_end) {
+      const int idx = pos / a.v.page_size;
       pg = idx < a.v.max_pages ? a.v.block_table[(size_t)b * a.v.max_pages + idx] : -1;
     }
-    const int sl = (i - t_lo) % PF_NSLOT;
-    issue_tile(a.v, b, kvh, i, kv_end, 0, pg, ring + sl * SLOT, &valid[sl], &bars[sl], SLOT);
-  };
-  if (threadIdx.x == 0)
-    for (int i = t_lo; i < min(t_hi, t_lo + PF_NSLOT); ++i) issue(i);
-
-  // rotated queries: (token j, head h) pairs spread over the warps; P4 fills rows h and h + 4
-  constexpr int HQ = P4 ? 4 : HMAX;
-  for (int idx = warp; idx < PF_QB * HQ; idx += DEC_WARPS) {
-    const int j = idx / HQ, h = idx % HQ;
-    const bool live = j < n_live && h < a.g_real;
-    const size_t row = (((size_t)b * a.n_tok + tok0 + j) * a.n_q_heads + (size_t)kvh * a.g_real + h) * D;
-    rotate_query_row<P4>(a.q, a.q_f32, row, live, a.v.rot, a.kc.k.alpha8, h, sprm, qfrag + j * 32 * QF_WORDS,
-                         kappa + j * HMAX);
-    if (P4 && lane == 0) kappa[j * HMAX + h + 4] = 0.f;  // rows of lo terms: their lanes' scores are unused
-  }
-  __syncthreads();
-
-  const int my_pos = p0 + warp;  // this warp's query position (live when warp < n_live)
-  const bool live = warp < n_live;
-  const float kap = kappa[warp * HMAX + (lane >> 2)];
-  const uint32_t* qf = qfrag + warp * 32 * QF_WORDS + lane * QF_WORDS;
-  WarpState st;
-  st.m = -CUDART_INF_F;
-  st.l = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) st.acc[j][e] = 0.f;
-
-  bool ok = true;
-  for (int i = t_lo; i < t_hi; ++i) {
-    const int k = i - t_lo, sl = k % PF_NSLOT;
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[sl], (k / PF_NSLOT) & 1, a.v.status));
-    const int tok_end = my_pos + 1 - TT * i;  // causal limit inside this tile
-    if (ok && live && tok_end > 0)
-      process_tile<P4, KB, VB>(ring + sl * SLOT, valid[sl] & token_range_mask(0, tok_end), qf, kap, a.kc, st);
-    __syncthreads();  // every warp is done with slot sl
-    if (threadIdx.x == 0 && i + PF_NSLOT < t_hi) issue(i + PF_NSLOT);
-  }
-  // leave no bulk copy in flight (only after a timed-out wait can one be pending)
-  if (!ok && threadIdx.x == 0)
-    for (int i = t_lo; i < t_hi; ++i) mbar_wait(&bars[(i - t_lo) % PF_NSLOT], ((i - t_lo) / PF_NSLOT) & 1, nullptr);
-
-  // ---- this warp's partial: (m, l) per head and O in the rotated basis
-  if (P4) {  // add the lo columns (lanes t >= 2) into the hi columns of the same heads
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st.acc[j][e] += __shfl_xor_sync(0xffffffffu, st.acc[j][e], 2);
-  }
-  float lq = st.l;
-  lq += __shfl_xor_sync(0xffffffffu, lq, 1);
-  lq += __shfl_xor_sync(0xffffffffu, lq, 2);
-  const size_t prow = ((size_t)group * a.splits + split) * PF_QB + warp;
-  const int g = lane >> 2, t = lane & 3;
-  if ((lane & 3) == 0) a.part_ml[prow * HMAX + g] = make_float2(live ? st.m : -CUDART_INF_F, live ? lq : 0.f);
-  float* po = a.part_o + prow * HMAX * D;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    po[(2 * t) * D + 16 * j + g] = st.acc[j][0];
-    po[(2 * t + 1) * D + 16 * j + g] = st.acc[j][1];
-    po[(2 * t) * D + 16 * j + g + 8] = st.acc[j][2];
-    po[(2 * t + 1) * D + 16 * j + g + 8] = st.acc[j][3];
+    issue_tile(a.v, b, kvh, i, kv_end, 0, pg, dst + t * tbytes, &mask[t], bar, tbytes);
   }
 }
 
-// Merge of the splits of every group: warp per (token, head); normalise; inverse rotation.
+template <int KB, int VB>
+__global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
+  using SM = PfSmem<KB, VB>;
+  constexpr int TB = SM::TB;
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::misc);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::misc + 4);
+  float* s_nk = reinterpret_cast<float*>(smem + SM::nk);
+  float* s_nv = reinterpret_cast<float*>(smem + SM::nv);
+  uint32_t* s_mrec = reinterpret_cast<uint32_t*>(smem + SM::mrec);
+  uint32_t* s_mkv = reinterpret_cast<uint32_t*>(smem + SM::mkv);
+  float* s_alpha = reinterpret_cast<float*>(smem + SM::alpha);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Hkv = a.v.n_kv_heads, G = a.g_real, TQ = pf_tokens(G);
+
+  const int group = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
+  const int qb = group % a.n_qblk, kvh = (group / a.n_qblk) % Hkv, b = group / (a.n_qblk * Hkv);
+  const int tok0 = qb * TQ;
+  const int n_live = min(TQ, a.n_tok - tok0);
+  int sp = a.start[b];
+  if (sp < 0 || sp > a.max_ctx - a.n_tok) {  // outside [0, max_ctx - n_tok]: clamped and flagged
+    if (a.v.status && split == 0 && qb == 0 && kvh == 0 && tid == 0) atomicOr(a.v.status, IQ_DEVERR_CTX);
+    sp = sp < 0 ? 0 : a.max_ctx - a.n_tok;
+  }
+  const int p0 = sp + tok0;        // position of the CTA's first query token
+  const int kv_end = p0 + n_live;  // positions 0 .. kv_end - 1 are read
+  const int steps = (kv_end + PF_BN - 1) / PF_BN;
+  const int s_lo = (int)((long long)split * steps / a.splits), s_hi = (int)((long long)(split + 1) * steps / a.splits);
+  const int n = s_hi - s_lo;
+  const size_t prow0 = ((size_t)group * a.splits + split) * PF_ROWS;
+  if (n <= 0) {  // an empty split: neutral partials (the merge skips them)
+    if (tid < PF_ROWS) a.part_ml[prow0 + tid] = make_float2(-CUDART_INF_F, 0.f);
+    return;
+  }
+
+  if (tid == 0) {
+    for (int i = 0; i < PB_COUNT; ++i) {
+      const bool by_threads = (i >= PB_KVFULL && i < PB_KVFULL + 2) || (i >= PB_SFREE && i < PB_SFREE + 2) ||
+                              (i >= PB_OFREE && i < PB_OFREE + 2) || i == PB_PFULL;
+      mbar_init(&bars[i], i < PB_REC + 2 ? 2 : by_threads ? 128 : 1);
+    }
+    mbar_fence_init();
+    *abort = 0;
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, PF_TMEM_COLS);
+  float* sprm = reinterpret_cast<float*>(smem + SM::p);  // this kv head's rotation parameters
+  float* sqs = sprm + 256;                               // rows' score scales
+  if (tid < params_per_head(a.v.rot) / 4)
+    reinterpret_cast<float4*>(sprm)[tid] =
+        reinterpret_cast<const float4*>(a.params_layer + (size_t)kvh * params_per_head(a.v.rot))[tid];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 256)  // the first two steps' records, in flight while the queries are rotated
+    for (int i = 0; i < 2 && i < n; ++i)
+      pf_stage(a, b, kvh, s_lo + i, kv_end, smem + SM::rec + i * 2 * TB, s_mrec + 2 * i, &bars[PB_REC + i], TB);
+
+  // ---- queries: row r = (token r / G, head r % G), rotated, scaled by the power of two that
+  // brings max |q'| into [1/2, 1), split into binary16 hi + lo (K-major rows of 128)
+  for (int r = warp; r < PF_ROWS; r += PF_THREADS / 32) {
+    const int tok = r / G, h = r % G;
+    const bool live = r < TQ * G && tok < n_live;
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live) {
+      const size_t row = (((size_t)b * a.n_tok + tok0 + tok) * a.n_q_heads + (size_t)kvh * G + h) * D + 4 * lane;
+      if (a.q_f32) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>((const float*)a.q + row));
+        x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+      } else {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>((const __half*)a.q + row));
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+      }
+      float Mp[4][4];
+      variant_block_matrix(a.v.rot, sprm + lane * params_per_block(a.v.rot), Mp);
+      warp_rotate_forward(x, Mp, a.v.rot == ROT_ISO);
+    }
+    float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int ex = 0;
+    if (amax > 0.f) frexpf(amax, &ex);
+    const float sig = ldexpf(1.f, -ex);  // exact: a power of two
+    uint32_t hw[2], lw[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float y0 = x[2 * i] * sig, y1 = x[2 * i + 1] * sig;
+      const __half2 hi = __floats2half2_rn(y0, y1);
+      const float2 hf = __half22float2(hi);
+      const __half2 lo = __floats2half2_rn(y0 - hf.x, y1 - hf.y);
+      hw[i] = *reinterpret_cast<const uint32_t*>(&hi);
+      lw[i] = *reinterpret_cast<const uint32_t*>(&lo);
+    }
+    const int off = (r >> 3) * 2048 + (lane >> 1) * 128 + (r & 7) * 16 + (lane & 1) * 8;
+    *reinterpret_cast<uint2*>(smem + SM::q_hi + off) = make_uint2(hw[0], hw[1]);
+    *reinterpret_cast<uint2*>(smem + SM::q_lo + off) = make_uint2(lw[0], lw[1]);
+    // log2-domain score of a key = S n_k log2(e) / (128 sigma): q' c / sqrt(128) is the rotated
+    // dot product with the unit key, n_k / sqrt(128) the key's norm and softmax scale
+    if (lane == 0) sqs[r] = live ? kLog2e / (128.f * sig) : 0.f;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the query tiles before the MMAs read them
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp < 4) {
+    // ==== softmax and output: thread r = score row r and output coordinate r
+    const int r = tid;
+    const int tok = r / G;
+    const bool live = r < TQ * G && tok < n_live;
+    const int qpos = p0 + tok;
+    const float qs = sqs[r];
+    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
+    float O[PF_ROWS];  // coordinate r of every row's output
+#pragma unroll
+    for (int j = 0; j < PF_ROWS; ++j) O[j] = 0.f;
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    auto fold_output = [&](int i) {  // O += the output tile of step i (rows rescaled first)
+      const uint32_t tcol = trow + PF_O_COL + 128 * (i & 1);
+#pragma unroll
+      for (int c = 0; c < PF_ROWS / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tcol + 16 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) O[16 * c + j] = fmaf(O[16 * c + j], s_alpha[16 * c + j], __uint_as_float(v[j]));
+      }
+    };
+    int i = 0;
+    for (; i < n; ++i) {
+      const int buf = i & 1;
+      // the step's scores, and its norms and masks (written by the expansion warps: their own
+      // barrier orders them before these reads; it has completed before the scores can)
+      ok = pf_wait(&bars[PB_SFULL + buf], (i >> 1) & 1, abort, a.v.status);
+      ok = wg_all(ok && pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status), 2);
+      if (!ok) break;
+      tc_fence_after();
+      const int kb = PF_BN * (s_lo + i);
+      const uint32_t mk0 = s_mkv[2 * buf], mk1 = s_mkv[2 * buf + 1];
+      const float* nkb = s_nk + 64 * buf;
+      const float* nvb = s_nv + 64 * buf;
+      const uint32_t scol = trow + PF_S_COL + 64 * buf;
+      auto key_ok = [&](int key) {
+        return live && (((key < 32 ? mk0 >> key : mk1 >> (key - 32)) & 1u) != 0u) && kb + key <= qpos;
+      };
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[16];
+        tmem_ld16(scol + 16 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int key = 16 * c + j;
+          if (key_ok(key)) mx = fmaxf(mx, __uint_as_float(v[j]) * nkb[key] * qs);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float alpha = (m == -CUDART_INF_F) ? 0.f : fast_exp2(m - m_new);
+      // the P buffer is free once the previous step's P.V is done
+      if (i >= 1) {
+        ok = wg_all(pf_wait(&bars[PB_OFULL + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort, a.v.status), 2);
+        if (!ok) break;
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[16];
+        tmem_ld16(scol + 16 * c, v);
+        tmem_wait_ld();
+        uint32_t ph[8], pl[8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          float pp[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = 16 * c + j + e;
+            const bool kv = key_ok(key);
+            const float p = kv ? fast_exp2(__uint_as_float(v[j + e]) * nkb[key] * qs - m_new) : 0.f;
+            lsum += p;
+            pp[e] = kv ? p * nvb[key] : 0.f;
+          }
+          const __half2 h2 = __floats2half2_rn(pp[0], pp[1]);
+          const float2 hf = __half22float2(h2);
+          const __half2 l2 = __floats2half2_rn(pp[0] - hf.x, pp[1] - hf.y);
+          ph[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+          pl[j >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+        uint8_t* prow = smem + SM::p + (r >> 3) * 1024 + (2 * c) * 128 + (r & 7) * 16;
+        *reinterpret_cast<uint4*>(prow) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(prow + 128) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+        *reinterpret_cast<uint4*>(prow + 16384) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        *reinterpret_cast<uint4*>(prow + 16384 + 128) = make_uint4(pl[4], pl[5], pl[6], pl[7]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[PB_SFREE + buf]);  // the scores of this buffer are read
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[PB_PFULL]);
+      l = l * alpha + lsum;
+      m = m_new;
+      if (i >= 1) {
+        named_barrier_sync(2, 128);  // every row's factor of step i - 1 is in s_alpha
+        fold_output(i - 1);
+        tc_fence_before();
+        mbar_arrive(&bars[PB_OFREE + ((i - 1) & 1)]);
+      }
+      named_barrier_sync(2, 128);  // s_alpha is read
+      s_alpha[r] = alpha;
+    }
+    if (ok) {
+      ok = wg_all(pf_wait(&bars[PB_OFULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, a.v.status), 2);
+      if (ok) {
+        tc_fence_after();
+        fold_output(n - 1);
+      }
+    }
+    // partials: (m, l) of row r, and coordinate r of every row's O
+    a.part_ml[prow0 + r] = make_float2(live && ok ? m : -CUDART_INF_F, live && ok ? l : 0.f);
+    float* po = a.part_o + prow0 * D + r;
+#pragma unroll
+    for (int j = 0; j < PF_ROWS; ++j) po[(size_t)j * D] = O[j];
+  } else if (warp < 8) {
+    // ==== code expansion: K as 64 keys x 128 coordinates, V^T as 128 coordinates x 64 keys
+    const int e = tid - 128;
+    const int key = e & 63, half = e >> 6;  // K: key and half of its coordinates
+    const int d = e, g = d & 7, hh = (d >> 3) & 1, e2 = (d >> 4) & 1, w = d >> 5;  // V: coordinate d
+    uint32_t kl0[4], kh0[4], kl1[4], kh1[4], vl0[4], vh0[4], vl1[4], vh1[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      kl0[t] = a.kc.k.f16_lb[0][t]; kh0[t] = a.kc.k.f16_hb[0][t];
+      kl1[t] = a.kc.k.f16_lb[1][t]; kh1[t] = a.kc.k.f16_hb[1][t];
+      vl0[t] = a.kc.v.f16_lb[0][t]; vh0[t] = a.kc.v.f16_hb[0][t];
+      vl1[t] = a.kc.v.f16_lb[1][t]; vh1[t] = a.kc.v.f16_hb[1][t];
+    }
+    int waited = 0, staged = min(n, 2);
+    for (int i = 0; i < n; ++i) {
+      const int buf = i & 1;
+      bool ok = pf_wait(&bars[PB_REC + buf], (i >> 1) & 1, abort, a.v.status);
+      if (ok) waited = i + 1;
+      ok = ok && pf_wait(&bars[PB_KVFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status);  // V^T buffer
+      ok = ok && (i == 0 || pf_wait(&bars[PB_KFREE], (i - 1) & 1, abort, a.v.status));    // K: S of step i - 1 done
+      if (!wg_all(ok, 1)) break;
+      const uint8_t* recb = smem + SM::rec + buf * 2 * TB;
+      {  // K: coordinates 64 half .. 64 half + 63 of key `key`, eight per 16-byte core-matrix row
+        const uint8_t* kr = recb + (key >> 5) * TB + (key & 31) * k_rec_bytes(KB);
+        uint8_t* khi = smem + SM::k0;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
+          uint32_t wd[KB], sel[4];
+#pragma unroll
+          for (int t = 0; t < KB; ++t) wd[t] = reinterpret_cast<const uint32_t*>(kr + c * chunk_bytes(KB))[t];
+          chunk_selectors<KB>(wd, sel);
+#pragma unroll
+          for (int wq = 0; wq < 4; ++wq) {
+            const uint2 a0 = lut_f16x4<KB>(kl0, kh0, sel[wq]), a1 = lut_f16x4<KB>(kl0, kh0, sel[wq] >> 16);
+            const uint2 b0 = lut_f16x4<KB>(kl1, kh1, sel[wq]), b1 = lut_f16x4<KB>(kl1, kh1, sel[wq] >> 16);
+            const int off = (key >> 3) * 2048 + (4 * c + wq) * 128 + (key & 7) * 16;
+            *reinterpret_cast<uint4*>(khi + off) = make_uint4(a0.x, a0.y, a1.x, a1.y);
+            *reinterpret_cast<uint4*>(khi + 16384 + off) = make_uint4(b0.x, b0.y, b1.x, b1.y);
+          }
+        }
+      }
+      {  // V^T: coordinate d of the 64 keys.  Coordinate d = 32 w + 16 e2 + 8 hh + g of the
+         // block's tokens u sits in chunk (g, tq = (u mod 8) / 2, hh), selector word w, nibble
+         // m + 4 e2 (m = 2 (u / 8) + u mod 2): byte 2 e2 of that word holds tokens 2 tq, 2 tq + 1,
+         // byte 2 e2 + 1 tokens 2 tq + 8, 2 tq + 9.
+        uint8_t* vhi = smem + SM::vt0 + buf * 32768;
+        const uint32_t b0 = 2 * e2, b1 = 2 * e2 + 1;
+        const uint32_t sl0 = b0 | ((4 + b0) << 4), sl1 = b1 | ((4 + b1) << 4);
+#pragma unroll
+        for (int v16 = 0; v16 < 4; ++v16) {  // the step's four 16-token V blocks
+          const uint8_t* vb = recb + (v16 >> 1) * TB + tr_v(KB) + (v16 & 1) * v_blk_bytes(VB);
+          uint32_t s[4];
+#pragma unroll
+          for (int tq = 0; tq < 4; ++tq) {
+            const uint32_t* ch =
+                reinterpret_cast<const uint32_t*>(vb + 2 * chunk_bytes(VB) * (4 * g + tq) + hh * chunk_bytes(VB));
+            uint32_t wd[VB], sel[4];
+#pragma unroll
+            for (int t = 0; t < VB; ++t) wd[t] = ch[t];
+            chunk_selectors<VB>(wd, sel);
+            s[tq] = w == 0 ? sel[0] : w == 1 ? sel[1] : w == 2 ? sel[2] : sel[3];
+          }
+          const uint32_t sA = prmt(s[0], s[1], sl0), sB = prmt(s[2], s[3], sl0);  // tokens 0-3, 4-7
+          const uint32_t sC = prmt(s[0], s[1], sl1), sD = prmt(s[2], s[3], sl1);  // tokens 8-11, 12-15
+          const int off = (d >> 3) * 1024 + (2 * v16) * 128 + (d & 7) * 16;
+          const uint2 hA = lut_f16x4<VB>(vl0, vh0, sA), hB = lut_f16x4<VB>(vl0, vh0, sB);
+          const uint2 hC = lut_f16x4<VB>(vl0, vh0, sC), hD = lut_f16x4<VB>(vl0, vh0, sD);
+          *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hA.x, hA.y, hB.x, hB.y);
+          *reinterpret_cast<uint4*>(vhi + off + 128) = make_uint4(hC.x, hC.y, hD.x, hD.y);
+          const uint2 lA = lut_f16x4<VB>(vl1, vh1, sA), lB = lut_f16x4<VB>(vl1, vh1, sB);
+          const uint2 lC = lut_f16x4<VB>(vl1, vh1, sC), lD = lut_f16x4<VB>(vl1, vh1, sD);
+          *reinterpret_cast<uint4*>(vhi + 16384 + off) = make_uint4(lA.x, lA.y, lB.x, lB.y);
+          *reinterpret_cast<uint4*>(vhi + 16384 + off + 128) = make_uint4(lC.x, lC.y, lD.x, lD.y);
+        }
+      }
+      if (e < 64) {  // the step's norms
+        const uint8_t* tr = recb + (e >> 5) * TB;
+        s_nk[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(tr + tr_kn(KB, VB))[e & 31]);
+        s_nv[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(tr + tr_vn(KB, VB))[e & 31]);
+      } else if (e < 66) {
+        s_mkv[2 * buf + (e - 64)] = s_mrec[2 * buf + (e - 64)];
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[PB_KVFULL + buf]);
+      named_barrier_sync(1, 128);  // every expansion thread is done with this record buffer
+      if (e == 0 && i + 2 < n) {
+        pf_stage(a, b, kvh, s_lo + i + 2, kv_end, smem + SM::rec + buf * 2 * TB, s_mrec + 2 * buf,
+                 &bars[PB_REC + buf], TB);
+        ++staged;
+      }
+    }
+    // leave no bulk copy in flight (only after a timed-out wait can one be pending)
+    if (e == 0)
+      for (; waited < staged; ++waited) mbar_wait(&bars[PB_REC + (waited & 1)], (waited >> 1) & 1, nullptr);
+  } else if (lane == 0) {
+    // ==== MMA issue: S_{i+1} = Q K_{i+1}^T ahead of O_i^T = V_i^T P_i'^T
+    const uint32_t idS = umma_idesc_f16(128, PF_BN), idO = umma_idesc_f16(128, 128);
+    const uint32_t qh = smem_addr(smem + SM::q_hi), ql = smem_addr(smem + SM::q_lo), pa = smem_addr(smem + SM::p);
+    auto issue_s = [&](int i) {
+      const int buf = i & 1;
+      if (!pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status)) return false;
+      if (!pf_wait(&bars[PB_SFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) return false;
+      tc_fence_after();
+      const uint32_t kh = smem_addr(smem + SM::k0), kl = kh + 16384;
+      const uint32_t dst = tmem + PF_S_COL + 64 * buf;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        umma_f16(dst, umma_sdesc(qh + 256 * ks, 128, 2048), umma_sdesc(kh + 256 * ks, 128, 2048), idS, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        umma_f16(dst, umma_sdesc(ql + 256 * ks, 128, 2048), umma_sdesc(kh + 256 * ks, 128, 2048), idS, 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        umma_f16(dst, umma_sdesc(qh + 256 * ks, 128, 2048), umma_sdesc(kl + 256 * ks, 128, 2048), idS, 1);
+      umma_commit(&bars[PB_SFULL + buf]);
+      umma_commit(&bars[PB_KFREE]);
+      return true;
+    };
+    auto issue_o = [&](int i) {
+      const int buf = i & 1;
+      if (!pf_wait(&bars[PB_PFULL], i & 1, abort, a.v.status)) return false;
+      if (!pf_wait(&bars[PB_OFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) return false;
+      tc_fence_after();
+      const uint32_t vh = smem_addr(smem + SM::vt0 + buf * 32768), vl = vh + 16384;
+      const uint32_t dst = tmem + PF_O_COL + 128 * buf;
+#pragma unroll
+      for (int ks = 0; ks < PF_BN / 16; ++ks)
+        umma_f16(dst, umma_sdesc(vh + 256 * ks, 128, 1024), umma_sdesc(pa + 256 * ks, 128, 1024), idO, ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < PF_BN / 16; ++ks)
+        umma_f16(dst, umma_sdesc(vl + 256 * ks, 128, 1024), umma_sdesc(pa + 256 * ks, 128, 1024), idO, 1);
+#pragma unroll
+      for (int ks = 0; ks < PF_BN / 16; ++ks)
+        umma_f16(dst, umma_sdesc(vh + 256 * ks, 128, 1024), umma_sdesc(pa + 16384 + 256 * ks, 128, 1024), idO, 1);
+      umma_commit(&bars[PB_OFULL + buf]);
+      umma_commit(&bars[PB_KVFREE + buf]);
+      return true;
+    };
+    bool ok = issue_s(0);
+    for (int i = 0; ok && i < n; ++i) {
+      if (i + 1 < n) ok = issue_s(i + 1);
+      if (ok) ok = issue_o(i);
+    }
+    // every MMA issued is complete before tensor memory is released
+    umma_commit(&bars[PB_DRAIN]);
+    mbar_wait(&bars[PB_DRAIN], 0, nullptr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_free(tmem, PF_TMEM_COLS);
+}
+
+// Merge of the splits of every group: warp per row; normalise; inverse rotation.
 static __global__ void __launch_bounds__(DEC_THREADS) prefill_merge_kernel(PreArgs a) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float sprm[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hkv = a.v.n_kv_heads;
+  const int Hkv = a.v.n_kv_heads, G = a.g_real, TQ = pf_tokens(G);
   const int group = blockIdx.x;
   const int qb = group % a.n_qblk, kvh = (group / a.n_qblk) % Hkv, b = group / (a.n_qblk * Hkv);
-  const int tok0 = qb * PF_QB, n_live = min(PF_QB, a.n_tok - tok0);
+  const int tok0 = qb * TQ, n_live = min(TQ, a.n_tok - tok0);
   if (threadIdx.x < params_per_head(a.v.rot) / 4)
     reinterpret_cast<float4*>(sprm)[threadIdx.x] =
         reinterpret_cast<const float4*>(a.params_layer + (size_t)kvh * params_per_head(a.v.rot))[threadIdx.x];
   __syncthreads();
   float Mp[4][4];
   variant_block_matrix(a.v.rot, sprm + lane * params_per_block(a.v.rot), Mp);
-  for (int idx = warp; idx < n_live * a.g_real; idx += DEC_WARPS) {
-    const int j = idx / a.g_real, h = idx % a.g_real;
+  for (int r = warp; r < TQ * G; r += DEC_WARPS) {
+    const int tok = r / G, h = r % G;
+    if (tok >= n_live) continue;
     float M = -CUDART_INF_F;
-    for (int s = 0; s < a.splits; ++s)
-      M = fmaxf(M, a.part_ml[(((size_t)group * a.splits + s) * PF_QB + j) * HMAX + h].x);
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((size_t)group * a.splits + s) * PF_ROWS + r].x);
     float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
     for (int s = 0; s < a.splits; ++s) {
-      const size_t prow = ((size_t)group * a.splits + s) * PF_QB + j;
-      const float2 ml = a.part_ml[prow * HMAX + h];
+      const size_t prow = ((size_t)group * a.splits + s) * PF_ROWS + r;
+      const float2 ml = a.part_ml[prow];
       if (ml.x == -CUDART_INF_F) continue;
-      const float w = fast_exp2(ml.x - M);
-      L = fmaf(ml.y, w, L);
-      const float4 v = reinterpret_cast<const float4*>(a.part_o + (prow * HMAX + h) * D)[lane];
-      o[0] = fmaf(v.x, w, o[0]); o[1] = fmaf(v.y, w, o[1]); o[2] = fmaf(v.z, w, o[2]); o[3] = fmaf(v.w, w, o[3]);
+      const float wgt = fast_exp2(ml.x - M);
+      L = fmaf(ml.y, wgt, L);
+      const float4 v = reinterpret_cast<const float4*>(a.part_o + prow * D)[lane];
+      o[0] = fmaf(v.x, wgt, o[0]); o[1] = fmaf(v.y, wgt, o[1]); o[2] = fmaf(v.z, wgt, o[2]); o[3] = fmaf(v.w, wgt, o[3]);
     }
-    const float sc = L > 0.f ? 0.08838834764831845f / (a.kc.v.alpha8 * L) : 0.f;
+    const float sc = L > 0.f ? 0.08838834764831845f / L : 0.f;  // V = n_v c / sqrt(128)
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[i] *= sc;
     warp_rotate_inverse(o, Mp, a.v.rot == ROT_ISO);
-    reinterpret_cast<float4*>(a.out + (((size_t)b * a.n_tok + tok0 + j) * a.n_q_heads + (size_t)kvh * a.g_real + h) *
-                                          D)[lane] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(a.out + (((size_t)b * a.n_tok + tok0 + tok) * a.n_q_heads + (size_t)kvh * G + h) * D)[lane] =
+        make_float4(o[0], o[1], o[2], o[3]);
   }
 }
 
-// Splits per group: enough CTAs for two per SM, each with at least two tiles.
-inline int prefill_splits(int groups, int max_tiles, int n_sm) {
-  int s = (2 * n_sm + groups - 1) / groups;
-  s = std::min(s, std::max(1, max_tiles / 2));
+// Splits per group: at most one CTA per SM in all, each with at least four steps.
+inline int prefill_splits(int groups, int max_steps, int n_sm) {
+  int s = std::max(1, n_sm / std::max(groups, 1));
+  s = std::min(s, std::max(1, max_steps / 4));
   return std::max(1, std::min(s, 64));
+}
+
+// Workspace rows (partials) of one call, for the group size g.
+inline size_t prefill_rows(int batch, int n_tok, int n_kv_heads, int max_ctx, int g, int n_sm, int* splits_out) {
+  const int n_qblk = (n_tok + pf_tokens(g) - 1) / pf_tokens(g);
+  const int groups = batch * n_kv_heads * n_qblk;
+  const int splits = prefill_splits(groups, (max_ctx + PF_BN - 1) / PF_BN, n_sm);
+  if (splits_out) *splits_out = splits;
+  return (size_t)groups * splits * PF_ROWS;
 }
 
 template <int KB, int VB>
@@ -222,24 +582,21 @@ int launch_prefill_kv(const LayerView& v, const void* q, int q_f32, int batch, i
   a.n_tok = n_tok;
   a.n_q_heads = n_q_heads;
   a.g_real = n_q_heads / v.n_kv_heads;
-  a.n_qblk = (n_tok + PF_QB - 1) / PF_QB;
+  a.n_qblk = (n_tok + pf_tokens(a.g_real) - 1) / pf_tokens(a.g_real);
   const int groups = batch * v.n_kv_heads * a.n_qblk;
-  a.splits = prefill_splits(groups, (max_ctx + TT - 1) / TT, n_sm);
+  const size_t rows = prefill_rows(batch, n_tok, v.n_kv_heads, max_ctx, a.g_real, n_sm, &a.splits);
   a.max_ctx = max_ctx;
   a.start = start;
   a.params_layer = params_layer;
-  const size_t rows = (size_t)groups * a.splits * PF_QB * HMAX;
   a.part_ml = (float2*)workspace;
   a.part_o = (float*)((char*)workspace + ((rows * sizeof(float2) + 255) & ~(size_t)255));
   a.out = out;
   a.kc = kc;
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(prefill_kernel<false, KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, PreSmem<KB, VB>::bytes);
-    cudaFuncSetAttribute(prefill_kernel<true, KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, PreSmem<KB, VB>::bytes);
+    cudaFuncSetAttribute(prefill_kernel<KB, VB>, cudaFuncAttributeMaxDynamicSharedMemorySize, PfSmem<KB, VB>::bytes);
   });
-  auto kern = a.g_real <= 4 ? prefill_kernel<true, KB, VB> : prefill_kernel<false, KB, VB>;
-  int e = (int)launch_pdl(kern, dim3(groups * a.splits), dim3(DEC_THREADS), PreSmem<KB, VB>::bytes,
+  int e = (int)launch_pdl(prefill_kernel<KB, VB>, dim3(groups * a.splits), dim3(PF_THREADS), PfSmem<KB, VB>::bytes,
                           (cudaStream_t)stream, a);
   if (e) return e;
   return (int)launch_pdl(prefill_merge_kernel, dim3(groups), dim3(DEC_THREADS), 0, (cudaStream_t)stream, a);
