@@ -172,6 +172,19 @@ __device__ __forceinline__ void chunk_selectors(const uint32_t* w, uint32_t sel[
   }
 }
 
+// Selector word w alone, reading only the storage words it depends on.
+template <int BITS>
+__device__ __forceinline__ uint32_t chunk_selector(const uint32_t* w, int sel) {
+  if constexpr (BITS == 3) {
+    if (sel < 3) return w[sel] & 0x77777777u;
+    return ((w[0] >> 3) & 0x11111111u) | ((w[1] >> 2) & 0x22222222u) | ((w[2] >> 1) & 0x44444444u);
+  } else if constexpr (BITS == 4) {
+    return w[sel];
+  } else {
+    return (w[sel >> 1] >> (2 * (sel & 1))) & 0x33333333u;
+  }
+}
+
 // Storage word k (k < BITS) of a chunk from its four selector words (the inverse of the
 // above).  Every token's codes sit in whole nibbles of the selector words, and this map keeps
 // nibble positions: a nibble of the selector words lands in the same nibble of storage words.

@@ -22,9 +22,11 @@
 //     V_hi P_lo) lands in tensor memory; one thread per coordinate folds each step's tile into
 //     its registers with the rows' rescale factors.  (The output sums terms of both signs, so a
 //     single binary16 term of P' would cost far more relative accuracy than its 2^-11.)
-// Roles (warp-specialised, double-buffered, synchronised by mbarriers): warps 4-7 expand the
-// codes of step i + 1 while warps 0-3 take the softmax of step i and the tensor cores compute
-// S of step i + 1 and O of step i; one thread of warp 8 issues the MMAs.  Splits of the key
+// Roles (warp-specialised, double-buffered, synchronised by mbarriers): warps 8-11 expand the
+// codes of step i + 1 while warps 0-7 take the softmax of step i (two warps per row quarter of
+// tensor memory: one per half of the keys, and per half of the rows when folding the output)
+// and the tensor cores compute S of step i + 1 and O of step i; one thread of warp 12 issues
+// the MMAs and one of warp 13 stages the tile records with bulk copies.  Splits of the key
 // range leave (m, l, O) partials that a second kernel merges, normalises and rotates back (R^T).
 #pragma once
 #include <algorithm>
@@ -36,7 +38,7 @@ namespace iq {
 
 constexpr int PF_ROWS = 128;     // query rows (token, head) per CTA: the MMA's M
 constexpr int PF_BN = 64;        // keys per step (two tile records)
-constexpr int PF_THREADS = 288;  // warps 0-3 softmax and output, 4-7 code expansion, 8 MMA issue
+constexpr int PF_THREADS = 448;  // warps 0-7 softmax and output, 8-11 code expansion, 12 MMA issue, 13 loads
 constexpr int PF_TMEM_COLS = 512;
 constexpr int PF_S_COL = 0;      // scores of buffer b: columns [64 b, 64 b + 64)
 constexpr int PF_O_COL = 128;    // output tile of buffer b: columns [128 + 128 b, 256 + 128 b)
@@ -70,7 +72,8 @@ struct PfSmem {
   static constexpr int mrec = nv + 2 * 64 * 4;  // uint32 [buf][2] token masks of the staged records
   static constexpr int mkv = mrec + 16;         // uint32 [buf][2] token masks of the expanded step
   static constexpr int alpha = mkv + 16;        // float [128] rows' rescale factors of the last step
-  static constexpr int bars = alpha + 128 * 4;  // uint64 [PB_COUNT]
+  static constexpr int red = alpha + 128 * 4;   // float [2][128] per key half: row maxima, at the end sums
+  static constexpr int bars = red + 256 * 4;    // uint64 [PB_COUNT]
   static constexpr int misc = bars + 24 * 8;    // uint32 tensor-memory base, int abort flag
   static constexpr int bytes = misc + 16;
   static_assert(bytes <= 232448, "one CTA's shared memory on sm_100");
@@ -78,9 +81,9 @@ struct PfSmem {
 
 // mbarriers: records staged [buf]; K and V^T expanded [buf]; V^T free again [buf]; scores ready
 // [buf]; scores read [buf]; output tile ready [buf]; output tile read [buf]; P' written; K read
-// (single buffer); the last MMAs done.
+// (single buffer); the last MMAs done; records read [buf].
 enum { PB_REC = 0, PB_KVFULL = 2, PB_KVFREE = 4, PB_SFULL = 6, PB_SFREE = 8, PB_OFULL = 10, PB_OFREE = 12,
-       PB_PFULL = 14, PB_KFREE = 15, PB_DRAIN = 16, PB_COUNT = 17 };
+       PB_PFULL = 14, PB_KFREE = 15, PB_DRAIN = 16, PB_RECFREE = 17, PB_COUNT = 19 };
 
 // Bounded wait on an mbarrier phase that also gives up once another thread has given up (the
 // abort flag); a timeout flags IQ_DEVERR_TIMEOUT.
@@ -98,13 +101,13 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile
   return true;
 }
 
-// AND of `ok` over the 128 threads of named barrier `id` (a barrier for them as well).
-__device__ __forceinline__ bool wg_all(bool ok, int id) {
+// AND of `ok` over the `count` threads of named barrier `id` (a barrier for them as well).
+__device__ __forceinline__ bool wg_all(bool ok, int id, int count) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, %2, 128, pi;\n selp.u32 %0, 1, 0, po;\n}\n"
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, %2, %3, pi;\n selp.u32 %0, 1, 0, po;\n}\n"
       : "=r"(r)
-      : "r"((uint32_t)ok), "r"(id)
+      : "r"((uint32_t)ok), "r"(id), "r"(count)
       : "memory");
   return r != 0;
 }
@@ -172,9 +175,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
 
   if (tid == 0) {
     for (int i = 0; i < PB_COUNT; ++i) {
-      const bool by_threads = (i >= PB_KVFULL && i < PB_KVFULL + 2) || (i >= PB_SFREE && i < PB_SFREE + 2) ||
+      const bool by_threads = (i >= PB_KVFULL && i < PB_KVFULL + 2) || (i >= PB_RECFREE && i < PB_RECFREE + 2) ||
                               (i >= PB_OFREE && i < PB_OFREE + 2) || i == PB_PFULL;
-      mbar_init(&bars[i], i < PB_REC + 2 ? 2 : by_threads ? 128 : 1);
+      const bool by_softmax = (i >= PB_SFREE && i < PB_SFREE + 2) || (i >= PB_OFREE && i < PB_OFREE + 2) || i == PB_PFULL;
+      mbar_init(&bars[i], i < PB_REC + 2 ? 2 : by_softmax ? 256 : by_threads ? 128 : 1);
     }
     mbar_fence_init();
     *abort = 0;
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (tid == 256)  // the first two steps' records, in flight while the queries are rotated
+  if (tid == 416)  // the first two steps' records, in flight while the queries are rotated
     for (int i = 0; i < 2 && i < n; ++i)
       pf_stage(a, b, kvh, s_lo + i, kv_end, smem + SM::rec + i * 2 * TB, s_mrec + 2 * i, &bars[PB_REC + i], TB);
 
@@ -242,83 +246,86 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
   __syncthreads();
   tc_fence_after();
 
-  if (warp < 4) {
-    // ==== softmax and output: thread r = score row r and output coordinate r
-    const int r = tid;
+  if (warp < 8) {
+    // ==== softmax and output.  Warp w reads tensor-memory lanes 32 (w % 4) ..: thread = score
+    // row r of those lanes for keys 32 kh .. 32 kh + 31 (kh = w / 4), and output coordinate r for
+    // rows 64 kh .. 64 kh + 63.
+    const int kh = warp >> 2;
+    const int r = 32 * (warp & 3) + lane;
+    float* s_red = reinterpret_cast<float*>(smem + SM::red);
     const int tok = r / G;
     const bool live = r < TQ * G && tok < n_live;
     const int qpos = p0 + tok;
     const float qs = sqs[r];
-    const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-    float O[PF_ROWS];  // coordinate r of every row's output
+    const uint32_t tlane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    float O[PF_ROWS / 2];  // coordinate r of rows 64 kh ..
 #pragma unroll
-    for (int j = 0; j < PF_ROWS; ++j) O[j] = 0.f;
-    float m = -CUDART_INF_F, l = 0.f;
+    for (int j = 0; j < PF_ROWS / 2; ++j) O[j] = 0.f;
+    float m = -CUDART_INF_F, l = 0.f;  // l: this key half's share of the row's sum
     bool ok = true;
     auto fold_output = [&](int i) {  // O += the output tile of step i (rows rescaled first)
-      const uint32_t tcol = trow + PF_O_COL + 128 * (i & 1);
+      const uint32_t tcol = tlane + PF_O_COL + 128 * (i & 1) + 64 * kh;
 #pragma unroll
-      for (int c = 0; c < PF_ROWS / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(tcol + 16 * c, v);
+      for (int c = 0; c < PF_ROWS / 64; ++c) {
+        uint32_t v[16], u[16];
+        tmem_ld16(tcol + 32 * c, v);
+        tmem_ld16(tcol + 32 * c + 16, u);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) O[16 * c + j] = fmaf(O[16 * c + j], s_alpha[16 * c + j], __uint_as_float(v[j]));
+        for (int j = 0; j < 16; ++j) {
+          O[32 * c + j] = fmaf(O[32 * c + j], s_alpha[64 * kh + 32 * c + j], __uint_as_float(v[j]));
+          O[32 * c + 16 + j] = fmaf(O[32 * c + 16 + j], s_alpha[64 * kh + 32 * c + 16 + j], __uint_as_float(u[j]));
+        }
       }
     };
-    int i = 0;
-    for (; i < n; ++i) {
+    for (int i = 0; i < n; ++i) {
       const int buf = i & 1;
       // the step's scores, and its norms and masks (written by the expansion warps: their own
       // barrier orders them before these reads; it has completed before the scores can)
       ok = pf_wait(&bars[PB_SFULL + buf], (i >> 1) & 1, abort, a.v.status);
-      ok = wg_all(ok && pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status), 2);
+      ok = wg_all(ok && pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status), 2, 256);
       if (!ok) break;
       tc_fence_after();
-      const int kb = PF_BN * (s_lo + i);
-      const uint32_t mk0 = s_mkv[2 * buf], mk1 = s_mkv[2 * buf + 1];
-      const float* nkb = s_nk + 64 * buf;
-      const float* nvb = s_nv + 64 * buf;
-      const uint32_t scol = trow + PF_S_COL + 64 * buf;
-      auto key_ok = [&](int key) {
-        return live && (((key < 32 ? mk0 >> key : mk1 >> (key - 32)) & 1u) != 0u) && kb + key <= qpos;
-      };
+      const int kb = PF_BN * (s_lo + i) + 32 * kh;  // position of this thread's first key
+      uint32_t vmask = live ? s_mkv[2 * buf + kh] : 0u;
+      if (qpos - kb < 31) vmask &= qpos < kb ? 0u : (2u << (qpos - kb)) - 1u;  // causal: keys <= qpos
+      const float* nkb = s_nk + 64 * buf + 32 * kh;
+      const float* nvb = s_nv + 64 * buf + 32 * kh;
+      float sv[32];
       float mx = -CUDART_INF_F;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[16];
-        tmem_ld16(scol + 16 * c, v);
+      {
+        uint32_t v[32];
+        tmem_ld16(tlane + PF_S_COL + 64 * buf + 32 * kh, *reinterpret_cast<uint32_t(*)[16]>(v));
+        tmem_ld16(tlane + PF_S_COL + 64 * buf + 32 * kh + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int key = 16 * c + j;
-          if (key_ok(key)) mx = fmaxf(mx, __uint_as_float(v[j]) * nkb[key] * qs);
+        for (int k = 0; k < 32; ++k) {
+          sv[k] = ((vmask >> k) & 1u) ? __uint_as_float(v[k]) * nkb[k] * qs : -CUDART_INF_F;
+          mx = fmaxf(mx, sv[k]);
         }
       }
-      const float m_new = fmaxf(m, mx);
+      tc_fence_before();
+      mbar_arrive(&bars[PB_SFREE + buf]);  // the scores of this buffer are read
+      s_red[128 * kh + r] = mx;
+      // the P buffer is free once the previous step's P.V is done (this also publishes s_red)
+      ok = wg_all(i == 0 || pf_wait(&bars[PB_OFULL + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort, a.v.status), 2, 256);
+      if (!ok) break;
+      const float m_new = fmaxf(m, fmaxf(s_red[r], s_red[128 + r]));
       const float alpha = (m == -CUDART_INF_F) ? 0.f : fast_exp2(m - m_new);
-      // the P buffer is free once the previous step's P.V is done
-      if (i >= 1) {
-        ok = wg_all(pf_wait(&bars[PB_OFULL + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort, a.v.status), 2);
-        if (!ok) break;
-      }
       float lsum = 0.f;
+      uint8_t* prow = smem + SM::p + (r >> 3) * 1024 + (4 * kh) * 128 + (r & 7) * 16;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[16];
-        tmem_ld16(scol + 16 * c, v);
-        tmem_wait_ld();
-        uint32_t ph[8], pl[8];
+      for (int c = 0; c < 4; ++c) {  // keys 8 c .. 8 c + 7 of this half: one 16-byte row of a core matrix
+        uint32_t ph[4], pl[4];
 #pragma unroll
-        for (int j = 0; j < 16; j += 2) {
+        for (int j = 0; j < 8; j += 2) {
           float pp[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int key = 16 * c + j + e;
-            const bool kv = key_ok(key);
-            const float p = kv ? fast_exp2(__uint_as_float(v[j + e]) * nkb[key] * qs - m_new) : 0.f;
+            const int k = 8 * c + j + e;
+            const float p = ((vmask >> k) & 1u) ? fast_exp2(sv[k] - m_new) : 0.f;
             lsum += p;
-            pp[e] = kv ? p * nvb[key] : 0.f;
+            pp[e] = ((vmask >> k) & 1u) ? p * nvb[k] : 0.f;
           }
           const __half2 h2 = __floats2half2_rn(pp[0], pp[1]);
           const float2 hf = __half22float2(h2);
@@ -326,42 +333,40 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           ph[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
           pl[j >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
         }
-        uint8_t* prow = smem + SM::p + (r >> 3) * 1024 + (2 * c) * 128 + (r & 7) * 16;
-        *reinterpret_cast<uint4*>(prow) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(prow + 128) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
-        *reinterpret_cast<uint4*>(prow + 16384) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-        *reinterpret_cast<uint4*>(prow + 16384 + 128) = make_uint4(pl[4], pl[5], pl[6], pl[7]);
+        *reinterpret_cast<uint4*>(prow + 128 * c) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(prow + 16384 + 128 * c) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
       }
-      tc_fence_before();
-      mbar_arrive(&bars[PB_SFREE + buf]);  // the scores of this buffer are read
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars[PB_PFULL]);
       l = l * alpha + lsum;
       m = m_new;
-      if (i >= 1) {
-        named_barrier_sync(2, 128);  // every row's factor of step i - 1 is in s_alpha
+      if (i >= 1) {  // every row's factor of step i - 1 is in s_alpha (published by the barriers above)
         fold_output(i - 1);
         tc_fence_before();
         mbar_arrive(&bars[PB_OFREE + ((i - 1) & 1)]);
       }
-      named_barrier_sync(2, 128);  // s_alpha is read
-      s_alpha[r] = alpha;
+      named_barrier_sync(2, 256);  // s_alpha and s_red are read
+      if (kh == 0) s_alpha[r] = alpha;
     }
     if (ok) {
-      ok = wg_all(pf_wait(&bars[PB_OFULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, a.v.status), 2);
+      ok = wg_all(pf_wait(&bars[PB_OFULL + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort, a.v.status), 2, 256);
       if (ok) {
         tc_fence_after();
         fold_output(n - 1);
       }
     }
-    // partials: (m, l) of row r, and coordinate r of every row's O
-    a.part_ml[prow0 + r] = make_float2(live && ok ? m : -CUDART_INF_F, live && ok ? l : 0.f);
-    float* po = a.part_o + prow0 * D + r;
+    // partials: (m, l) of row r (the two key halves' sums), and coordinate r of rows 64 kh ..
+    named_barrier_sync(2, 256);
+    s_red[128 * kh + r] = l;
+    named_barrier_sync(2, 256);
+    if (kh == 0)
+      a.part_ml[prow0 + r] = make_float2(live && ok ? m : -CUDART_INF_F, live && ok ? l + s_red[128 + r] : 0.f);
+    float* po = a.part_o + (prow0 + 64 * kh) * D + r;
 #pragma unroll
-    for (int j = 0; j < PF_ROWS; ++j) po[(size_t)j * D] = O[j];
-  } else if (warp < 8) {
+    for (int j = 0; j < PF_ROWS / 2; ++j) po[(size_t)j * D] = O[j];
+  } else if (warp < 12) {
     // ==== code expansion: K as 64 keys x 128 coordinates, V^T as 128 coordinates x 64 keys
-    const int e = tid - 128;
+    const int e = tid - 256;
     const int key = e & 63, half = e >> 6;  // K: key and half of its coordinates
     const int d = e, g = d & 7, hh = (d >> 3) & 1, e2 = (d >> 4) & 1, w = d >> 5;  // V: coordinate d
     uint32_t kl0[4], kh0[4], kl1[4], kh1[4], vl0[4], vh0[4], vl1[4], vh1[4];
@@ -372,14 +377,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       vl0[t] = a.kc.v.f16_lb[0][t]; vh0[t] = a.kc.v.f16_hb[0][t];
       vl1[t] = a.kc.v.f16_lb[1][t]; vh1[t] = a.kc.v.f16_hb[1][t];
     }
-    int waited = 0, staged = min(n, 2);
     for (int i = 0; i < n; ++i) {
       const int buf = i & 1;
       bool ok = pf_wait(&bars[PB_REC + buf], (i >> 1) & 1, abort, a.v.status);
-      if (ok) waited = i + 1;
       ok = ok && pf_wait(&bars[PB_KVFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status);  // V^T buffer
       ok = ok && (i == 0 || pf_wait(&bars[PB_KFREE], (i - 1) & 1, abort, a.v.status));    // K: S of step i - 1 done
-      if (!wg_all(ok, 1)) break;
+      if (!wg_all(ok, 1, 128)) break;
       const uint8_t* recb = smem + SM::rec + buf * 2 * TB;
       {  // K: coordinates 64 half .. 64 half + 63 of key `key`, eight per 16-byte core-matrix row
         const uint8_t* kr = recb + (key >> 5) * TB + (key & 31) * k_rec_bytes(KB);
@@ -413,15 +416,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           const uint8_t* vb = recb + (v16 >> 1) * TB + tr_v(KB) + (v16 & 1) * v_blk_bytes(VB);
           uint32_t s[4];
 #pragma unroll
-          for (int tq = 0; tq < 4; ++tq) {
-            const uint32_t* ch =
-                reinterpret_cast<const uint32_t*>(vb + 2 * chunk_bytes(VB) * (4 * g + tq) + hh * chunk_bytes(VB));
-            uint32_t wd[VB], sel[4];
-#pragma unroll
-            for (int t = 0; t < VB; ++t) wd[t] = ch[t];
-            chunk_selectors<VB>(wd, sel);
-            s[tq] = w == 0 ? sel[0] : w == 1 ? sel[1] : w == 2 ? sel[2] : sel[3];
-          }
+          for (int tq = 0; tq < 4; ++tq)
+            s[tq] = chunk_selector<VB>(
+                reinterpret_cast<const uint32_t*>(vb + 2 * chunk_bytes(VB) * (4 * g + tq) + hh * chunk_bytes(VB)), w);
           const uint32_t sA = prmt(s[0], s[1], sl0), sB = prmt(s[2], s[3], sl0);  // tokens 0-3, 4-7
           const uint32_t sC = prmt(s[0], s[1], sl1), sD = prmt(s[2], s[3], sl1);  // tokens 8-11, 12-15
           const int off = (d >> 3) * 1024 + (2 * v16) * 128 + (d & 7) * 16;
@@ -442,18 +439,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       } else if (e < 66) {
         s_mkv[2 * buf + (e - 64)] = s_mrec[2 * buf + (e - 64)];
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tiles, and the record reads, before the async proxy
       mbar_arrive(&bars[PB_KVFULL + buf]);
-      named_barrier_sync(1, 128);  // every expansion thread is done with this record buffer
-      if (e == 0 && i + 2 < n) {
-        pf_stage(a, b, kvh, s_lo + i + 2, kv_end, smem + SM::rec + buf * 2 * TB, s_mrec + 2 * buf,
-                 &bars[PB_REC + buf], TB);
-        ++staged;
-      }
+      mbar_arrive(&bars[PB_RECFREE + buf]);
     }
-    // leave no bulk copy in flight (only after a timed-out wait can one be pending)
-    if (e == 0)
-      for (; waited < staged; ++waited) mbar_wait(&bars[PB_REC + (waited & 1)], (waited >> 1) & 1, nullptr);
+  } else if (warp == 13) {
+    // ==== loads: the records of step i go into buffer i % 2 once the expansion warps have read
+    // the records of step i - 2 (steps 0 and 1 were staged before the query rotation)
+    if (lane == 0) {
+      int i = 2;
+      for (; i < n; ++i) {
+        const int buf = i & 1;
+        if (!pf_wait(&bars[PB_RECFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) break;
+        pf_stage(a, b, kvh, s_lo + i, kv_end, smem + SM::rec + buf * 2 * TB, s_mrec + 2 * buf, &bars[PB_REC + buf], TB);
+      }
+      // leave no bulk copy in flight (only after a timed-out wait can one be pending)
+      for (int j = max(0, i - 2); j < i && j < n; ++j) mbar_wait(&bars[PB_REC + (j & 1)], (j >> 1) & 1, nullptr);
+    }
   } else if (lane == 0) {
     // ==== MMA issue: S_{i+1} = Q K_{i+1}^T ahead of O_i^T = V_i^T P_i'^T
     const uint32_t idS = umma_idesc_f16(128, PF_BN), idO = umma_idesc_f16(128, 128);
