@@ -26,7 +26,8 @@
 // codes of step i + 1 while warps 0-7 take the softmax of step i (two warps per row quarter of
 // tensor memory: one per half of the keys, and per half of the rows when folding the output)
 // and the tensor cores compute S of step i + 1 and O of step i; one thread of warp 12 issues
-// the MMAs and one of warp 13 stages the tile records with bulk copies.  Splits of the key
+// the score MMAs as soon as a step's K is expanded, one of warp 14 the output MMAs as soon as
+// its P' is written, and one of warp 13 stages the tile records with bulk copies.  Splits of the key
 // range leave (m, l, O) partials that a second kernel merges, normalises and rotates back (R^T).
 #pragma once
 #include <algorithm>
@@ -38,7 +39,7 @@ namespace iq {
 
 constexpr int PF_ROWS = 128;     // query rows (token, head) per CTA: the MMA's M
 constexpr int PF_BN = 64;        // keys per step (two tile records)
-constexpr int PF_THREADS = 448;  // warps 0-7 softmax and output, 8-11 code expansion, 12 MMA issue, 13 loads
+constexpr int PF_THREADS = 480;  // warps 0-7 softmax and output, 8-11 code expansion, 12 and 14 MMA issue, 13 loads
 constexpr int PF_TMEM_COLS = 512;
 constexpr int PF_S_COL = 0;      // scores of buffer b: columns [64 b, 64 b + 64)
 constexpr int PF_O_COL = 128;    // output tile of buffer b: columns [128 + 128 b, 256 + 128 b)
@@ -79,11 +80,14 @@ struct PfSmem {
   static_assert(bytes <= 232448, "one CTA's shared memory on sm_100");
 };
 
-// mbarriers: records staged [buf]; K and V^T expanded [buf]; V^T free again [buf]; scores ready
-// [buf]; scores read [buf]; output tile ready [buf]; output tile read [buf]; P' written; K read
-// (single buffer); the last MMAs done; records read [buf].
-enum { PB_REC = 0, PB_KVFULL = 2, PB_KVFREE = 4, PB_SFULL = 6, PB_SFREE = 8, PB_OFULL = 10, PB_OFREE = 12,
-       PB_PFULL = 14, PB_KFREE = 15, PB_DRAIN = 16, PB_RECFREE = 17, PB_COUNT = 19 };
+// mbarriers, by step parity [buf] where marked: records staged [buf]; K, K norms and masks
+// expanded [buf]; V^T and V norms expanded [buf]; V^T free again [buf]; scores ready [buf];
+// scores read [buf]; output tile ready [buf]; output tile read [buf]; P' written; K read
+// (single buffer); the score MMAs done; the output MMAs done; records read [buf].
+enum { PB_REC = 0, PB_KFULL = 2, PB_VFULL = 4, PB_VFREE = 6, PB_SFULL = 8, PB_SFREE = 10, PB_OFULL = 12,
+       PB_OFREE = 14, PB_PFULL = 16, PB_KFREE = 17, PB_DRAIN_S = 18, PB_DRAIN_O = 19, PB_RECFREE = 20,
+       PB_COUNT = 22 };
+static_assert(PB_COUNT <= 24, "mbarrier slots of PfSmem");
 
 // Bounded wait on an mbarrier phase that also gives up once another thread has given up (the
 // abort flag); a timeout flags IQ_DEVERR_TIMEOUT.
@@ -175,10 +179,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
 
   if (tid == 0) {
     for (int i = 0; i < PB_COUNT; ++i) {
-      const bool by_threads = (i >= PB_KVFULL && i < PB_KVFULL + 2) || (i >= PB_RECFREE && i < PB_RECFREE + 2) ||
-                              (i >= PB_OFREE && i < PB_OFREE + 2) || i == PB_PFULL;
+      const bool by_expansion = (i >= PB_KFULL && i < PB_VFULL + 2) || (i >= PB_RECFREE && i < PB_RECFREE + 2);
       const bool by_softmax = (i >= PB_SFREE && i < PB_SFREE + 2) || (i >= PB_OFREE && i < PB_OFREE + 2) || i == PB_PFULL;
-      mbar_init(&bars[i], i < PB_REC + 2 ? 2 : by_softmax ? 256 : by_threads ? 128 : 1);
+      mbar_init(&bars[i], i < PB_REC + 2 ? 2 : by_softmax ? 256 : by_expansion ? 128 : 1);
     }
     mbar_fence_init();
     *abort = 0;
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       // the step's scores, and its norms and masks (written by the expansion warps: their own
       // barrier orders them before these reads; it has completed before the scores can)
       ok = pf_wait(&bars[PB_SFULL + buf], (i >> 1) & 1, abort, a.v.status);
-      ok = wg_all(ok && pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status), 2, 256);
+      ok = wg_all(ok && pf_wait(&bars[PB_KFULL + buf], (i >> 1) & 1, abort, a.v.status), 2, 256);
       if (!ok) break;
       tc_fence_after();
       const int kb = PF_BN * (s_lo + i) + 32 * kh;  // position of this thread's first key
@@ -307,8 +310,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       tc_fence_before();
       mbar_arrive(&bars[PB_SFREE + buf]);  // the scores of this buffer are read
       s_red[128 * kh + r] = mx;
-      // the P buffer is free once the previous step's P.V is done (this also publishes s_red)
-      ok = wg_all(i == 0 || pf_wait(&bars[PB_OFULL + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort, a.v.status), 2, 256);
+      // the P buffer is free once the previous step's P.V is done; the V norms are in once V^T is
+      // (this barrier also publishes s_red)
+      ok = i == 0 || pf_wait(&bars[PB_OFULL + ((i - 1) & 1)], ((i - 1) >> 1) & 1, abort, a.v.status);
+      ok = wg_all(ok && pf_wait(&bars[PB_VFULL + buf], (i >> 1) & 1, abort, a.v.status), 2, 256);
       if (!ok) break;
       const float m_new = fmaxf(m, fmaxf(s_red[r], s_red[128 + r]));
       const float alpha = (m == -CUDART_INF_F) ? 0.f : fast_exp2(m - m_new);
@@ -379,9 +384,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
     }
     for (int i = 0; i < n; ++i) {
       const int buf = i & 1;
+      // K (single buffer: the score MMAs of step i - 1 are done), its norms and masks (their
+      // buffer: the softmax of step i - 2 has read them)
       bool ok = pf_wait(&bars[PB_REC + buf], (i >> 1) & 1, abort, a.v.status);
-      ok = ok && pf_wait(&bars[PB_KVFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status);  // V^T buffer
-      ok = ok && (i == 0 || pf_wait(&bars[PB_KFREE], (i - 1) & 1, abort, a.v.status));    // K: S of step i - 1 done
+      ok = ok && (i == 0 || pf_wait(&bars[PB_KFREE], (i - 1) & 1, abort, a.v.status));
+      ok = ok && pf_wait(&bars[PB_SFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status);
       if (!wg_all(ok, 1, 128)) break;
       const uint8_t* recb = smem + SM::rec + buf * 2 * TB;
       {  // K: coordinates 64 half .. 64 half + 63 of key `key`, eight per 16-byte core-matrix row
@@ -404,6 +411,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           }
         }
       }
+      if (e < 64) {  // the step's K norms and token masks
+        s_nk[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(recb + (e >> 5) * TB + tr_kn(KB, VB))[e & 31]);
+      } else if (e < 66) {
+        s_mkv[2 * buf + (e - 64)] = s_mrec[2 * buf + (e - 64)];
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bars[PB_KFULL + buf]);
+      // V^T and the V norms (buffer buf: the output MMAs of step i - 2 are done)
+      if (!wg_all(pf_wait(&bars[PB_VFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status), 1, 128)) break;
       {  // V^T: coordinate d of the 64 keys.  Coordinate d = 32 w + 16 e2 + 8 hh + g of the
          // block's tokens u sits in chunk (g, tq = (u mod 8) / 2, hh), selector word w, nibble
          // m + 4 e2 (m = 2 (u / 8) + u mod 2): byte 2 e2 of that word holds tokens 2 tq, 2 tq + 1,
@@ -432,15 +448,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           *reinterpret_cast<uint4*>(vhi + 16384 + off + 128) = make_uint4(lC.x, lC.y, lD.x, lD.y);
         }
       }
-      if (e < 64) {  // the step's norms
-        const uint8_t* tr = recb + (e >> 5) * TB;
-        s_nk[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(tr + tr_kn(KB, VB))[e & 31]);
-        s_nv[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(tr + tr_vn(KB, VB))[e & 31]);
-      } else if (e < 66) {
-        s_mkv[2 * buf + (e - 64)] = s_mrec[2 * buf + (e - 64)];
-      }
+      if (e < 64)
+        s_nv[64 * buf + e] = __half2float(reinterpret_cast<const __half*>(recb + (e >> 5) * TB + tr_vn(KB, VB))[e & 31]);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the tiles, and the record reads, before the async proxy
-      mbar_arrive(&bars[PB_KVFULL + buf]);
+      mbar_arrive(&bars[PB_VFULL + buf]);
       mbar_arrive(&bars[PB_RECFREE + buf]);
     }
   } else if (warp == 13) {
@@ -456,16 +467,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       // leave no bulk copy in flight (only after a timed-out wait can one be pending)
       for (int j = max(0, i - 2); j < i && j < n; ++j) mbar_wait(&bars[PB_REC + (j & 1)], (j >> 1) & 1, nullptr);
     }
-  } else if (lane == 0) {
-    // ==== MMA issue: S_{i+1} = Q K_{i+1}^T ahead of O_i^T = V_i^T P_i'^T
-    const uint32_t idS = umma_idesc_f16(128, PF_BN), idO = umma_idesc_f16(128, 128);
-    const uint32_t qh = smem_addr(smem + SM::q_hi), ql = smem_addr(smem + SM::q_lo), pa = smem_addr(smem + SM::p);
-    auto issue_s = [&](int i) {
+  } else if (warp == 12 && lane == 0) {
+    // ==== score MMAs: S_i = Q K_i^T (hi.hi, lo.hi, hi.lo) once K_i is expanded and buffer i % 2 read
+    const uint32_t idS = umma_idesc_f16(128, PF_BN);
+    const uint32_t qh = smem_addr(smem + SM::q_hi), ql = smem_addr(smem + SM::q_lo);
+    const uint32_t kh = smem_addr(smem + SM::k0), kl = kh + 16384;
+    for (int i = 0; i < n; ++i) {
       const int buf = i & 1;
-      if (!pf_wait(&bars[PB_KVFULL + buf], (i >> 1) & 1, abort, a.v.status)) return false;
-      if (!pf_wait(&bars[PB_SFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) return false;
+      if (!pf_wait(&bars[PB_KFULL + buf], (i >> 1) & 1, abort, a.v.status)) break;
+      if (!pf_wait(&bars[PB_SFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) break;
       tc_fence_after();
-      const uint32_t kh = smem_addr(smem + SM::k0), kl = kh + 16384;
       const uint32_t dst = tmem + PF_S_COL + 64 * buf;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
@@ -478,12 +489,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
         umma_f16(dst, umma_sdesc(qh + 256 * ks, 128, 2048), umma_sdesc(kl + 256 * ks, 128, 2048), idS, 1);
       umma_commit(&bars[PB_SFULL + buf]);
       umma_commit(&bars[PB_KFREE]);
-      return true;
-    };
-    auto issue_o = [&](int i) {
+    }
+    umma_commit(&bars[PB_DRAIN_S]);  // every MMA issued is complete before tensor memory is released
+    mbar_wait(&bars[PB_DRAIN_S], 0, nullptr);
+  } else if (warp == 14 && lane == 0) {
+    // ==== output MMAs: O_i^T = V_i^T P_i'^T (V hi.P hi, V lo.P hi, V hi.P lo) once P_i' is written
+    const uint32_t idO = umma_idesc_f16(128, 128);
+    const uint32_t pa = smem_addr(smem + SM::p);
+    for (int i = 0; i < n; ++i) {
       const int buf = i & 1;
-      if (!pf_wait(&bars[PB_PFULL], i & 1, abort, a.v.status)) return false;
-      if (!pf_wait(&bars[PB_OFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) return false;
+      if (!pf_wait(&bars[PB_VFULL + buf], (i >> 1) & 1, abort, a.v.status)) break;
+      if (!pf_wait(&bars[PB_PFULL], i & 1, abort, a.v.status)) break;
+      if (!pf_wait(&bars[PB_OFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) break;
       tc_fence_after();
       const uint32_t vh = smem_addr(smem + SM::vt0 + buf * 32768), vl = vh + 16384;
       const uint32_t dst = tmem + PF_O_COL + 128 * buf;
@@ -497,17 +514,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       for (int ks = 0; ks < PF_BN / 16; ++ks)
         umma_f16(dst, umma_sdesc(vh + 256 * ks, 128, 1024), umma_sdesc(pa + 16384 + 256 * ks, 128, 1024), idO, 1);
       umma_commit(&bars[PB_OFULL + buf]);
-      umma_commit(&bars[PB_KVFREE + buf]);
-      return true;
-    };
-    bool ok = issue_s(0);
-    for (int i = 0; ok && i < n; ++i) {
-      if (i + 1 < n) ok = issue_s(i + 1);
-      if (ok) ok = issue_o(i);
+      umma_commit(&bars[PB_VFREE + buf]);
     }
-    // every MMA issued is complete before tensor memory is released
-    umma_commit(&bars[PB_DRAIN]);
-    mbar_wait(&bars[PB_DRAIN], 0, nullptr);
+    umma_commit(&bars[PB_DRAIN_O]);
+    mbar_wait(&bars[PB_DRAIN_O], 0, nullptr);
   }
   tc_fence_before();
   __syncthreads();
