@@ -36,13 +36,13 @@ BYTES_PER_VECTOR_ENCODE = 306  # 256 B fp16 in + 48 B codes + 2 B norm out
 DECODE_SOURCES = ["rotated_bit_kv_iq_b200/csrc/iq_decode_impl.cuh", "rotated_bit_kv_iq_b200/csrc/iq_decode.cu",
                   "rotated_bit_kv_iq_b200/csrc/iq_decode_k3v3.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
                   "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"]
-DECODE_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "fe4804efa0cd8b7d039f42f37d3fdf723b7ab34851666dabbc5f3b539b001be6", "bytes": 13240320}
-SERVING_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "fe4804efa0cd8b7d039f42f37d3fdf723b7ab34851666dabbc5f3b539b001be6", "bytes": 235545600 + 4383488}
+DECODE_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "87e42d60ae292aa63bbfb37815960c51c4f3f57b19d69ce46d32365e6118029b", "bytes": 13241600}
+SERVING_TRAFFIC = {"sources": DECODE_SOURCES, "sha256": "87e42d60ae292aa63bbfb37815960c51c4f3f57b19d69ce46d32365e6118029b", "bytes": 235573248 + 4002816}
 # DRAM bytes of one encode_kernel launch of the ingest layer (one-pass capture; the records still
 # in L2 at kernel end are not counted as written)
 ENCODE_SOURCES = ["rotated_bit_kv_iq_b200/csrc/iq_encode.cu", "rotated_bit_kv_iq_b200/csrc/iq_device.cuh",
                   "rotated_bit_kv_iq_b200/csrc/iq_internal.h", "include/iq.h"]
-ENCODE_TRAFFIC = {"sources": ENCODE_SOURCES, "sha256": "c2bb32722db638bf75dd6bc8f0c3e33b77a5613472dbffa66eb86a101560aad1", "bytes": 134294528 + 13356544}
+ENCODE_TRAFFIC = {"sources": ENCODE_SOURCES, "sha256": "021d3cb4d7e857e3015f9c1c10248d44a7fc18154f83d14de9fcfc4802b4330a", "bytes": 134293248 + 13251840}
 
 
 def kernel_source_hash(paths):
