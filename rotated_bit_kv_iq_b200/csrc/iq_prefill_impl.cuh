@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       if (qpos - kb < 31) vmask &= qpos < kb ? 0u : (2u << (qpos - kb)) - 1u;  // causal: keys <= qpos
       const float* nkb = s_nk + 64 * buf + 32 * kh;
       const float* nvb = s_nv + 64 * buf + 32 * kh;
+      const bool full = __all_sync(0xffffffffu, vmask == 0xFFFFFFFFu);
       float sv[32];
       float mx = -CUDART_INF_F;
       {
@@ -301,10 +302,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
         tmem_ld16(tlane + PF_S_COL + 64 * buf + 32 * kh, *reinterpret_cast<uint32_t(*)[16]>(v));
         tmem_ld16(tlane + PF_S_COL + 64 * buf + 32 * kh + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
         tmem_wait_ld();
+        if (full) {  // every key of the half valid for every row of the warp (below the diagonal)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          sv[k] = ((vmask >> k) & 1u) ? __uint_as_float(v[k]) * nkb[k] * qs : -CUDART_INF_F;
-          mx = fmaxf(mx, sv[k]);
+          for (int k = 0; k < 32; ++k) {
+            sv[k] = __uint_as_float(v[k]) * nkb[k] * qs;
+            mx = fmaxf(mx, sv[k]);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            sv[k] = ((vmask >> k) & 1u) ? __uint_as_float(v[k]) * nkb[k] * qs : -CUDART_INF_F;
+            mx = fmaxf(mx, sv[k]);
+          }
         }
       }
       tc_fence_before();
@@ -328,9 +337,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int k = 8 * c + j + e;
-            const float p = ((vmask >> k) & 1u) ? fast_exp2(sv[k] - m_new) : 0.f;
+            const bool kv = full || ((vmask >> k) & 1u);
+            const float p = kv ? fast_exp2(sv[k] - m_new) : 0.f;
             lsum += p;
-            pp[e] = ((vmask >> k) & 1u) ? p * nvb[k] : 0.f;
+            pp[e] = kv ? p * nvb[k] : 0.f;
           }
           const __half2 h2 = __floats2half2_rn(pp[0], pp[1]);
           const float2 hf = __half22float2(h2);
@@ -525,7 +535,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
   if (warp == 0) tmem_free(tmem, PF_TMEM_COLS);
 }
 
-// Merge of the splits of every group: warp per row; normalise; inverse rotation.
+// Merge of the splits of every group: CTA (group, block of 8 rows), warp per row, one pass over
+// the splits (online rescaling); normalise; inverse rotation.
 static __global__ void __launch_bounds__(DEC_THREADS) prefill_merge_kernel(PreArgs a) {
   pdl_launch_dependents();
   pdl_wait();
@@ -539,30 +550,30 @@ static __global__ void __launch_bounds__(DEC_THREADS) prefill_merge_kernel(PreAr
     reinterpret_cast<float4*>(sprm)[threadIdx.x] =
         reinterpret_cast<const float4*>(a.params_layer + (size_t)kvh * params_per_head(a.v.rot))[threadIdx.x];
   __syncthreads();
+  const int r = DEC_WARPS * blockIdx.y + warp;
+  const int tok = r / G, h = r % G;
+  if (r >= TQ * G || tok >= n_live) return;
+  float M = -CUDART_INF_F, L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < a.splits; ++s) {
+    const size_t prow = ((size_t)group * a.splits + s) * PF_ROWS + r;
+    const float2 ml = a.part_ml[prow];
+    const float4 v = reinterpret_cast<const float4*>(a.part_o + prow * D)[lane];
+    if (ml.x == -CUDART_INF_F) continue;
+    const float Mn = fmaxf(M, ml.x);
+    const float fo = (M == -CUDART_INF_F) ? 0.f : fast_exp2(M - Mn), wgt = fast_exp2(ml.x - Mn);
+    L = L * fo + ml.y * wgt;
+    o[0] = fmaf(v.x, wgt, o[0] * fo); o[1] = fmaf(v.y, wgt, o[1] * fo);
+    o[2] = fmaf(v.z, wgt, o[2] * fo); o[3] = fmaf(v.w, wgt, o[3] * fo);
+    M = Mn;
+  }
+  const float sc = L > 0.f ? 0.08838834764831845f / L : 0.f;  // V = n_v c / sqrt(128)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) o[i] *= sc;
   float Mp[4][4];
   variant_block_matrix(a.v.rot, sprm + lane * params_per_block(a.v.rot), Mp);
-  for (int r = warp; r < TQ * G; r += DEC_WARPS) {
-    const int tok = r / G, h = r % G;
-    if (tok >= n_live) continue;
-    float M = -CUDART_INF_F;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((size_t)group * a.splits + s) * PF_ROWS + r].x);
-    float L = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < a.splits; ++s) {
-      const size_t prow = ((size_t)group * a.splits + s) * PF_ROWS + r;
-      const float2 ml = a.part_ml[prow];
-      if (ml.x == -CUDART_INF_F) continue;
-      const float wgt = fast_exp2(ml.x - M);
-      L = fmaf(ml.y, wgt, L);
-      const float4 v = reinterpret_cast<const float4*>(a.part_o + prow * D)[lane];
-      o[0] = fmaf(v.x, wgt, o[0]); o[1] = fmaf(v.y, wgt, o[1]); o[2] = fmaf(v.z, wgt, o[2]); o[3] = fmaf(v.w, wgt, o[3]);
-    }
-    const float sc = L > 0.f ? 0.08838834764831845f / L : 0.f;  // V = n_v c / sqrt(128)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] *= sc;
-    warp_rotate_inverse(o, Mp, a.v.rot == ROT_ISO);
-    reinterpret_cast<float4*>(a.out + (((size_t)b * a.n_tok + tok0 + tok) * a.n_q_heads + (size_t)kvh * G + h) * D)[lane] =
-        make_float4(o[0], o[1], o[2], o[3]);
-  }
+  warp_rotate_inverse(o, Mp, a.v.rot == ROT_ISO);
+  reinterpret_cast<float4*>(a.out + (((size_t)b * a.n_tok + tok0 + tok) * a.n_q_heads + (size_t)kvh * G + h) * D)[lane] =
+      make_float4(o[0], o[1], o[2], o[3]);
 }
 
 // Splits per group: at most one CTA per SM in all, each with at least four steps.
@@ -611,7 +622,8 @@ int launch_prefill_kv(const LayerView& v, const void* q, int q_f32, int batch, i
   int e = (int)launch_pdl(prefill_kernel<KB, VB>, dim3(groups * a.splits), dim3(PF_THREADS), PfSmem<KB, VB>::bytes,
                           (cudaStream_t)stream, a);
   if (e) return e;
-  return (int)launch_pdl(prefill_merge_kernel, dim3(groups), dim3(DEC_THREADS), 0, (cudaStream_t)stream, a);
+  return (int)launch_pdl(prefill_merge_kernel, dim3(groups, PF_ROWS / DEC_WARPS), dim3(DEC_THREADS), 0,
+                         (cudaStream_t)stream, a);
 }
 
 }  // namespace iq
