@@ -50,7 +50,8 @@ def _prefill(cache, q, start, max_ctx, P):
 
 @pytest.mark.parametrize("kb,vb,rot,G", [(3, 3, "iso", 4), (3, 3, "iso", 8), (3, 3, "iso", 1), (4, 3, "iso", 8),
                                          (3, 2, "planar", 4), (3, 3, "quat", 2), (3, 3, "iso", 3),
-                                         (3, 3, "iso", 6)])
+                                         (3, 3, "iso", 6), (2, 2, "iso", 4), (4, 4, "iso", 5),
+                                         (4, 2, "quat", 7)])
 def test_prefill_ragged_chunks_match_oracle(kb, vb, rot, G):
     """Two sequences with different prefixes (0 and 300 tokens) and a 37-token chunk (a ragged last
     block of query tokens) over shuffled 64-token pages; every query token compared."""
