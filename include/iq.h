@@ -262,9 +262,12 @@ size_t iq_decode_deferred_workspace_size(int32_t batch, int32_t n_q_heads, int32
  * errors as for iq_decode_step, with the workspace of iq_decode_deferred_workspace_size.  Two
  * kernels: the prefix's attention (split partials, rotated forward into the packed basis), then
  * the fused step, which merges both before its single inverse rotation.  Ordering: the first
- * kernel waits for the kernel issued before the call before it reads anything; the second
- * starts once the first is past that wait, attends over the packed tail while the first is
- * still running, and waits for it only before merging its partials. */
+ * kernel may start while the kernel issued just before the call is still running; before
+ * waiting for it, it reads only len_dev and ctx_len_dev and starts the bulk loads of the fp16
+ * arrays' first tiles, so that kernel must not write len, ctx_len or the fp16 arrays (host
+ * copies and earlier kernels may).  q is read, and the workspace written, only after the wait.
+ * The second kernel starts once the first is past that wait, attends over the packed tail
+ * while the first is still running, and waits for it only before merging its partials. */
 iq_status iq_decode_step_deferred(const iq_cache* cache, int32_t layer, const iq_fp16_prefix* prefix, const void* q_dev,
                                   iq_dtype q_dtype, const void* k_new_dev, const void* v_new_dev, int32_t batch,
                                   int32_t n_q_heads, const int32_t* ctx_len_dev, int32_t max_ctx,
@@ -289,10 +292,12 @@ size_t iq_prefill_workspace_size(int32_t batch, int32_t n_tokens, int32_t n_kv_h
  *                  not exceed the per-sequence capacity.
  *   out_dev      : float32 [batch][n_tokens][n_q_heads][128].
  *   workspace_dev: at least iq_prefill_workspace_size(...) bytes, 256-byte aligned.
- * Each block of 8 query tokens shares every tile of packed K/V it loads (one warp per query
- * token, tensor-core tiles as in decode); the result equals iq_decode_attention of each query
- * token over its own causal context.  Two kernels (attention splits, then their merge with the
- * inverse rotation); they wait for the preceding kernel on the stream before reading anything. */
+ * Each CTA takes up to 128 query rows (floor(128 / G) tokens x the G query heads of one kv head)
+ * and expands every 64-token step of packed K/V it loads once for all of them
+ * (binary16 hi/lo operands on the tensor cores, fp32 accumulators); the result equals
+ * iq_decode_attention of each query token over its own causal context within the tolerance of
+ * that call.  Two kernels (attention splits, then their merge with the inverse rotation); they
+ * wait for the preceding kernel on the stream before reading anything. */
 iq_status iq_prefill_attention(const iq_cache* cache, int32_t layer, const void* q_dev, iq_dtype q_dtype, int32_t batch,
                                int32_t n_tokens, int32_t n_q_heads, const int32_t* start_pos_dev, int32_t max_ctx,
                                const float* params_dev, float* out_dev, void* workspace_dev, size_t workspace_bytes,
