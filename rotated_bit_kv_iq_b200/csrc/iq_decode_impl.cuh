@@ -66,12 +66,13 @@ struct DecSmem {
   static constexpr int qfrag = sl + DEC_WARPS * HMAX * 4;                 // uint32 [lane][QF_WORDS] query fragments
   static constexpr int kappa = qfrag + 32 * QF_WORDS * 4;                 // float [head] score scales
   static constexpr int sparams = kappa + HMAX * 4;                        // float [256] one head's parameters
-  static constexpr int flags = sparams + 256 * 4;                         // int [4]
-  static constexpr int valid = flags + 16;                                // uint32 [warp][slot] token masks
+  static constexpr int appbar = sparams + 256 * 4;                        // uint64: new token appended
+  static constexpr int valid = appbar + 16;                               // uint32 [warp][slot] token masks
   static constexpr int bars = valid + DEC_WARPS * NSLOT * 4;              // uint64 [warp][slot]
   static constexpr int cursors = bars + DEC_WARPS * NSLOT * 8;           // Cursor [warp]
   static constexpr int plan = cursors + DEC_WARPS * 48;  // int [batch+1] tile prefix, [batch] ctx, [batch] fp16 prefix
   static size_t bytes(int batch) { return (size_t)plan + 4 * (size_t)(3 * batch + 1); }
+  static_assert(appbar % 8 == 0 && bars % 8 == 0, "mbarriers are 8-byte aligned");
 };
 
 struct Workspace {
@@ -264,16 +265,24 @@ __device__ __forceinline__ void issue_tile(const LayerView& v, int b, int kvh, i
 // The new token of sequence b (position ctx-1): encode K and V into the cache (whole warp).
 // Inlined: as an out-of-line call its register saves cost more than the encoding itself.
 template <int KB, int VB>
-__device__ __forceinline__ void append_new_token(const DecArgs& a, int b, int kvh, int ctx) {
+// One side (0: K, 1: V) of the new token, by one warp; prm: the kv head's rotation parameters
+// (shared memory).  The vector and the block-table entry are requested together, the vector
+// through L2: the kernel may have started before the one that wrote k_new and v_new finished
+// (see decode_kernel).
+__device__ __forceinline__ void append_new_token(const DecArgs& a, int b, int kvh, int ctx, const float* prm,
+                                                 int side) {
   const int p = ctx - 1;
-  const int page = resolve_page(a.v, b, p);
-  if (page < 0) return;
   const int lane = threadIdx.x & 31;
+  const size_t off = ((size_t)b * a.v.n_kv_heads + kvh) * D + 4 * lane;
+  const uint2 raw = __ldcg(reinterpret_cast<const uint2*>((side ? a.v_new : a.k_new) + off));
+  const int page = resolve_page(a.v, b, p);
   float Mp[4][4];
-  variant_block_matrix(a.v.rot, block_params(a.params_layer, a.v.rot, kvh, lane), Mp);
-  const size_t off = ((size_t)b * a.v.n_kv_heads + kvh) * D;
-  warp_encode_vector<KB>(a.v, a.k_new + off, kvh, 0, page, p % a.v.page_size, Mp, a.kc.k);
-  warp_encode_vector<VB>(a.v, a.v_new + off, kvh, 1, page, p % a.v.page_size, Mp, a.kc.v);
+  variant_block_matrix(a.v.rot, prm + lane * params_per_block(a.v.rot), Mp);
+  if (page < 0) return;
+  if (side == 0)
+    warp_encode_loaded<KB>(a.v, raw, kvh, 0, page, p % a.v.page_size, Mp, a.kc.k);
+  else
+    warp_encode_loaded<VB>(a.v, raw, kvh, 1, page, p % a.v.page_size, Mp, a.kc.v);
 }
 
 // ------------------------------------------------------------------ per-tile compute
@@ -643,8 +652,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   uint8_t* ring = smem + DecSmem::ring + warp * NSLOT * SLOT_BYTES;
   uint32_t* valid = reinterpret_cast<uint32_t*>(smem + DecSmem::valid) + warp * NSLOT;
   uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + DecSmem::bars) + warp * NSLOT;
+  uint64_t* appbar = reinterpret_cast<uint64_t*>(smem + DecSmem::appbar);
   if (lane == 0) {
     for (int s = 0; s < NSLOT; ++s) mbar_init(&wbar[s], 1);
+    if (warp == 0) mbar_init(appbar, 2);  // the K and the V half of an append
     mbar_fence_init();
   }
   build_plan(a, pre);  // ends with __syncthreads (barrier inits visible)
@@ -656,7 +667,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
   const long long c1 = cta < n_cta ? cta_begin(cta + 1, T, n_cta) : 0;
 
   // ---- prefetch: the warp's first tiles (a tile holding this call's new token waits)
-  long long app_done = -1;  // first global tile of the group whose new token this warp has appended
+  // the segment whose new token is being appended (its first global tile), and the parity of
+  // that append's phase of appbar (one phase per segment holding a group's last tile)
+  long long app_gstart = -1;
+  uint32_t app_parity = 0;
   Cursor* curs = reinterpret_cast<Cursor*>(smem + DecSmem::cursors) + warp;
   Cursor fc;
   int pg = -1;  // lane 0: block-table entry of the cursor's tile
@@ -685,7 +699,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     while (!fc.done && k_fetch < k_done + NSLOT) {
       const int ctx = fc.s.ctx;
       // a tile holding this call's new token is loaded only after this warp has appended it
-      if (is_new_token_tile<FUSED>(fc.s, fc.i) && fc.s.gstart != app_done) break;
+      if (is_new_token_tile<FUSED>(fc.s, fc.i) &&
+          (fc.s.gstart != app_gstart || !__shfl_sync(0xffffffffu, mbar_test_wait(appbar, app_parity), 0)))
+        break;
       const int sl_i = k_fetch % NSLOT;
       if (lane == 0)
         issue_tile(a.v, fc.s.b, fc.s.kvh, fc.s.first + fc.i, ctx, fc.s.plo, pg, ring + sl_i * SLOT_BYTES, &valid[sl_i],
@@ -719,6 +735,19 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       const size_t row = ((size_t)s0.b * a.n_q_heads + (size_t)s0.kvh * a.g_real + (threadIdx.x >> 1)) * D;
       const char* p = a.q_f32 ? (const char*)((const float*)a.q + row) : (const char*)((const __half*)a.q + row);
       asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * (threadIdx.x & 1) * (a.q_f32 ? 2 : 1)));
+    }
+    // and the new token (K and V rows, two lines each) of the groups whose last tile this CTA
+    // holds: the segments of the run that end at their group's end (the first four)
+    if (warp == 1) {
+      long long x = c0;
+      for (int n = 0; x < c1 && n < 4; ++n) {
+        const Seg s = segment_at(a, pre, B, Hkv, x, c1);
+        if (s.hi == s.ntiles && lane < 4) {
+          const __half* src = ((lane & 2) ? a.v_new : a.k_new) + ((size_t)s.b * Hkv + s.kvh) * D;
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(src) + 128 * (lane & 1)));
+        }
+        x = s.gstart + s.hi;
+      }
     }
     // After an fp16 prefix's kernel (a.n_extra > 0) the wait moves to the final merge, the first
     // read of what that kernel writes (its partials): it starts only once it has waited for the
@@ -757,14 +786,17 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
     else if (P4 && warp < HMAX && lane == 0)
       kappa[warp] = 0.f;  // rows of lo terms: their lanes' scores are not used
     __syncthreads();
-    // the new token is appended by the warp that loads its tile, before its tile loop (after the
-    // wait and outside the CTA-wide barriers, so only that warp spends the time; and outside the
-    // loop, whose registers it would otherwise crowd)
-    if (FUSED && seg.hi == seg.ntiles && (seg.ntiles - 1 - seg.lo) % DEC_WARPS == warp) {
-      append_new_token<KB, VB>(a, seg.b, seg.kvh, seg.ctx);
-      __syncwarp();
-      fence_proxy_async_global();  // the appended records before the bulk reads of them
-      app_done = seg.gstart;
+    // The new token is appended before the tile loops, K by the last warp and V by the one before
+    // it: the round robin gives those warps the fewest tiles of the segment.  The warp whose tile
+    // holds the token (normally its last tile) copies it only once both have arrived on appbar.
+    if (FUSED && seg.hi == seg.ntiles) {
+      if (warp >= DEC_WARPS - 2) {
+        append_new_token<KB, VB>(a, seg.b, seg.kvh, seg.ctx, sprm, warp == DEC_WARPS - 1 ? 0 : 1);
+        __syncwarp();
+        fence_proxy_async_global();  // the appended records before the bulk reads of them
+        if (lane == 0) mbar_arrive(appbar);
+      }
+      app_gstart = seg.gstart;
     }
     const float kap = kappa[lane >> 2];
     WarpState st;
@@ -777,6 +809,15 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
 
     for (int i = seg.lo + warp; i < seg.hi; i += DEC_WARPS) {
       top_up();  // issues this tile if it is not in flight yet, and refills the ring
+      if (FUSED && k_fetch == k_done && !aborted) {
+        // not issued: the tile holds the new token, whose append is still running
+        if (__all_sync(0xffffffffu, mbar_wait(appbar, app_parity, a.v.status))) {
+          fence_proxy_async_global();
+          top_up();
+        } else {
+          aborted = true;
+        }
+      }
       const int sl_i = k_done % NSLOT;
       if (!aborted) {
         const bool landed = __all_sync(0xffffffffu, mbar_wait(&wbar[sl_i], (k_done / NSLOT) & 1, a.v.status));
@@ -886,6 +927,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) decode_kernel(DecArgs a) {
       // reduction: no value comes back, so nothing waits for the counter itself)
       asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&a.ws.counters[gid]) : "memory");
     }
+    if (FUSED && seg.hi == seg.ntiles) app_parity ^= 1;  // that append's phase is over
     x = seg.gstart + seg.hi;
   }
 

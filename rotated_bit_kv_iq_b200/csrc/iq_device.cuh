@@ -343,6 +343,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the same (this thread's view).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -415,12 +425,11 @@ __device__ __forceinline__ void scaled_thresholds(const SideConsts& sc, float n,
 // (side 1, width VB) record of kv head `head` at (page, slot); lane l owns coordinates
 // 4l..4l+3 (one rotation block).  The WHT stages (ROT_ISO) run as shuffles; the lane's block
 // matrix is passed in.  A V block gets only this token's bits (see below).
+// raw: this lane's four fp16 coordinates 4 lane .. 4 lane + 3 (see warp_encode_vector).
 template <int BITS>
-__device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __half* __restrict__ src, int head,
-                                                   int side, int page, int slot, const float Mp[4][4],
-                                                   const SideConsts& sc) {
+__device__ __forceinline__ void warp_encode_loaded(const LayerView& v, uint2 raw, int head, int side, int page,
+                                                   int slot, const float Mp[4][4], const SideConsts& sc) {
   const int lane = threadIdx.x & 31;
-  const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(src + 4 * lane));  // through L2 (see decode_kernel)
   const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
   const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
   float x[4] = {f0.x, f0.y, f1.x, f1.y};
@@ -490,6 +499,13 @@ __device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __h
     }
   }
   if (lane == 0) *norm_slot(v, page, head, slot, side) = __half_as_ushort(__float2half_rn(fminf(n, 65504.f)));
+}
+template <int BITS>
+__device__ __forceinline__ void warp_encode_vector(const LayerView& v, const __half* __restrict__ src, int head,
+                                                   int side, int page, int slot, const float Mp[4][4],
+                                                   const SideConsts& sc) {
+  const uint2 raw = __ldcg(reinterpret_cast<const uint2*>(src + 4 * (threadIdx.x & 31)));
+  warp_encode_loaded<BITS>(v, raw, head, side, page, slot, Mp, sc);
 }
 
 }  // namespace iq
