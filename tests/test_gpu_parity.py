@@ -433,6 +433,26 @@ def test_decode_step_matches_oracle(G):
     record_parity(f"decode step, ragged paged (G={G})", **rec)
 
 
+@pytest.mark.parametrize("G", [4, 8])
+def test_decode_step_many_short_sequences(G):
+    """Fused step over 120 short sequences (1..200 tokens, 2 kv heads): a CTA's run crosses
+    several groups, so one CTA appends the new tokens of several groups in turn and hands each
+    token's tile from the appending warps to the loading warp again.  Every output row and
+    every appended record is compared with the oracle."""
+    ctx = [int(x) for x in inputs.context_lengths(inputs.DATA_SEED + G, 120, 1, 200)]
+    cache, P, cases = _step_case(G, ctx, ps=64, maxp=4)
+    q, knew, vnew, refs = cases[0]
+    o = _run_step(cache, 0, q, knew, vnew, ctx, 200, P)
+    rec = {"max_rel_err": 0.0}
+    for b, T in enumerate(ctx):
+        err = max_rel_err(o[b], refs[b][0])
+        rec["max_rel_err"] = max(rec["max_rel_err"], err)
+        assert err < TOL, (b, T, err)
+        _check_appended(cache, 0, b, T - 1, knew[b], vnew[b], P[0], rec)
+    assert cache.status.item() == 0
+    record_parity(f"decode step, 120 short sequences (G={G})", **rec)
+
+
 def _oracle_fill_contiguous(cache, layer, P_layer, T_cached, seed, heads):
     """Oracle encodings of tokens 0..T_cached-1 of each kv head uploaded to page 0 (a contiguous
     cache); returns the codes and norms per head, for the oracle's attention."""
