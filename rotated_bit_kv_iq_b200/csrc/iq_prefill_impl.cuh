@@ -59,7 +59,8 @@ struct PreArgs {
   KernelConsts kc;
 };
 
-// Shared memory (bytes).  Operand tiles use the no-swizzle K-major layout of iq_tcgen05.cuh.
+// Shared memory (bytes, from a 1024-byte aligned base).  Operand tiles use the 128-byte swizzled
+// K-major layout of iq_tcgen05.cuh.
 template <int KB, int VB>
 struct PfSmem {
   static constexpr int TB = tile_bytes(KB, VB);
@@ -76,7 +77,7 @@ struct PfSmem {
   static constexpr int red = alpha + 128 * 4;   // float [2][128] per key half: row maxima, at the end sums
   static constexpr int bars = red + 256 * 4;    // uint64 [PB_COUNT]
   static constexpr int misc = bars + 24 * 8;    // uint32 tensor-memory base, int abort flag
-  static constexpr int bytes = misc + 16;
+  static constexpr int bytes = misc + 16 + 1024;  // + the alignment of the base
   static_assert(bytes <= 232448, "one CTA's shared memory on sm_100");
 };
 
@@ -145,7 +146,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
   constexpr int TB = SM::TB;
   pdl_launch_dependents();
   pdl_wait();
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* const smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::bars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::misc);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + SM::misc + 4);
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       hw[i] = *reinterpret_cast<const uint32_t*>(&hi);
       lw[i] = *reinterpret_cast<const uint32_t*>(&lo);
     }
-    const int off = (r >> 3) * 2048 + (lane >> 1) * 128 + (r & 7) * 16 + (lane & 1) * 8;
+    const int off = umma_sw128_off(r, 4 * (lane & ~1), PF_ROWS) + (lane & 1) * 8;  // coordinates 4 lane ..
     *reinterpret_cast<uint2*>(smem + SM::q_hi + off) = make_uint2(hw[0], hw[1]);
     *reinterpret_cast<uint2*>(smem + SM::q_lo + off) = make_uint2(lw[0], lw[1]);
     // log2-domain score of a key = S n_k log2(e) / (128 sigma): q' c / sqrt(128) is the rotated
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       const float m_new = fmaxf(m, fmaxf(s_red[r], s_red[128 + r]));
       const float alpha = (m == -CUDART_INF_F) ? 0.f : fast_exp2(m - m_new);
       float lsum = 0.f;
-      uint8_t* prow = smem + SM::p + (r >> 3) * 1024 + (4 * kh) * 128 + (r & 7) * 16;
+      uint8_t* prow = smem + SM::p;  // row r, keys 32 kh .. 32 kh + 31
 #pragma unroll
       for (int c = 0; c < 4; ++c) {  // keys 8 c .. 8 c + 7 of this half: one 16-byte row of a core matrix
         uint32_t ph[4], pl[4];
@@ -348,8 +350,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           ph[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
           pl[j >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
         }
-        *reinterpret_cast<uint4*>(prow + 128 * c) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-        *reinterpret_cast<uint4*>(prow + 16384 + 128 * c) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+        const int off = umma_sw128_off(r, 32 * kh + 8 * c, PF_ROWS);
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(prow + 16384 + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bars[PB_PFULL]);
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
           for (int wq = 0; wq < 4; ++wq) {
             const uint2 a0 = lut_f16x4<KB>(kl0, kh0, sel[wq]), a1 = lut_f16x4<KB>(kl0, kh0, sel[wq] >> 16);
             const uint2 b0 = lut_f16x4<KB>(kl1, kh1, sel[wq]), b1 = lut_f16x4<KB>(kl1, kh1, sel[wq] >> 16);
-            const int off = (key >> 3) * 2048 + (4 * c + wq) * 128 + (key & 7) * 16;
+            const int off = umma_sw128_off(key, 8 * (4 * c + wq), PF_BN);
             *reinterpret_cast<uint4*>(khi + off) = make_uint4(a0.x, a0.y, a1.x, a1.y);
             *reinterpret_cast<uint4*>(khi + 16384 + off) = make_uint4(b0.x, b0.y, b1.x, b1.y);
           }
@@ -447,15 +450,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
                 reinterpret_cast<const uint32_t*>(vb + 2 * chunk_bytes(VB) * (4 * g + tq) + hh * chunk_bytes(VB)), w);
           const uint32_t sA = prmt(s[0], s[1], sl0), sB = prmt(s[2], s[3], sl0);  // tokens 0-3, 4-7
           const uint32_t sC = prmt(s[0], s[1], sl1), sD = prmt(s[2], s[3], sl1);  // tokens 8-11, 12-15
-          const int off = (d >> 3) * 1024 + (2 * v16) * 128 + (d & 7) * 16;
+          const int off0 = umma_sw128_off(d, 16 * v16, 128), off1 = umma_sw128_off(d, 16 * v16 + 8, 128);
           const uint2 hA = lut_f16x4<VB>(vl0, vh0, sA), hB = lut_f16x4<VB>(vl0, vh0, sB);
           const uint2 hC = lut_f16x4<VB>(vl0, vh0, sC), hD = lut_f16x4<VB>(vl0, vh0, sD);
-          *reinterpret_cast<uint4*>(vhi + off) = make_uint4(hA.x, hA.y, hB.x, hB.y);
-          *reinterpret_cast<uint4*>(vhi + off + 128) = make_uint4(hC.x, hC.y, hD.x, hD.y);
+          *reinterpret_cast<uint4*>(vhi + off0) = make_uint4(hA.x, hA.y, hB.x, hB.y);
+          *reinterpret_cast<uint4*>(vhi + off1) = make_uint4(hC.x, hC.y, hD.x, hD.y);
           const uint2 lA = lut_f16x4<VB>(vl1, vh1, sA), lB = lut_f16x4<VB>(vl1, vh1, sB);
           const uint2 lC = lut_f16x4<VB>(vl1, vh1, sC), lD = lut_f16x4<VB>(vl1, vh1, sD);
-          *reinterpret_cast<uint4*>(vhi + 16384 + off) = make_uint4(lA.x, lA.y, lB.x, lB.y);
-          *reinterpret_cast<uint4*>(vhi + 16384 + off + 128) = make_uint4(lC.x, lC.y, lD.x, lD.y);
+          *reinterpret_cast<uint4*>(vhi + 16384 + off0) = make_uint4(lA.x, lA.y, lB.x, lB.y);
+          *reinterpret_cast<uint4*>(vhi + 16384 + off1) = make_uint4(lC.x, lC.y, lD.x, lD.y);
         }
       }
       if (e < 64)
@@ -488,15 +491,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       if (!pf_wait(&bars[PB_SFREE + buf], ((i >> 1) & 1) ^ 1, abort, a.v.status)) break;
       tc_fence_after();
       const uint32_t dst = tmem + PF_S_COL + 64 * buf;
+      // k-step ks: K block ks / 4, 32 bytes per step inside it (128 query rows, 64 keys)
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        umma_f16(dst, umma_sdesc(qh + 256 * ks, 128, 2048), umma_sdesc(kh + 256 * ks, 128, 2048), idS, ks > 0);
+        umma_f16(dst, umma_sdesc_sw128(qh + (ks >> 2) * 16384 + (ks & 3) * 32),
+                 umma_sdesc_sw128(kh + (ks >> 2) * 8192 + (ks & 3) * 32), idS, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        umma_f16(dst, umma_sdesc(ql + 256 * ks, 128, 2048), umma_sdesc(kh + 256 * ks, 128, 2048), idS, 1);
+        umma_f16(dst, umma_sdesc_sw128(ql + (ks >> 2) * 16384 + (ks & 3) * 32),
+                 umma_sdesc_sw128(kh + (ks >> 2) * 8192 + (ks & 3) * 32), idS, 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        umma_f16(dst, umma_sdesc(qh + 256 * ks, 128, 2048), umma_sdesc(kl + 256 * ks, 128, 2048), idS, 1);
+        umma_f16(dst, umma_sdesc_sw128(qh + (ks >> 2) * 16384 + (ks & 3) * 32),
+                 umma_sdesc_sw128(kl + (ks >> 2) * 8192 + (ks & 3) * 32), idS, 1);
       umma_commit(&bars[PB_SFULL + buf]);
       umma_commit(&bars[PB_KFREE]);
     }
@@ -514,15 +521,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_kernel(PreArgs a) {
       tc_fence_after();
       const uint32_t vh = smem_addr(smem + SM::vt0 + buf * 32768), vl = vh + 16384;
       const uint32_t dst = tmem + PF_O_COL + 128 * buf;
+      // k-step ks: 32 bytes per step in the single K block (64 keys)
 #pragma unroll
       for (int ks = 0; ks < PF_BN / 16; ++ks)
-        umma_f16(dst, umma_sdesc(vh + 256 * ks, 128, 1024), umma_sdesc(pa + 256 * ks, 128, 1024), idO, ks > 0);
+        umma_f16(dst, umma_sdesc_sw128(vh + 32 * ks), umma_sdesc_sw128(pa + 32 * ks), idO, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < PF_BN / 16; ++ks)
-        umma_f16(dst, umma_sdesc(vl + 256 * ks, 128, 1024), umma_sdesc(pa + 256 * ks, 128, 1024), idO, 1);
+        umma_f16(dst, umma_sdesc_sw128(vl + 32 * ks), umma_sdesc_sw128(pa + 32 * ks), idO, 1);
 #pragma unroll
       for (int ks = 0; ks < PF_BN / 16; ++ks)
-        umma_f16(dst, umma_sdesc(vh + 256 * ks, 128, 1024), umma_sdesc(pa + 16384 + 256 * ks, 128, 1024), idO, 1);
+        umma_f16(dst, umma_sdesc_sw128(vh + 32 * ks), umma_sdesc_sw128(pa + 16384 + 32 * ks), idO, 1);
       umma_commit(&bars[PB_OFULL + buf]);
       umma_commit(&bars[PB_VFREE + buf]);
     }

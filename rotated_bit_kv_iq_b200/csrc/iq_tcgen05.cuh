@@ -2,11 +2,12 @@
 // shared-memory matrix and instruction descriptors of a kind::f16 MMA, the MMA itself, its
 // completion signal on an mbarrier, and tensor-memory loads.
 //
-// Operand layout used throughout (no swizzle): a K-major tile of R rows and K 16-bit elements is
-// stored as 8 x 16-byte core matrices, element (r, k) at
-//     (r / 8) * (K / 8) * 128 + (k / 8) * 128 + (r % 8) * 16 + (k % 8) * 2   bytes,
-// so the stride between K-adjacent core matrices (LBO) is 128 bytes and between 8-row groups
-// (SBO) K * 16 bytes; the MMA over elements 16 s .. 16 s + 15 of K starts at byte 256 s.
+// Operand layout (K-major, 128-byte swizzle): a tile of R rows and K 16-bit elements is stored
+// as K / 64 blocks of R rows x 128 bytes, element (r, k) at
+//     (k / 64) * R * 128 + r * 128 + ((((k / 8) % 8) ^ (r % 8)) * 16) + (k % 8) * 2   bytes
+// from a 1024-byte aligned base (the hardware applies the XOR on address bits 4-6 from bits
+// 7-9).  Groups of 8 rows are 1024 bytes apart (SBO); the MMA over elements 16 s .. 16 s + 15
+// starts at byte (s / 4) * R * 128 + (s % 4) * 32.
 #pragma once
 #include <cstdint>
 
@@ -14,11 +15,15 @@ namespace iq {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// Shared-memory matrix descriptor: start address, LBO and SBO in 16-byte units, descriptor
-// version 1, no swizzle.
-__device__ __forceinline__ uint64_t umma_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+// Shared-memory matrix descriptor of the layout above: start address (16-byte units), leading
+// offset 1 (unused by this layout), 8-row stride 1024 bytes, descriptor version 1, layout type
+// 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+// Byte offset of element (r, k) (k a multiple of 8: the start of a 16-byte chunk) in an R-row tile.
+__host__ __device__ constexpr int umma_sw128_off(int r, int k, int R) {
+  return (k >> 6) * R * 128 + r * 128 + ((((k >> 3) & 7) ^ (r & 7)) << 4);
 }
 
 // Instruction descriptor of kind::f16 with fp16 A and B (both K-major) and an fp32 accumulator.
