@@ -109,6 +109,17 @@ def test_deferred_step_matches_oracle(G, kb, vb, rot):
     assert max(max_rel_err(out2.cpu().numpy()[b], refs[b]) for b in range(len(ctxs))) < TOL
 
 
+def test_deferred_flags_out_of_range_prefix_length():
+    """A prefix length equal to the context length (it must be below: the step's new token is
+    packed) or far above the arrays' capacity is clamped and flagged with IQ_DEVERR_CTX; the
+    guard bands stay intact and every output is finite."""
+    lens, ctxs = [5, 64], [40, 100]
+    cache, P, q, k16, v16, knew, vnew, refs, max_ctx = _case(4, lens, ctxs)
+    o, ws = _run(cache, P, q, k16, v16, [40, 10**6], knew, vnew, ctxs, max_ctx)
+    assert np.isfinite(o).all()
+    assert cache.status.item() & B.IQ_DEVERR_CTX
+
+
 def test_deferred_llama8b_layer_full():
     """The bench's deferred shape: one Llama-3.1-8B-shaped layer (32 q / 8 kv heads), an 8192-token
     fp16 prompt and 512 generated tokens packed (the step appends the last), every head compared."""
