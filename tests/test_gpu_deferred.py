@@ -88,7 +88,8 @@ def _run(cache, P, q, k16, v16, lens, knew, vnew, ctxs, max_ctx):
 
 
 @pytest.mark.parametrize("G,kb,vb,rot", [(4, 3, 3, "iso"), (8, 3, 3, "iso"), (8, 4, 3, "iso"), (4, 3, 2, "planar"),
-                                         (1, 3, 3, "quat"), (3, 3, 3, "iso"), (5, 3, 3, "iso"), (7, 3, 3, "iso")])
+                                         (1, 3, 3, "quat"), (3, 3, 3, "iso"), (5, 3, 3, "iso"), (7, 3, 3, "iso"),
+                                         (2, 3, 3, "iso"), (6, 3, 3, "iso")])
 def test_deferred_step_matches_oracle(G, kb, vb, rot):
     """Prefixes of 0, 5, 64 (a whole tile) and 300 tokens; contexts 1, 40, 100, 777; the positions
     of the packed pool below each prefix hold other tokens' codes."""
